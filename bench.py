@@ -1,0 +1,443 @@
+"""Benchmark of the TTT layer forward on B200: head-tokens/s (B x H x T / s).
+
+One step is one call of the layer forward (every stage of the hot path, fused in
+one kernel) over the whole workload, inputs resident in HBM.  Defaults: the
+TTT-Linear + LN + residual workload with B=16, H=32, d=64, T=8192, b=16 (bf16
+Q/K/V).  Under torchrun every rank runs its own batch shard of the same size
+(weak scaling, no collective on the data path); the step time is the max over
+ranks.  ``--impl reference`` times the fp64 CPU oracle instead, on a bounded
+sample of the same workload.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from test_sequence_modeling_b200 import inputs as I  # noqa: E402
+
+METRIC = "TTT layer fwd tokens/s (B×H×T/s) on 1 B200; % of roofline (HBM vs tensor)"
+UNIT = "head-tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ("test_sequence_modeling_b200/csrc",)
+
+
+# --- workload accounting --------------------------------------------------------
+
+def flops_per_head_token(cfg) -> float:
+    """Dense matmul FLOPs of the dual form per head-token (elementwise work not counted).
+    Linear: [K;Q] W (4d^2), K^T G (2d^2), tril(QK^T) (2bd) and its product with G (2bd).
+    MLP: 14 d h + 4 b (d + h)."""
+    d, b, h = cfg.d, cfg.b, cfg.hidden
+    if cfg.variant == "mlp":
+        return 14.0 * d * h + 4.0 * b * (d + h)
+    return 6.0 * d * d + 4.0 * b * d
+
+
+def bytes_per_launch(cfg, units=None) -> float:
+    """Algorithmic HBM bytes of one call: Q, K, V read once, eta read once, Z written
+    once, and each unit's initial state read and final state written once."""
+    units = cfg.units if units is None else units
+    qkv = 2 if cfg.dtype == "bf16" else 4
+    per_token = 3 * cfg.d * qkv + 4 + 4 * cfg.d
+    state = 4 * (2 * cfg.d * cfg.hidden if cfg.variant == "mlp" else cfg.d * cfg.d)
+    return units * (cfg.T * per_token + 2 * state)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for d in KERNEL_SOURCES:
+        full = os.path.join(ROOT, d)
+        for name in sorted(os.listdir(full)):
+            with open(os.path.join(full, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t[workload]
+        if e.get("kernel_source_sha") == kernel_source_sha():
+            return float(e["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return None
+
+
+# --- clocks ------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.out = []
+        self.gpu_id = gpu_id
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            text, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            text, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in text.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
+        loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_id_for(torch, device) -> str | None:
+    try:
+        uuid = str(torch.cuda.get_device_properties(device).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:  # noqa: BLE001
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        return vis.split(",")[0] if vis else None
+
+
+# --- reference arm and CPU baseline: the fp64 oracle on host cores -------------------
+
+def oracle_sample(cfg, units, T, nthreads):
+    """Run the oracle on `units` whole units truncated to T tokens; returns seconds."""
+    import oracle
+    sub = cfg.replace(T=T)
+    data = {"Q": [], "K": [], "V": [], "eta": []}
+    for bi, hi in units:
+        q, k, v, e = I.unit_inputs(cfg, bi, hi, T=T)
+        for n, a in zip(("Q", "K", "V", "eta"), (q, k, v, e)):
+            data[n].append(a.astype(np.float64))
+    Q, K, V = (np.stack(data[n])[:, None] for n in ("Q", "K", "V"))
+    eta = np.stack(data["eta"])[:, None]
+    # Each sampled unit runs as its own batch row with its head's parameters.
+    heads = [hi for _, hi in units]
+    P = {k: np.stack([I.head_params(sub, h)[k] for h in heads]).astype(np.float64)
+         for k in I.head_params(sub, 0)}
+    t0 = time.perf_counter()
+    if cfg.variant == "mlp":
+        Hn, d, h = len(units), cfg.d, cfg.hidden
+        params = np.concatenate([P["W1"].reshape(Hn, -1), P["W2"].reshape(Hn, -1)], axis=1)
+        # one "head" per sampled unit: lay the units out as B=1, H=len(units)
+        oracle.default().forward(oracle.MLP_LN, Q.transpose(1, 0, 2, 3), K.transpose(1, 0, 2, 3),
+                                 V.transpose(1, 0, 2, 3), eta.transpose(1, 0, 2), params, cfg.b,
+                                 P["gamma"], P["beta"], cfg.ln_eps, hidden=h, nthreads=nthreads)
+    else:
+        kind = oracle.LINEAR if cfg.variant == "linear" else oracle.LINEAR_LN
+        Hn, d = len(units), cfg.d
+        ln = kind == oracle.LINEAR_LN
+        oracle.default().forward(kind, Q.transpose(1, 0, 2, 3), K.transpose(1, 0, 2, 3),
+                                 V.transpose(1, 0, 2, 3), eta.transpose(1, 0, 2),
+                                 P["W0"].reshape(Hn, d * d), cfg.b, P["gamma"] if ln else None,
+                                 P["beta"] if ln else None, cfg.ln_eps, nthreads=nthreads)
+    return time.perf_counter() - t0
+
+
+def sample_plan(cfg, budget_s, cores):
+    """Units and tokens of a bounded oracle sample taking about budget_s on `cores` threads."""
+    T_cal = min(cfg.T, 1024)
+    t_cal = oracle_sample(cfg, [(0, 0)], T_cal, 1)
+    per_unit = t_cal * cfg.T / T_cal
+    n_units = int(budget_s * cores / max(per_unit, 1e-6))
+    if n_units >= cores:
+        n_units = min(cfg.units, max(cores, (n_units // cores) * cores))
+        T = cfg.T
+    else:  # fewer whole units than cores: shorten the sequences instead
+        n_units = min(cfg.units, cores)
+        T = max(cfg.b, int(budget_s / (t_cal / T_cal)) // cfg.b * cfg.b)
+        T = min(T, cfg.T)
+    rng = np.random.default_rng(123)
+    idx = sorted(rng.choice(cfg.units, size=n_units, replace=False).tolist())
+    return [divmod(int(u), cfg.H) for u in idx], T
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    import oracle
+    cores = oracle.default().default_threads()
+    units, T = sample_plan(cfg, budget_s, cores)
+    dt = oracle_sample(cfg, units, T, cores)
+    return {"value": len(units) * T / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(units)} of {cfg.units} (batch, head) units x {T} tokens of {cfg.name}, "
+                      f"fp64 primal oracle on {cores} threads, {dt:.2f} s"}
+
+
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    cores = oracle.default().default_threads()
+    units, T = sample_plan(cfg, 2.0, cores)  # ~2 s of host work per step
+    for _ in range(args.warmup):
+        oracle_sample(cfg, units, T, cores)
+    times = [oracle_sample(cfg, units, T, cores) for _ in range(args.steps)]
+    tot = sum(times)
+    value = args.steps * len(units) * T / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(cfg, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {len(units)} of {cfg.units} (batch, head) units x "
+                                   f"{T} tokens of {cfg.name}, fp64 primal oracle"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, args, world=1):
+    return {"workload": cfg.name, "variant": cfg.variant, "B_per_gpu": cfg.B, "H": cfg.H,
+            "T": cfg.T, "d": cfg.d, "b": cfg.b, "qkv_dtype": cfg.dtype,
+            "global_batch": cfg.B * world, "sharding": f"batch over {world} GPU(s), no collective",
+            "l2": "inputs larger than L2 (no flush needed)"
+            if bytes_per_launch(cfg) > 4 * L2_BYTES else "L2 flushed between steps",
+            "path": args.path}
+
+
+# --- our arm ----------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="linear_ln_B16H32T8192", choices=I.CONFIG_ORDER)
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling cases)")
+    ap.add_argument("--seq", type=int, default=None, help="override T (smaller profiling cases)")
+    args = ap.parse_args()
+    cfg = I.CONFIGS[args.workload]
+    if args.batch is not None or args.seq is not None:
+        cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T,
+                          name=f"{cfg.name}[B={args.batch or cfg.B},T={args.seq or cfg.T}]")
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    import torch
+    import torch.distributed as dist
+
+    import test_sequence_modeling_b200 as ttt
+    from test_sequence_modeling_b200 import _lib
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    small = cfg.units * cfg.T * cfg.d * 3 * 2 < 4 * L2_BYTES
+    lib = _lib.load()
+    ttt.set_path({"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT, "tc": ttt.TTT_PATH_TC}[args.path])
+
+    data = I.make_inputs(cfg, batch_offset=rank * cfg.B)
+    if data["qkv_bits"]:
+        host = {k: torch.from_numpy(data[k].view(np.int16)).view(torch.bfloat16) for k in "QKV"}
+    else:
+        host = {k: torch.from_numpy(data[k]) for k in "QKV"}
+    for k in ("eta", "W0", "W1", "W2", "gamma", "beta"):
+        if k in data:
+            host[k] = torch.from_numpy(np.ascontiguousarray(data[k]))
+    d_in = {k: v.to(dev) for k, v in host.items()}
+    B, H, T, d = cfg.B, cfg.H, cfg.T, cfg.d
+    outs = {"Z": torch.empty(B, H, T, d, device=dev)}
+    if cfg.variant == "mlp":
+        outs["W1_out"] = torch.empty(B, H, d, cfg.hidden, device=dev)
+        outs["W2_out"] = torch.empty(B, H, cfg.hidden, d, device=dev)
+    else:
+        outs["W_out"] = torch.empty(B, H, d, d, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, device=dev) if small else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step(src=d_in, dst=outs):
+        if cfg.variant == "linear":
+            ttt.ttt_linear_fwd(src["Q"], src["K"], src["V"], src["eta"], src["W0"], cfg.b,
+                               Z=dst["Z"], W_out=dst["W_out"], stream=stream)
+        elif cfg.variant == "linear_ln":
+            ttt.ttt_linear_ln_fwd(src["Q"], src["K"], src["V"], src["eta"], src["W0"], src["gamma"],
+                                  src["beta"], cfg.b, cfg.ln_eps, Z=dst["Z"], W_out=dst["W_out"],
+                                  stream=stream)
+        else:
+            ttt.ttt_mlp_fwd(src["Q"], src["K"], src["V"], src["eta"], src["W1"], src["W2"],
+                            src["gamma"], src["beta"], cfg.b, cfg.ln_eps, Z=dst["Z"],
+                            W1_out=dst["W1_out"], W2_out=dst["W2_out"], stream=stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if ttt.last_device_status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    clocks = ClockSampler(gpu_id_for(torch, local))
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    n0 = lib.ttt_launch_count()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    launches = lib.ttt_launch_count() - n0
+    clock_info = clocks.stop()
+    kernel_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(kernel_ms) if flush is not None else t_start.elapsed_time(t_end)
+    status = ttt.last_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    t = torch.tensor([total_ms, statistics.mean(kernel_ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, kernel_avg_ms = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    value = world * cfg.head_tokens * args.steps / (total_ms / 1e3)
+
+    # End to end through the public binding: pinned host inputs in, host outputs back.
+    e2e = None if args.e2e_steps <= 0 else measure_e2e(args, cfg, host, outs, d_in, step, stream,
+                                                       barrier, world, dev, torch, dist)
+    peaks, peak_kind = load_peaks()
+    nbytes = bytes_per_launch(cfg)
+    nflops = flops_per_head_token(cfg) * cfg.head_tokens
+    return finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info, launches,
+                  e2e, peaks, peak_kind, nbytes, nflops, dist)
+
+
+def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, torch, dist):
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    h_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
+    d_e2e = {k: torch.empty_like(v) for k, v in d_in.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = sum(v.numel() * v.element_size() for v in h_out.values())
+
+    def e2e_step():
+        for k in pin:
+            d_e2e[k].copy_(pin[k], non_blocking=True)
+        step(d_e2e, outs)
+        for k in h_out:
+            h_out[k].copy_(outs[k], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = world * cfg.head_tokens * args.e2e_steps / (float(te[0]) / 1e3)
+    return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps}
+
+
+def finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info, launches, e2e,
+           peaks, peak_kind, nbytes, nflops, dist):
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = nflops / (peaks["bf16_tflops_sustained"] * 1e12)
+    if t_hbm >= t_tc:
+        achieved = nbytes / (kernel_avg_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"]}
+    else:
+        achieved = nflops / (kernel_avg_ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"]}
+    traffic = committed_traffic(cfg.name)
+    roof.update({"traffic": traffic, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"
+                 if peak_kind == "measured" else "fallback",
+                 "algorithmic_bytes_per_launch": nbytes, "flops_per_launch": nflops,
+                 "kernel_ms": kernel_avg_ms})
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32",  # every product of the CUDA-core path is an fp32 FMA
+        "data": "synthetic", "config": workload_config(cfg, args, world),
+        "roofline": roof, "clocks": clock_info, "gpu_launches": int(launches), "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

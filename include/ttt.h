@@ -1,0 +1,147 @@
+/*
+ * ttt.h - C ABI of the Test-Time-Training (TTT) layer forward on NVIDIA B200 (sm_100a).
+ *
+ * The method (TTT write-up "大模型最强架构TTT问世！斯坦福UCSD等5年磨一剑，一夜推翻
+ * Transformer", a summary of arXiv 2407.04620):
+ *   - §03.1 "TTT hidden state": the layer's hidden state is the weight W of a
+ *     small model f; each token takes one gradient step on a self-supervised
+ *     loss, W_t = W_{t-1} - eta_t * grad l, and the output is f evaluated at the
+ *     updated weight, z_t = f(q_t; W_t).
+ *   - §03.5 "self-supervised task": l(W; t) = || f(k_t; W) - v_t ||^2, where
+ *     k, v, q are learned projections of the input computed outside this layer.
+ *   - §03.6 "mini-batch TTT": tokens are grouped in mini-batches of b; every
+ *     gradient of a mini-batch is taken at the state left by the previous one
+ *     (t' = t - mod(t, b), tokens 0-indexed).
+ *   - §03.7 "dual form": a whole mini-batch is computed with matrix products,
+ *     never materialising the b per-token gradients.
+ *   - §03.9 "two variants": TTT-Linear f(x) = x W (W square, d x d); TTT-MLP with
+ *     hidden width 4d and GELU; f carries a layer norm and a residual,
+ *     f(x) = x + LN(f_res(x)).
+ * Readings where the text is silent: the loss has no 1/2 (gradients carry a
+ * factor 2); LN uses the population variance and the caller's epsilon; gamma
+ * and beta are fixed per head and not updated by the inner loop; GELU is the
+ * exact x * Phi(x); f has no bias; the per-token step size eta_t scales the
+ * gradient of token t.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Row-vector convention: f(x) = x W with W[i][j] mapping input feature i to
+ * output feature j.  All arrays are dense, row-major and contiguous:
+ *   Q, K, V   [B][H][T][d]   dtype qkv_dtype (TTT_F32 or TTT_BF16)
+ *   eta       [B][H][T]      float32, step size of each token
+ *   W0        [H][d][d]      float32, initial state per head, shared by the batch
+ *   W1_0      [H][d][hidden], W2_0 [H][hidden][d]   (TTT-MLP initial state)
+ *   ln_gamma, ln_beta [H][d] float32
+ *   Z         [B][H][T][d]   float32 output
+ *   W_out     [B][H][d][d]   float32 final state of each (batch, head)
+ *   W1_out    [B][H][d][hidden], W2_out [B][H][hidden][d]
+ * Every pointer is a DEVICE pointer of the current CUDA device, 16-byte aligned.
+ * The caller owns every buffer; the library allocates nothing and keeps no
+ * pointer after the call.  Inputs are read only; outputs must not overlap any
+ * input or each other.  The work is enqueued on `stream` (a cudaStream_t; NULL
+ * is the legacy default stream) and the call returns without synchronising.
+ *
+ * Supported sizes: d = 64; 1 <= b <= 64 with T % b == 0 (b <= 16 for TTT-MLP);
+ * hidden = 4 d; B, H, T >= 0 with B*H*T*d < 2^40.  B*H == 0 is a no-op; T == 0
+ * copies the initial state to the outputs.  b = 16 with bf16 inputs runs the
+ * tensor-core path; every other supported case runs the exact-fp32 CUDA-core
+ * path.
+ *
+ * Errors: a call returns TTT_OK or a negative ttt_status.  Argument errors are
+ * detected on the host BEFORE anything is enqueued (nothing is launched and no
+ * CUDA call is made).  Launch failures return TTT_ERR_CUDA.  A device-side
+ * wait that runs past its bound stops that CTA, leaves its outputs undefined
+ * and records TTT_ERR_TIMEOUT in a device status word that
+ * ttt_last_device_status() reports.
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#if defined(__GNUC__)
+#define TTT_API __attribute__((visibility("default")))
+#else
+#define TTT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TTT_OK = 0,
+  TTT_ERR_ARG = -1,         /* null pointer, negative size, bad dtype, T % b != 0, overlap */
+  TTT_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+  TTT_ERR_UNSUPPORTED = -3, /* well-formed but outside the supported sizes (d, b, hidden) */
+  TTT_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+  TTT_ERR_TIMEOUT = -5      /* a bounded device-side wait expired (device status word) */
+} ttt_status;
+
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+/*
+ * TTT-Linear forward, f(x) = x W (§03.9; configs without LN).
+ * Per (batch, head) and mini-batch n with tiles Q, K, V [b x d], eta [b] and
+ * state W at the start of the mini-batch (dual form, §03.7):
+ *   G      = 2 (K W - V)                       gradient w.r.t. f's output
+ *   Z      = Q W - tril(Q K^T) diag(eta) G     (tril keeps s <= t)
+ *   W_next = W - K^T diag(eta) G
+ * Writes Z for every token and the final state to W_out.
+ */
+TTT_API int ttt_linear_fwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                   const float *W0, int B, int H, int T, int d, int b, float *Z, float *W_out,
+                   void *stream);
+
+/*
+ * TTT-Linear with layer norm and residual, f(x) = x + LN(x W) (§03.9).
+ * LN(y) = gamma * (y - mean(y)) / sqrt(var(y) + ln_eps) + beta over the d
+ * features of one row, population variance.  Per mini-batch:
+ *   G      = d l / d(K W) at the mini-batch base, through LN and the residual
+ *   Z      = Q + LN(Q W - tril(Q K^T) diag(eta) G)
+ *   W_next = W - K^T diag(eta) G
+ * ln_eps must be finite and > 0.
+ */
+TTT_API int ttt_linear_ln_fwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                      const float *W0, const float *ln_gamma, const float *ln_beta, float ln_eps,
+                      int B, int H, int T, int d, int b, float *Z, float *W_out, void *stream);
+
+/*
+ * TTT-MLP forward, f(x) = x + LN(GELU(x W1) W2), W1 [d x hidden],
+ * W2 [hidden x d], hidden = 4 d (§03.9).  Per mini-batch, with X1 = K W1,
+ * X2 = GELU(X1) and G3, G2 the loss gradients w.r.t. X2 W2 and X1 at the base:
+ *   Z1 = Q W1 - tril(Q K^T) diag(eta) G2,  Z2 = GELU(Z1)
+ *   Z  = Q + LN(Z2 W2 - tril(Z2 X2^T) diag(eta) G3)
+ *   W1_next = W1 - K^T diag(eta) G2,  W2_next = W2 - X2^T diag(eta) G3
+ */
+TTT_API int ttt_mlp_fwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                const float *W1_0, const float *W2_0, const float *ln_gamma, const float *ln_beta,
+                float ln_eps, int B, int H, int T, int d, int hidden, int b, float *Z,
+                float *W1_out, float *W2_out, void *stream);
+
+/* Static English text for a ttt_status value (never NULL). */
+TTT_API const char *ttt_status_string(int status);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the
+ * current device: TTT_OK, or TTT_ERR_TIMEOUT if a bounded wait of an earlier
+ * launch expired.  Returns TTT_ERR_CUDA if the synchronisation itself fails.
+ */
+TTT_API int ttt_last_device_status(void *stream);
+
+/*
+ * Kernel path selection for the next calls from any thread: TTT_PATH_AUTO
+ * (default: tensor cores where supported), TTT_PATH_SIMT (exact-fp32 CUDA-core
+ * kernels for every case) or TTT_PATH_TC (tensor cores; calls outside the
+ * tensor-core sizes return TTT_ERR_UNSUPPORTED).  Returns the previous path, or
+ * TTT_ERR_ARG for an unknown value.
+ */
+typedef enum { TTT_PATH_AUTO = 0, TTT_PATH_SIMT = 1, TTT_PATH_TC = 2 } ttt_path;
+TTT_API int ttt_set_path(int path);
+
+/* Number of CUDA kernels this library enqueued since load (for launch accounting). */
+TTT_API long long ttt_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H_ */

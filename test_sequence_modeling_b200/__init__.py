@@ -1,0 +1,18 @@
+"""TTT layer forward (mini-batch TTT, dual form) on NVIDIA B200, sm_100a.
+
+The computation lives in ``libttt.so`` (C ABI in ``include/ttt.h``); the
+functions below are its Python binding over torch CUDA tensors.  ``inputs``
+holds the seeded synthetic workloads.
+"""
+from ._lib import (TTT_BF16, TTT_F32, TTT_PATH_AUTO, TTT_PATH_SIMT, TTT_PATH_TC,  # noqa: F401
+                   TTTError)
+
+
+def __getattr__(name):
+    # The torch-facing binding is imported on first use so that ``inputs`` and the
+    # ABI constants stay importable without touching CUDA.
+    if name in ("ttt_linear_fwd", "ttt_linear_ln_fwd", "ttt_mlp_fwd", "set_path",
+                "last_device_status", "launch_count"):
+        from . import ttt
+        return getattr(ttt, name)
+    raise AttributeError(name)

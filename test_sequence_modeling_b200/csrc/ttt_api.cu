@@ -1,0 +1,225 @@
+// ttt_api.cu - C ABI of the TTT layer forward: argument checks, kernel
+// selection and launch.  Everything the ABI promises about errors is decided
+// here on the host before any CUDA call.  The kernels live in the headers this
+// file includes, so that the library is one translation unit and one device
+// status word.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ttt.h"
+#include "device_status.cuh"
+#include "simt.cuh"
+
+namespace simt = ttt::simt;
+
+namespace {
+
+std::atomic<int> g_path{TTT_PATH_AUTO};
+std::atomic<long long> g_launches{0};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;
+};
+Range range_of(const void *p, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return {a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+enum Kind { LINEAR = 0, LINEAR_LN = 1, MLP_LN = 2 };
+
+struct Call {
+  Kind kind;
+  const void *Q, *K, *V;
+  int qkv_dtype;
+  const float *eta, *W0, *W2_0, *gamma, *beta;
+  float eps;
+  int B, H, T, d, hidden, b;
+  float *Z, *W_out, *W2_out;
+  void *stream;
+};
+
+// Host-side checks shared by every entry point.  Returns TTT_OK or the status
+// to return without launching.
+int validate(const Call &c) {
+  if (c.qkv_dtype != TTT_F32 && c.qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (c.B < 0 || c.H < 0 || c.T < 0 || c.d <= 0 || c.b <= 0) return TTT_ERR_ARG;
+  if (c.T % c.b != 0) return TTT_ERR_ARG;
+  if (c.kind != LINEAR && !(std::isfinite(c.eps) && c.eps > 0.f)) return TTT_ERR_ARG;
+  if (c.kind == MLP_LN && c.hidden <= 0) return TTT_ERR_ARG;
+  if (c.d != simt::D) return TTT_ERR_UNSUPPORTED;
+  if (c.kind == MLP_LN && c.hidden != simt::HID) return TTT_ERR_UNSUPPORTED;
+  if (c.b > (c.kind == MLP_LN ? 16 : 64)) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)c.B * c.H;
+  if (units == 0) return TTT_OK;
+  if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  const long long elems = units * c.T * c.d;
+  if (elems >= (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+
+  // Pointers: required ones non-null and 16-byte aligned.
+  const bool has_tokens = c.T > 0;
+  const void *req[] = {c.W0, c.W_out, c.kind == MLP_LN ? (const void *)c.W2_0 : c.W0,
+                       c.kind == MLP_LN ? (const void *)c.W2_out : c.W_out,
+                       c.kind != LINEAR ? (const void *)c.gamma : c.W0,
+                       c.kind != LINEAR ? (const void *)c.beta : c.W0};
+  for (const void *p : req)
+    if (!p) return TTT_ERR_ARG;
+  if (has_tokens && (!c.Q || !c.K || !c.V || !c.eta || !c.Z)) return TTT_ERR_ARG;
+  for (const void *p : req)
+    if (!aligned16(p)) return TTT_ERR_ALIGN;
+  if (has_tokens) {
+    const void *tok[] = {c.Q, c.K, c.V, c.eta, c.Z};
+    for (const void *p : tok)
+      if (!aligned16(p)) return TTT_ERR_ALIGN;
+  }
+
+  // Outputs must not overlap inputs or each other.
+  const size_t in_elt = c.qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t P1 = c.kind == MLP_LN ? (size_t)c.d * c.hidden : (size_t)c.d * c.d;
+  Range ins[8];
+  int nin = 0;
+  if (has_tokens) {
+    ins[nin++] = range_of(c.Q, (size_t)elems * in_elt);
+    ins[nin++] = range_of(c.K, (size_t)elems * in_elt);
+    ins[nin++] = range_of(c.V, (size_t)elems * in_elt);
+    ins[nin++] = range_of(c.eta, (size_t)units * c.T * 4);
+  }
+  ins[nin++] = range_of(c.W0, (size_t)c.H * P1 * 4);
+  if (c.kind == MLP_LN) ins[nin++] = range_of(c.W2_0, (size_t)c.H * P1 * 4);
+  if (c.kind != LINEAR) {
+    ins[nin++] = range_of(c.gamma, (size_t)c.H * c.d * 4);
+    ins[nin++] = range_of(c.beta, (size_t)c.H * c.d * 4);
+  }
+  Range outs[3];
+  int nout = 0;
+  if (has_tokens) outs[nout++] = range_of(c.Z, (size_t)elems * 4);
+  outs[nout++] = range_of(c.W_out, (size_t)units * P1 * 4);
+  if (c.kind == MLP_LN) outs[nout++] = range_of(c.W2_out, (size_t)units * P1 * 4);
+  for (int o = 0; o < nout; ++o) {
+    for (int i = 0; i < nin; ++i)
+      if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
+    for (int o2 = o + 1; o2 < nout; ++o2)
+      if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
+  }
+  return TTT_OK;
+}
+
+template <typename KernelT>
+int launch(KernelT kernel, int grid, size_t smem, cudaStream_t stream,
+           const simt::Params &p) {
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return TTT_ERR_CUDA;
+  }
+  kernel<<<grid, simt::THREADS, smem, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
+int run_simt(const Call &c) {
+  simt::Params p;
+  p.Q = c.Q;
+  p.K = c.K;
+  p.V = c.V;
+  p.eta = c.eta;
+  p.W0 = c.W0;
+  p.W2_0 = c.W2_0;
+  p.gamma = c.gamma;
+  p.beta = c.beta;
+  p.eps = c.eps;
+  p.H = c.H;
+  p.T = c.T;
+  p.b = c.b;
+  p.Z = c.Z;
+  p.W_out = c.W_out;
+  p.W2_out = c.W2_out;
+  const int grid = c.B * c.H;
+  cudaStream_t s = static_cast<cudaStream_t>(c.stream);
+  const bool bf16 = c.qkv_dtype == TTT_BF16;
+  if (c.kind == MLP_LN) {
+    const size_t smem = simt::mlp_smem_bytes(c.b);
+    return bf16 ? launch(simt::mlp_kernel<__nv_bfloat16>, grid, smem, s, p)
+                : launch(simt::mlp_kernel<float>, grid, smem, s, p);
+  }
+  const size_t smem = simt::linear_smem_bytes(c.b);
+  if (c.kind == LINEAR_LN)
+    return bf16 ? launch(simt::linear_kernel<true, __nv_bfloat16>, grid, smem, s, p)
+                : launch(simt::linear_kernel<true, float>, grid, smem, s, p);
+  return bf16 ? launch(simt::linear_kernel<false, __nv_bfloat16>, grid, smem, s, p)
+              : launch(simt::linear_kernel<false, float>, grid, smem, s, p);
+}
+
+int run(const Call &c) {
+  const int st = validate(c);
+  if (st != TTT_OK) return st;
+  if ((long long)c.B * c.H == 0) return TTT_OK;
+  const int path = g_path.load();
+  if (path == TTT_PATH_TC) return TTT_ERR_UNSUPPORTED;  // no tensor-core kernel for this case
+  return run_simt(c);
+}
+
+}  // namespace
+
+extern "C" {
+
+int ttt_linear_fwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                   const float *W0, int B, int H, int T, int d, int b, float *Z, float *W_out,
+                   void *stream) {
+  Call c{LINEAR, Q, K, V, qkv_dtype, eta, W0, nullptr, nullptr, nullptr, 0.f,
+         B,      H, T, d, 0,         b,   Z,  W_out,   nullptr, stream};
+  return run(c);
+}
+
+int ttt_linear_ln_fwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                      const float *W0, const float *ln_gamma, const float *ln_beta, float ln_eps,
+                      int B, int H, int T, int d, int b, float *Z, float *W_out, void *stream) {
+  Call c{LINEAR_LN, Q, K, V, qkv_dtype, eta, W0, nullptr, ln_gamma, ln_beta, ln_eps,
+         B,         H, T, d, 0,         b,   Z,  W_out,   nullptr,  stream};
+  return run(c);
+}
+
+int ttt_mlp_fwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                const float *W1_0, const float *W2_0, const float *ln_gamma, const float *ln_beta,
+                float ln_eps, int B, int H, int T, int d, int hidden, int b, float *Z,
+                float *W1_out, float *W2_out, void *stream) {
+  Call c{MLP_LN, Q, K, V, qkv_dtype, eta, W1_0, W2_0, ln_gamma, ln_beta, ln_eps,
+         B,      H, T, d, hidden,    b,   Z,    W1_out, W2_out, stream};
+  return run(c);
+}
+
+const char *ttt_status_string(int status) {
+  switch (status) {
+    case TTT_OK: return "success";
+    case TTT_ERR_ARG: return "invalid argument (null pointer, negative size, bad dtype, T % b != 0 or overlapping buffers)";
+    case TTT_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case TTT_ERR_UNSUPPORTED: return "unsupported size (d, b or hidden) for this library";
+    case TTT_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+    case TTT_ERR_TIMEOUT: return "a bounded device-side wait expired";
+    default: return "unknown status";
+  }
+}
+
+int ttt_last_device_status(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TTT_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, ttt::g_device_status, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(ttt::g_device_status, &zero, sizeof(int)) != cudaSuccess) return TTT_ERR_CUDA;
+  return v;
+}
+
+int ttt_set_path(int path) {
+  if (path != TTT_PATH_AUTO && path != TTT_PATH_SIMT && path != TTT_PATH_TC) return TTT_ERR_ARG;
+  return g_path.exchange(path);
+}
+
+long long ttt_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -136,9 +136,12 @@ def params(cfg: TTTConfig) -> dict:
     return {k: np.stack([p[k] for p in per]) for k in per[0]}
 
 
-def make_inputs(cfg: TTTConfig, threads: int = 8, bf16_as_bits: bool = True) -> dict:
+def make_inputs(cfg: TTTConfig, threads: int = 8, bf16_as_bits: bool = True,
+                batch_offset: int = 0) -> dict:
     """Full workload.  Q, K, V [B,H,T,d]: float32, or (bf16 with bf16_as_bits) uint16
-    bf16 encodings; eta [B,H,T] float32; plus the per-head parameters."""
+    bf16 encodings; eta [B,H,T] float32; plus the per-head parameters.  Batch row i
+    holds the units of global batch index batch_offset + i (how a data-parallel
+    rank draws its own shard)."""
     B, H, T, d = cfg.B, cfg.H, cfg.T, cfg.d
     as_bits = cfg.dtype == "bf16" and bf16_as_bits
     qkv_dt = np.uint16 if as_bits else np.float32
@@ -149,7 +152,7 @@ def make_inputs(cfg: TTTConfig, threads: int = 8, bf16_as_bits: bool = True) -> 
 
     def fill(u):
         bi, hi = divmod(u, H)
-        q, k, v, e = unit_inputs(cfg, bi, hi)
+        q, k, v, e = unit_inputs(cfg, batch_offset + bi, hi)
         if as_bits:
             q, k, v = bf16_bits(q), bf16_bits(k), bf16_bits(v)
         Q[bi, hi], K[bi, hi], V[bi, hi], eta[bi, hi] = q, k, v, e

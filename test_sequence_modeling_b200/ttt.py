@@ -1,0 +1,128 @@
+"""Python binding of the TTT layer forward: marshals torch CUDA tensors into the C ABI.
+
+Every step of the computation runs in the CUDA kernels of libttt.so; this module
+only checks shapes and dtypes, allocates outputs when the caller passes none,
+and hands raw device pointers and the current CUDA stream to the library.  There
+is no CPU path: tensors that are not on a CUDA device are rejected.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _lib
+from ._lib import TTT_BF16, TTT_F32, TTTError, check  # noqa: F401
+
+_QKV_DTYPES = {torch.float32: TTT_F32, torch.bfloat16: TTT_BF16}
+
+
+def _cuda(t, name, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _qkv(Q, K, V):
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        _cuda(t, n)
+    if not (Q.dtype == K.dtype == V.dtype) or Q.dtype not in _QKV_DTYPES:
+        raise TypeError("Q, K, V must share one dtype, float32 or bfloat16")
+    if not (Q.shape == K.shape == V.shape) or Q.dim() != 4:
+        raise ValueError("Q, K, V must have the same shape [B, H, T, d]")
+    return _QKV_DTYPES[Q.dtype]
+
+
+def _out(t, shape, device, name):
+    if t is None:
+        return torch.empty(shape, dtype=torch.float32, device=device)
+    _cuda(t, name, torch.float32)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}")
+    return t
+
+
+def _stream(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes_stream(s)
+
+
+def ctypes_stream(s) -> int:
+    return int(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def ttt_linear_fwd(Q, K, V, eta, W0, b, Z=None, W_out=None, stream=None):
+    """TTT-Linear forward.  Q, K, V [B,H,T,d] (f32 or bf16), eta [B,H,T] f32, W0 [H,d,d] f32.
+    Returns (Z [B,H,T,d] f32, W_out [B,H,d,d] f32)."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    _cuda(eta, "eta", torch.float32)
+    _cuda(W0, "W0", torch.float32)
+    Z = _out(Z, (B, H, T, d), Q.device, "Z")
+    W_out = _out(W_out, (B, H, d, d), Q.device, "W_out")
+    with torch.cuda.device(Q.device):
+        st = _lib.load().ttt_linear_fwd(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W0), B, H, T,
+                                        d, int(b), _ptr(Z), _ptr(W_out), _stream(stream, Q.device))
+    check(st, "ttt_linear_fwd")
+    return Z, W_out
+
+
+def ttt_linear_ln_fwd(Q, K, V, eta, W0, gamma, beta, b, eps=1e-6, Z=None, W_out=None, stream=None):
+    """TTT-Linear with LN + residual.  gamma, beta [H,d] f32."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    for n, t in (("eta", eta), ("W0", W0), ("gamma", gamma), ("beta", beta)):
+        _cuda(t, n, torch.float32)
+    Z = _out(Z, (B, H, T, d), Q.device, "Z")
+    W_out = _out(W_out, (B, H, d, d), Q.device, "W_out")
+    with torch.cuda.device(Q.device):
+        st = _lib.load().ttt_linear_ln_fwd(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W0),
+                                           _ptr(gamma), _ptr(beta), float(eps), B, H, T, d, int(b),
+                                           _ptr(Z), _ptr(W_out), _stream(stream, Q.device))
+    check(st, "ttt_linear_ln_fwd")
+    return Z, W_out
+
+
+def ttt_mlp_fwd(Q, K, V, eta, W1, W2, gamma, beta, b, eps=1e-6, Z=None, W1_out=None, W2_out=None,
+                stream=None):
+    """TTT-MLP forward.  W1 [H,d,h], W2 [H,h,d] f32.  Returns (Z, W1_out, W2_out)."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    for n, t in (("eta", eta), ("W1", W1), ("W2", W2), ("gamma", gamma), ("beta", beta)):
+        _cuda(t, n, torch.float32)
+    hidden = W1.shape[-1]
+    Z = _out(Z, (B, H, T, d), Q.device, "Z")
+    W1_out = _out(W1_out, (B, H, d, hidden), Q.device, "W1_out")
+    W2_out = _out(W2_out, (B, H, hidden, d), Q.device, "W2_out")
+    with torch.cuda.device(Q.device):
+        st = _lib.load().ttt_mlp_fwd(_ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W1), _ptr(W2),
+                                     _ptr(gamma), _ptr(beta), float(eps), B, H, T, d, hidden,
+                                     int(b), _ptr(Z), _ptr(W1_out), _ptr(W2_out),
+                                     _stream(stream, Q.device))
+    check(st, "ttt_mlp_fwd")
+    return Z, W1_out, W2_out
+
+
+def set_path(path: int) -> int:
+    """Select the kernel path (TTT_PATH_AUTO / _SIMT / _TC); returns the previous one."""
+    prev = _lib.load().ttt_set_path(int(path))
+    if prev < 0:
+        raise TTTError(prev, "ttt_set_path")
+    return prev
+
+
+def last_device_status(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(_lib.load().ttt_last_device_status(ctypes_stream(s)))
+
+
+def launch_count() -> int:
+    return int(_lib.load().ttt_launch_count())

@@ -1,0 +1,121 @@
+"""The C ABI without a GPU: the library loads, exports what include/ttt.h declares,
+and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from test_sequence_modeling_b200 import _lib as L
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "ttt.h")).read()
+    return sorted(set(re.findall(r"TTT_API\s+[\w\s\*]*?\b(ttt_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from test_sequence_modeling_b200.build import build
+    build()
+    return L.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(L.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_status_strings(lib):
+    for s in (0, -1, -2, -3, -4, -5):
+        assert L.status_string(s)
+    assert L.status_string(12345) == "unknown status"
+
+
+def test_set_path(lib):
+    prev = lib.ttt_set_path(L.TTT_PATH_SIMT)
+    assert prev in (0, 1, 2)
+    assert lib.ttt_set_path(prev) == L.TTT_PATH_SIMT
+    assert lib.ttt_set_path(7) == L.TTT_ERR_ARG
+
+
+# Fake, never-dereferenced device addresses: every call below fails validation,
+# which runs before any CUDA call.
+A = 0x100000
+
+
+def _ptrs(n, step=1 << 30, base=A):
+    return [base + i * step for i in range(n)]
+
+
+def linear(lib, **kw):
+    q, k, v, eta, w0, z, wo = _ptrs(7)
+    a = dict(Q=q, K=k, V=v, dt=L.TTT_BF16, eta=eta, W0=w0, B=2, H=3, T=64, d=64, b=16, Z=z, W=wo)
+    a.update(kw)
+    return lib.ttt_linear_fwd(a["Q"], a["K"], a["V"], a["dt"], a["eta"], a["W0"], a["B"], a["H"],
+                              a["T"], a["d"], a["b"], a["Z"], a["W"], None)
+
+
+def ln(lib, **kw):
+    q, k, v, eta, w0, g, bt, z, wo = _ptrs(9)
+    a = dict(Q=q, K=k, V=v, dt=L.TTT_BF16, eta=eta, W0=w0, g=g, bt=bt, eps=1e-6, B=2, H=3, T=64,
+             d=64, b=16, Z=z, W=wo)
+    a.update(kw)
+    return lib.ttt_linear_ln_fwd(a["Q"], a["K"], a["V"], a["dt"], a["eta"], a["W0"], a["g"], a["bt"],
+                                 a["eps"], a["B"], a["H"], a["T"], a["d"], a["b"], a["Z"], a["W"], None)
+
+
+def mlp(lib, **kw):
+    q, k, v, eta, w1, w2, g, bt, z, w1o, w2o = _ptrs(11)
+    a = dict(Q=q, K=k, V=v, dt=L.TTT_BF16, eta=eta, W1=w1, W2=w2, g=g, bt=bt, eps=1e-6, B=2, H=3,
+             T=64, d=64, h=256, b=16, Z=z, W1o=w1o, W2o=w2o)
+    a.update(kw)
+    return lib.ttt_mlp_fwd(a["Q"], a["K"], a["V"], a["dt"], a["eta"], a["W1"], a["W2"], a["g"],
+                           a["bt"], a["eps"], a["B"], a["H"], a["T"], a["d"], a["h"], a["b"], a["Z"],
+                           a["W1o"], a["W2o"], None)
+
+
+@pytest.mark.parametrize("fn", [linear, ln, mlp])
+def test_argument_errors(lib, fn):
+    n0 = lib.ttt_launch_count()
+    assert fn(lib, T=60) == L.TTT_ERR_ARG                # T % b != 0
+    assert fn(lib, b=0) == L.TTT_ERR_ARG
+    assert fn(lib, B=-1) == L.TTT_ERR_ARG
+    assert fn(lib, dt=5) == L.TTT_ERR_ARG                # unknown dtype
+    assert fn(lib, d=32) == L.TTT_ERR_UNSUPPORTED
+    assert fn(lib, b=128, T=128) == L.TTT_ERR_UNSUPPORTED
+    assert fn(lib, Q=None) == L.TTT_ERR_ARG
+    assert fn(lib, Z=None) == L.TTT_ERR_ARG
+    assert fn(lib, Q=A + 8) == L.TTT_ERR_ALIGN
+    assert fn(lib, eta=A + 4) == L.TTT_ERR_ALIGN
+    assert fn(lib, Z=A + (3 << 30) + 64) == L.TTT_ERR_ARG  # Z overlaps V
+    assert fn(lib, B=0) == L.TTT_OK                      # empty: nothing to do, no CUDA call
+    assert fn(lib, H=0) == L.TTT_OK
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
+
+
+def test_ln_specific_errors(lib):
+    assert ln(lib, eps=0.0) == L.TTT_ERR_ARG
+    assert ln(lib, eps=float("nan")) == L.TTT_ERR_ARG
+    assert ln(lib, g=None) == L.TTT_ERR_ARG
+
+
+def test_mlp_specific_errors(lib):
+    assert mlp(lib, h=128) == L.TTT_ERR_UNSUPPORTED
+    assert mlp(lib, h=0) == L.TTT_ERR_ARG
+    assert mlp(lib, b=32, T=64) == L.TTT_ERR_UNSUPPORTED
+    assert mlp(lib, W2o=None) == L.TTT_ERR_ARG
+    assert mlp(lib, W2o=A + (9 << 30) + 16) == L.TTT_ERR_ARG  # W2_out overlaps W1_out
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    import test_sequence_modeling_b200 as ttt
+    x = torch.zeros(1, 1, 16, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        ttt.ttt_linear_fwd(x, x, x, torch.zeros(1, 1, 16), torch.zeros(1, 64, 64), 16)

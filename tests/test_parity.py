@@ -1,0 +1,115 @@
+"""GPU parity: the CUDA path against the fp64 oracle, through the C ABI.
+
+Reduced sizes compare every unit element by element; the full workloads (in the
+same launch configuration the benchmark times) compare sampled units.
+"""
+import numpy as np
+import pytest
+import torch
+
+import test_sequence_modeling_b200 as ttt
+from test_sequence_modeling_b200 import inputs as I
+from gpu_helpers import TOL, all_units, compare, run_gpu, sample_units, to_device
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT}
+
+
+@pytest.fixture(autouse=True)
+def _restore_path():
+    yield
+    ttt.set_path(ttt.TTT_PATH_AUTO)
+
+
+def reduced(cfg):
+    """Several mini-batches, several units and an odd unit count."""
+    if cfg.name.startswith("linear_f32"):
+        return cfg.replace(B=3, H=5, T=256)
+    return cfg.replace(B=3, H=5, T=128 if cfg.variant == "mlp" else 256)
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+@pytest.mark.parametrize("name", I.CONFIG_ORDER)
+def test_reduced_config_every_unit(name, path):
+    cfg = reduced(I.CONFIGS[name])
+    ttt.set_path(PATHS[path])
+    dev = to_device(cfg, I.make_inputs(cfg))
+    out = run_gpu(cfg, dev)
+    worst = compare(cfg, out, all_units(cfg))
+    tol = TOL[cfg.dtype]
+    assert max(worst.values()) <= tol, (name, path, worst)
+
+
+@pytest.mark.parametrize("name", I.CONFIG_ORDER)
+def test_full_size_sampled_units(name):
+    cfg = I.CONFIGS[name]
+    dev = to_device(cfg, I.make_inputs(cfg))
+    out = run_gpu(cfg, dev)
+    n = 6 if cfg.variant != "mlp" else 3
+    worst = compare(cfg, out, sample_units(cfg, n))
+    assert max(worst.values()) <= TOL[cfg.dtype], (name, worst)
+    # Properties that hold at any size: finite everywhere, no unit left unwritten.
+    for k, v in out.items():
+        assert np.all(np.isfinite(v)), k
+        assert np.all(np.abs(v).reshape(cfg.B * cfg.H, -1).max(axis=1) > 0), k
+
+
+@pytest.mark.parametrize("variant", ["linear", "linear_ln", "mlp"])
+@pytest.mark.parametrize("b", [1, 4, 16, 64])
+def test_mini_batch_sizes(variant, b):
+    if variant == "mlp" and b > 16:
+        pytest.skip("TTT-MLP supports b <= 16")
+    base = {"linear": "linear_bf16_B16H12T2048", "linear_ln": "linear_ln_B16H32T8192",
+            "mlp": "mlp_B8H32T8192"}[variant]
+    cfg = I.CONFIGS[base].replace(B=2, H=2, T=max(2 * b, 64), b=b)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    worst = compare(cfg, run_gpu(cfg, dev), all_units(cfg))
+    assert max(worst.values()) <= TOL[cfg.dtype], (variant, b, worst)
+
+
+@pytest.mark.parametrize("name", ["linear_bf16_B16H12T2048", "linear_ln_B16H32T8192", "mlp_B8H32T8192"])
+def test_empty_sequence_copies_initial_state(name):
+    cfg = I.CONFIGS[name].replace(B=2, H=3, T=0)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    out = run_gpu(cfg, dev)
+    for k in ("W0", "W1", "W2"):
+        if k in dev:
+            key = "W" if k == "W0" else k
+            ref = np.broadcast_to(dev[k].cpu().numpy()[None], out[key].shape)
+            assert np.array_equal(out[key], ref)
+
+
+def test_deterministic_and_stream_ordered():
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=2, H=4, T=512)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    a = run_gpu(cfg, dev)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b = run_gpu(cfg, dev, stream=s)
+    for k in a:
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_outputs_stay_in_bounds():
+    """Outputs carved from a larger buffer: the guard bytes around them stay untouched."""
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=2, H=3, T=64)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    nz = cfg.B * cfg.H * cfg.T * cfg.d
+    nw = cfg.B * cfg.H * cfg.d * cfg.d
+    buf = torch.full((nz + nw + 3 * 1024,), 7.0, device="cuda")
+    Z = buf[1024:1024 + nz].view(cfg.B, cfg.H, cfg.T, cfg.d)
+    W = buf[2048 + nz:2048 + nz + nw].view(cfg.B, cfg.H, cfg.d, cfg.d)
+    ttt.ttt_linear_ln_fwd(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], dev["gamma"],
+                          dev["beta"], cfg.b, cfg.ln_eps, Z=Z, W_out=W)
+    torch.cuda.synchronize()
+    h = buf.cpu().numpy()
+    assert np.all(h[:1024] == 7.0) and np.all(h[1024 + nz:2048 + nz] == 7.0)
+    assert np.all(h[2048 + nz + nw:] == 7.0)
+
+
+def test_device_status_clean_after_runs():
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=1, H=2, T=64)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    run_gpu(cfg, dev)
+    assert ttt.last_device_status() == 0
