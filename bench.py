@@ -183,28 +183,29 @@ def oracle_sample(cfg, units, T, nthreads):
     return time.perf_counter() - t0
 
 
-def sample_plan(cfg, budget_s, cores):
-    """Units and tokens of a bounded oracle sample taking about budget_s on `cores` threads."""
+def sample_plan(cfg, budget_cpu_s, cores):
+    """Units and tokens of a bounded oracle sample taking about budget_cpu_s of CPU time
+    (summed over `cores` threads)."""
     T_cal = min(cfg.T, 1024)
     t_cal = oracle_sample(cfg, [(0, 0)], T_cal, 1)
     per_unit = t_cal * cfg.T / T_cal
-    n_units = int(budget_s * cores / max(per_unit, 1e-6))
+    n_units = int(budget_cpu_s / max(per_unit, 1e-6))
     if n_units >= cores:
         n_units = min(cfg.units, max(cores, (n_units // cores) * cores))
         T = cfg.T
     else:  # fewer whole units than cores: shorten the sequences instead
         n_units = min(cfg.units, cores)
-        T = max(cfg.b, int(budget_s / (t_cal / T_cal)) // cfg.b * cfg.b)
+        T = max(cfg.b, int(budget_cpu_s / cores / (t_cal / T_cal)) // cfg.b * cfg.b)
         T = min(T, cfg.T)
     rng = np.random.default_rng(123)
     idx = sorted(rng.choice(cfg.units, size=n_units, replace=False).tolist())
     return [divmod(int(u), cfg.H) for u in idx], T
 
 
-def cpu_baseline(cfg, budget_s=15.0):
+def cpu_baseline(cfg, budget_cpu_s=20.0):
     import oracle
     cores = oracle.default().default_threads()
-    units, T = sample_plan(cfg, budget_s, cores)
+    units, T = sample_plan(cfg, budget_cpu_s, cores)
     dt = oracle_sample(cfg, units, T, cores)
     return {"value": len(units) * T / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{len(units)} of {cfg.units} (batch, head) units x {T} tokens of {cfg.name}, "
@@ -217,7 +218,7 @@ def run_reference(args, cfg):
         return 0
     import oracle
     cores = oracle.default().default_threads()
-    units, T = sample_plan(cfg, 2.0, cores)  # ~2 s of host work per step
+    units, T = sample_plan(cfg, 2.0 * cores, cores)  # ~2 s of wall time per step
     for _ in range(args.warmup):
         oracle_sample(cfg, units, T, cores)
     times = [oracle_sample(cfg, units, T, cores) for _ in range(args.steps)]
