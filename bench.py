@@ -238,6 +238,14 @@ def run_reference(args, cfg):
     return 0
 
 
+def dtype_of(cfg, path):
+    """Arithmetic type of the path that runs: tensor-core products take bf16 operands
+    (fp32 values split into bf16 hi + lo) with fp32 accumulation; the CUDA-core path
+    is fp32 throughout."""
+    tc = cfg.dtype == "bf16" and cfg.b == 16 and cfg.variant != "mlp" and path != "simt"
+    return "bf16" if tc else "f32"
+
+
 def workload_config(cfg, args, world=1):
     return {"workload": cfg.name, "variant": cfg.variant, "B_per_gpu": cfg.B, "H": cfg.H,
             "T": cfg.T, "d": cfg.d, "b": cfg.b, "qkv_dtype": cfg.dtype,
@@ -426,7 +434,7 @@ def finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32",  # every product of the CUDA-core path is an fp32 FMA
+        "dtype": dtype_of(cfg, args.path),
         "data": "synthetic", "config": workload_config(cfg, args, world),
         "roofline": roof, "clocks": clock_info, "gpu_launches": int(launches), "e2e": e2e,
     }

@@ -6,14 +6,18 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include "ttt.h"
 #include "device_status.cuh"
 #include "simt.cuh"
+#include "tc_linear.cuh"
 
 namespace simt = ttt::simt;
+namespace tc = ttt::tc;
 
 namespace {
 
@@ -156,12 +160,79 @@ int run_simt(const Call &c) {
               : launch(simt::linear_kernel<false, float>, grid, smem, s, p);
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so that the
+// library does not link against libcuda.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// [units][T][64] bf16 viewed as a 3-D tensor; boxes of 64 tokens x 64 features
+// with the 128-byte swizzle.  Rows past T read as zeros.
+bool make_qkv_map(CUtensorMap *map, const void *base, int T, long long units) {
+  auto encode = tensor_map_encoder();
+  if (!encode) return false;
+  cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)units};
+  cuuint64_t strides[2] = {64 * 2, (cuuint64_t)T * 64 * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tc_supported(const Call &c) {
+  return c.kind != MLP_LN && c.qkv_dtype == TTT_BF16 && c.b == tc::MB && c.T > 0;
+}
+
+template <bool LN>
+int launch_linear_tc(const Call &c) {
+  const long long units = (long long)c.B * c.H;
+  CUtensorMap mq, mk, mv;
+  if (!make_qkv_map(&mq, c.Q, c.T, units) || !make_qkv_map(&mk, c.K, c.T, units) ||
+      !make_qkv_map(&mv, c.V, c.T, units))
+    return TTT_ERR_CUDA;
+  tc::Params p;
+  p.eta = c.eta;
+  p.W0 = c.W0;
+  p.gamma = c.gamma;
+  p.beta = c.beta;
+  p.eps = c.eps;
+  p.H = c.H;
+  p.T = c.T;
+  p.Z = c.Z;
+  p.W_out = c.W_out;
+  auto kernel = tc::linear_tc_kernel<LN>;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tc::SMEM_BYTES) != cudaSuccess ||
+      cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  kernel<<<(unsigned)units, tc::THREADS, tc::SMEM_BYTES, static_cast<cudaStream_t>(c.stream)>>>(
+      mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 int run(const Call &c) {
   const int st = validate(c);
   if (st != TTT_OK) return st;
   if ((long long)c.B * c.H == 0) return TTT_OK;
   const int path = g_path.load();
-  if (path == TTT_PATH_TC) return TTT_ERR_UNSUPPORTED;  // no tensor-core kernel for this case
+  const bool tc_ok = tc_supported(c);
+  if (path == TTT_PATH_TC && !tc_ok) return TTT_ERR_UNSUPPORTED;
+  if (path != TTT_PATH_SIMT && tc_ok)
+    return c.kind == LINEAR_LN ? launch_linear_tc<true>(c) : launch_linear_tc<false>(c);
   return run_simt(c);
 }
 

@@ -13,7 +13,11 @@ from gpu_helpers import TOL, all_units, compare, run_gpu, sample_units, to_devic
 
 pytestmark = pytest.mark.gpu
 
-PATHS = {"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT}
+PATHS = {"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT, "tc": ttt.TTT_PATH_TC}
+
+
+def tc_capable(cfg):
+    return cfg.dtype == "bf16" and cfg.variant != "mlp" and cfg.b == 16
 
 
 @pytest.fixture(autouse=True)
@@ -33,6 +37,8 @@ def reduced(cfg):
 @pytest.mark.parametrize("name", I.CONFIG_ORDER)
 def test_reduced_config_every_unit(name, path):
     cfg = reduced(I.CONFIGS[name])
+    if path == "tc" and not tc_capable(cfg):
+        pytest.skip("no tensor-core kernel for this case")
     ttt.set_path(PATHS[path])
     dev = to_device(cfg, I.make_inputs(cfg))
     out = run_gpu(cfg, dev)
@@ -113,3 +119,29 @@ def test_device_status_clean_after_runs():
     dev = to_device(cfg, I.make_inputs(cfg))
     run_gpu(cfg, dev)
     assert ttt.last_device_status() == 0
+
+
+@pytest.mark.parametrize("variant", ["linear", "linear_ln"])
+@pytest.mark.parametrize("T", [16, 48, 80, 208, 1040])
+def test_tensor_core_ragged_chunks(variant, T):
+    """Sequences whose length is not a multiple of the 64-token chunk."""
+    base = {"linear": "linear_bf16_B16H12T2048", "linear_ln": "linear_ln_B16H32T8192"}[variant]
+    cfg = I.CONFIGS[base].replace(B=2, H=3, T=T)
+    ttt.set_path(ttt.TTT_PATH_TC)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    worst = compare(cfg, run_gpu(cfg, dev), all_units(cfg))
+    assert max(worst.values()) <= TOL[cfg.dtype], (variant, T, worst)
+
+
+@pytest.mark.parametrize("name", ["linear_bf16_B16H12T2048", "linear_ln_B16H32T8192"])
+def test_tensor_core_matches_cuda_core_path(name):
+    """The two CUDA paths agree far below the oracle tolerance."""
+    cfg = I.CONFIGS[name].replace(B=2, H=4, T=1024)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    ttt.set_path(ttt.TTT_PATH_TC)
+    a = run_gpu(cfg, dev)
+    ttt.set_path(ttt.TTT_PATH_SIMT)
+    b = run_gpu(cfg, dev)
+    for k in a:
+        rel = np.linalg.norm(a[k] - b[k]) / np.linalg.norm(b[k])
+        assert rel < 2e-4, (k, rel)
