@@ -68,13 +68,14 @@ constexpr uint32_t OFF_BETA = 49664;  // LN beta, 64 floats
 constexpr uint32_t OFF_BAR = 49920;   // mbarriers
 constexpr uint32_t OFF_TSLOT = 49984; // TMEM base address
 constexpr uint32_t OFF_ABORT = 49988; // set when a bounded wait expired
-constexpr uint32_t SMEM_USED = 49992;
+constexpr uint32_t SMEM_USED = 50000;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
-// mbarriers: tile loads; MMA P,S; mini-batch 0,1,2 updates; last update; dW.
-enum { BAR_LOAD = 0, BAR_PS = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, NUM_BARS = 7 };
+// mbarriers: K/V/eta loads; Q load; MMA P,S; mini-batch 0,1,2 updates; last update; dW.
+enum { BAR_LOAD = 0, BAR_PS = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, BAR_LOADQ = 7, NUM_BARS = 8 };
 
 struct Params {
+  const __nv_bfloat16 *Q;  // for the residual of the output (read back from L2)
   const float *eta;
   const float *W0;
   const float *gamma, *beta;
@@ -170,13 +171,18 @@ __global__ void __launch_bounds__(THREADS, 4)
   const int nchunks = (T + CHUNK - 1) / CHUNK;
   const size_t tok_base = (size_t)unit * T;
 
-  auto issue_loads = [&](int c) {
+  // Loads are split so that each tile is fetched as soon as its buffer is free:
+  // Q once P and S are computed, K / V / eta once dW is computed.
+  auto issue_loads_kv = [&](int c) {
     const int ntok = min(CHUNK, T - c * CHUNK);
-    mbar_arrive_expect_tx(&bars[BAR_LOAD], 3u * 8192u + (uint32_t)ntok * 4u);
+    mbar_arrive_expect_tx(&bars[BAR_LOAD], 2u * 8192u + (uint32_t)ntok * 4u);
     tma_load_3d(sm + OFF_K, &tmK, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
-    tma_load_3d(sm + OFF_Q, &tmQ, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
     tma_load_3d(sm + OFF_GLO, &tmV, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
     bulk_load(eta_s, p.eta + tok_base + (size_t)c * CHUNK, (uint32_t)ntok * 4u, &bars[BAR_LOAD]);
+  };
+  auto issue_load_q = [&](int c) {
+    mbar_arrive_expect_tx(&bars[BAR_LOADQ], 8192u);
+    tma_load_3d(sm + OFF_Q, &tmQ, 0, c * CHUNK, unit, &bars[BAR_LOADQ]);
   };
 
   fence_proxy_async_smem();
@@ -185,7 +191,10 @@ __global__ void __launch_bounds__(THREADS, 4)
   tc_fence_after_sync();
   const uint32_t tb = *tslot;
   const uint32_t tP = tb, tS = tb + 64;  // column bases of P and S (lane 0)
-  if (tid == 0 && nchunks > 0) issue_loads(0);
+  if (tid == 0 && nchunks > 0) {
+    issue_loads_kv(0);
+    issue_load_q(0);
+  }
 
   constexpr uint32_t ID_PW = idesc_bf16_f32(128, 64, false, true, false);   // [K;Q] x W
   constexpr uint32_t ID_S = idesc_bf16_f32(128, 64, false, false, false);   // [K;Q] x K^T
@@ -199,6 +208,7 @@ __global__ void __launch_bounds__(THREADS, 4)
 
     // ---- 1-2: tiles in, P = [K;Q] W and S = [K;Q] K^T ----------------------------
     wait_or_abort(&bars[BAR_LOAD], par, abort);
+    wait_or_abort(&bars[BAR_LOADQ], par, abort);
     if (tid == 0 && !*abort) {
       tc_fence_after_sync();
 #pragma unroll
@@ -257,6 +267,10 @@ __global__ void __launch_bounds__(THREADS, 4)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
+    // The Q buffer is free (P and S are done).  Issued only after this barrier:
+    // every thread has then passed its wait on this chunk's Q phase, so the Q
+    // barrier cannot complete twice while a thread still waits on it.
+    if (tid == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
 
     // ---- 4: the mini-batch chain (warp 0: mini-batches 0-1, warp 1: 2-3) ---------
     if (warp < 2) {
@@ -277,18 +291,29 @@ __global__ void __launch_bounds__(THREADS, 4)
           g1[2 * j] = __uint_as_float(yr[4 * j + 2]);
           g1[2 * j + 1] = __uint_as_float(yr[4 * j + 3]);
         }
+        const uint32_t sbase = smem_u32(sm);
         auto ld2 = [&](uint32_t off, int row, int col) {
-          return unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + off + sw128_offset(row, col)));
+          return unpack_bf16x2(lds_u32(sbase + off + sw128_offset(row, col)));
+        };
+        const float e0 = eta_s[r0], e1 = eta_s[r1];
+        // Stores eta * (dl/dy) of one column pair of both rows as bf16 hi + lo; the
+        // lo half overwrites V, which this thread has read for exactly these cells.
+        auto store_grad = [&](int col, float ga0, float ga1, float gb0, float gb1) {
+          uint32_t h0, l0, h1, l1;
+          split_bf16x2(e0 * ga0, e0 * ga1, h0, l0);
+          split_bf16x2(e1 * gb0, e1 * gb1, h1, l1);
+          *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r0, col)) = h0;
+          *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r0, col)) = l0;
+          *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r1, col)) = h1;
+          *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r1, col)) = l1;
         };
         if (!LN) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int col = 8 * j + 2 * q4;
             const float2 va = ld2(OFF_GLO, r0, col), vb = ld2(OFF_GLO, r1, col);
-            g0[2 * j] = 2.f * (g0[2 * j] - va.x);
-            g0[2 * j + 1] = 2.f * (g0[2 * j + 1] - va.y);
-            g1[2 * j] = 2.f * (g1[2 * j] - vb.x);
-            g1[2 * j + 1] = 2.f * (g1[2 * j + 1] - vb.y);
+            store_grad(col, 2.f * (g0[2 * j] - va.x), 2.f * (g0[2 * j + 1] - va.y),
+                       2.f * (g1[2 * j] - vb.x), 2.f * (g1[2 * j + 1] - vb.y));
           }
         } else {
           // LN backward of ||k + gamma*xhat + beta - v||^2 w.r.t. y: with
@@ -311,23 +336,27 @@ __global__ void __launch_bounds__(THREADS, 4)
           }
           const float rstd0 = rsqrtf(quad_sum(q0) * (1.f / D) + p.eps);
           const float rstd1 = rsqrtf(quad_sum(q1) * (1.f / D) + p.eps);
-          float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             g0[e] *= rstd0;  // xhat
             g1[e] *= rstd1;
           }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int col = 8 * j + 2 * q4;
+          auto dxhat = [&](int col, float xa0, float xa1, float xb0, float xb1, float &d00,
+                           float &d01, float &d10, float &d11) {
             const float2 ka = ld2(OFF_K, r0, col), kb = ld2(OFF_K, r1, col);
             const float2 va = ld2(OFF_GLO, r0, col), vb = ld2(OFF_GLO, r1, col);
-            const float2 gm = *reinterpret_cast<const float2 *>(gam_s + col);
-            const float2 bt = *reinterpret_cast<const float2 *>(bet_s + col);
-            const float d00 = 2.f * (ka.x + gm.x * g0[2 * j] + bt.x - va.x) * gm.x;
-            const float d01 = 2.f * (ka.y + gm.y * g0[2 * j + 1] + bt.y - va.y) * gm.y;
-            const float d10 = 2.f * (kb.x + gm.x * g1[2 * j] + bt.x - vb.x) * gm.x;
-            const float d11 = 2.f * (kb.y + gm.y * g1[2 * j + 1] + bt.y - vb.y) * gm.y;
+            const float2 gm = lds_f2(sbase + OFF_GAMMA + 4 * col);
+            const float2 bt = lds_f2(sbase + OFF_BETA + 4 * col);
+            d00 = 2.f * (ka.x + gm.x * xa0 + bt.x - va.x) * gm.x;
+            d01 = 2.f * (ka.y + gm.y * xa1 + bt.y - va.y) * gm.y;
+            d10 = 2.f * (kb.x + gm.x * xb0 + bt.x - vb.x) * gm.x;
+            d11 = 2.f * (kb.y + gm.y * xb1 + bt.y - vb.y) * gm.y;
+          };
+          float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float d00, d01, d10, d11;
+            dxhat(8 * j + 2 * q4, g0[2 * j], g0[2 * j + 1], g1[2 * j], g1[2 * j + 1], d00, d01, d10, d11);
             a0 += d00 + d01;
             a1 += d10 + d11;
             b0 += d00 * g0[2 * j] + d01 * g0[2 * j + 1];
@@ -336,34 +365,15 @@ __global__ void __launch_bounds__(THREADS, 4)
           const float mg0 = quad_sum(a0) * (1.f / D), mg1 = quad_sum(a1) * (1.f / D);
           const float mx0 = quad_sum(b0) * (1.f / D), mx1 = quad_sum(b1) * (1.f / D);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {  // second pass: recompute dx, finish dl/dy
+          for (int j = 0; j < 8; ++j) {  // second pass: recompute dx, finish and store
             const int col = 8 * j + 2 * q4;
-            const float2 ka = ld2(OFF_K, r0, col), kb = ld2(OFF_K, r1, col);
-            const float2 va = ld2(OFF_GLO, r0, col), vb = ld2(OFF_GLO, r1, col);
-            const float2 gm = *reinterpret_cast<const float2 *>(gam_s + col);
-            const float2 bt = *reinterpret_cast<const float2 *>(bet_s + col);
-            const float d00 = 2.f * (ka.x + gm.x * g0[2 * j] + bt.x - va.x) * gm.x;
-            const float d01 = 2.f * (ka.y + gm.y * g0[2 * j + 1] + bt.y - va.y) * gm.y;
-            const float d10 = 2.f * (kb.x + gm.x * g1[2 * j] + bt.x - vb.x) * gm.x;
-            const float d11 = 2.f * (kb.y + gm.y * g1[2 * j + 1] + bt.y - vb.y) * gm.y;
-            g0[2 * j] = rstd0 * (d00 - mg0 - g0[2 * j] * mx0);
-            g0[2 * j + 1] = rstd0 * (d01 - mg0 - g0[2 * j + 1] * mx0);
-            g1[2 * j] = rstd1 * (d10 - mg1 - g1[2 * j] * mx1);
-            g1[2 * j + 1] = rstd1 * (d11 - mg1 - g1[2 * j + 1] * mx1);
+            float d00, d01, d10, d11;
+            dxhat(col, g0[2 * j], g0[2 * j + 1], g1[2 * j], g1[2 * j + 1], d00, d01, d10, d11);
+            store_grad(col, rstd0 * (d00 - mg0 - g0[2 * j] * mx0),
+                       rstd0 * (d01 - mg0 - g0[2 * j + 1] * mx0),
+                       rstd1 * (d10 - mg1 - g1[2 * j] * mx1),
+                       rstd1 * (d11 - mg1 - g1[2 * j + 1] * mx1));
           }
-        }
-        // eta * G as bf16 hi + lo, in place of V for the lo half.
-        const float e0 = eta_s[r0], e1 = eta_s[r1];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          uint32_t h0, l0, h1, l1;
-          split_bf16x2(e0 * g0[2 * j], e0 * g0[2 * j + 1], h0, l0);
-          split_bf16x2(e1 * g1[2 * j], e1 * g1[2 * j + 1], h1, l1);
-          *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r0, col)) = h0;
-          *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r0, col)) = l0;
-          *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r1, col)) = h1;
-          *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r1, col)) = l1;
         }
         fence_proxy_async_smem();
         tc_fence_before_sync();
@@ -398,6 +408,7 @@ __global__ void __launch_bounds__(THREADS, 4)
     if (warp >= 2) {
       const int q4 = lane & 3;
       float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
+      const __nv_bfloat16 *Qc = p.Q + (tok_base + (size_t)c * CHUNK) * D;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         uint32_t zr[32];
@@ -433,21 +444,28 @@ __global__ void __launch_bounds__(THREADS, 4)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int col = 8 * j + 2 * q4;
-            const float2 qa = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + OFF_Q + sw128_offset(t0, col)));
-            const float2 qb = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(sm + OFF_Q + sw128_offset(t1, col)));
-            const float2 gm = *reinterpret_cast<const float2 *>(gam_s + col);
-            const float2 bt = *reinterpret_cast<const float2 *>(bet_s + col);
-            z0[2 * j] = qa.x + gm.x * (z0[2 * j] * rstd0) + bt.x;
-            z0[2 * j + 1] = qa.y + gm.y * (z0[2 * j + 1] * rstd0) + bt.y;
-            z1[2 * j] = qb.x + gm.x * (z1[2 * j] * rstd1) + bt.x;
-            z1[2 * j + 1] = qb.y + gm.y * (z1[2 * j + 1] * rstd1) + bt.y;
+            const float2 qa = t0 < ntok ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(Qc + t0 * D + col))
+                                        : make_float2(0.f, 0.f);
+            const float2 qb = t1 < ntok ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(Qc + t1 * D + col))
+                                        : make_float2(0.f, 0.f);
+            const float2 gm = lds_f2(smem_u32(sm) + OFF_GAMMA + 4 * col);
+            const float2 bt = lds_f2(smem_u32(sm) + OFF_BETA + 4 * col);
+            if (t0 < ntok)
+              *reinterpret_cast<float2 *>(Zc + t0 * D + col) =
+                  make_float2(qa.x + gm.x * (z0[2 * j] * rstd0) + bt.x,
+                              qa.y + gm.y * (z0[2 * j + 1] * rstd0) + bt.y);
+            if (t1 < ntok)
+              *reinterpret_cast<float2 *>(Zc + t1 * D + col) =
+                  make_float2(qb.x + gm.x * (z1[2 * j] * rstd1) + bt.x,
+                              qb.y + gm.y * (z1[2 * j + 1] * rstd1) + bt.y);
           }
-        }
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          if (t0 < ntok) *reinterpret_cast<float2 *>(Zc + t0 * D + col) = make_float2(z0[2 * j], z0[2 * j + 1]);
-          if (t1 < ntok) *reinterpret_cast<float2 *>(Zc + t1 * D + col) = make_float2(z1[2 * j], z1[2 * j + 1]);
+          for (int j = 0; j < 8; ++j) {
+            const int col = 8 * j + 2 * q4;
+            if (t0 < ntok) *reinterpret_cast<float2 *>(Zc + t0 * D + col) = make_float2(z0[2 * j], z0[2 * j + 1]);
+            if (t1 < ntok) *reinterpret_cast<float2 *>(Zc + t1 * D + col) = make_float2(z1[2 * j], z1[2 * j + 1]);
+          }
         }
       }
     }
@@ -455,6 +473,9 @@ __global__ void __launch_bounds__(THREADS, 4)
     // ---- 6: state update W -= dW and the next chunk's operand copy --------------
     wait_or_abort(&bars[BAR_DW], par, abort);
     tc_fence_after_sync();
+    // K, V (lo half of eta*G) and eta are free once dW is done; every thread passed
+    // this chunk's wait on their barrier before the A-operand barrier above.
+    if (tid == 0 && c + 1 < nchunks && !*abort) issue_loads_kv(c + 1);
     {
       uint32_t dw[32];
       tmem_ld_32x32b_x32(tmem_addr(tS, 32 * warp, wc0), dw);
@@ -468,7 +489,6 @@ __global__ void __launch_bounds__(THREADS, 4)
     __syncthreads();
     tc_fence_after_sync();
     if (*abort) break;
-    if (tid == 0 && c + 1 < nchunks) issue_loads(c + 1);
   }
 
   // Final state.

@@ -202,6 +202,7 @@ int launch_linear_tc(const Call &c) {
       !make_qkv_map(&mv, c.V, c.T, units))
     return TTT_ERR_CUDA;
   tc::Params p;
+  p.Q = static_cast<const __nv_bfloat16 *>(c.Q);
   p.eta = c.eta;
   p.W0 = c.W0;
   p.gamma = c.gamma;
