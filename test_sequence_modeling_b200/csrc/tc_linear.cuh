@@ -8,28 +8,29 @@
 // Work decomposition.  One CTA of 4 warps owns one (batch, head) sequence for
 // its whole length and keeps the fp32 state W in registers.  Tokens are taken
 // in chunks of 64 (four mini-batches), so that every tensor-core product has
-// M = 128 rows: the 64 K rows of the chunk stacked over its 64 Q rows.  With
-// W_c the state at the start of the chunk and G_m (m = 0..3) the gradients of
-// the loss w.r.t. the pre-activation of mini-batch m (taken at that mini-batch's
-// own base state), the state at the start of mini-batch m is
-//   W_m = W_c - sum_{j<m} K_j^T diag(eta_j) G_j,
-// so that, exactly,
+// M = 128 rows: the 64 K rows and the 64 Q rows of the chunk, interleaved by
+// mini-batch as [K0; Q0; K1; Q1; K2; Q2; K3; Q3] (16 rows each).  TMEM lane =
+// operand row, so warp m (which can read TMEM lanes 32m..32m+31) holds exactly
+// the K and Q rows of mini-batch m.  With W_c the state at the start of the
+// chunk and G_m the gradient of the loss w.r.t. the pre-activation of
+// mini-batch m (taken at that mini-batch's own base state), the state at the
+// start of mini-batch m is W_m = W_c - sum_{j<m} K_j^T diag(eta_j) G_j, so that
 //   K_m W_m = (K W_c)_m - sum_{j<m} (K_m K_j^T) diag(eta_j) G_j
-//   Q_t W_t = (Q W_c)_t - sum_{s<=t} (q_t . k_s) eta_s G_s    (the dual-form output)
+//   q_t W_t = (Q W_c)_t - sum_{s<=t} (q_t . k_s) eta_s G_s    (dual-form output)
 //   W_next  = W_c - K^T diag(eta) G.
 // Per chunk:
-//   1. TMA: K, Q (64 x 64 bf16 each, 128-byte swizzle) and V, eta.
-//   2. tcgen05: P = [K; Q] W_c (TMEM cols 0..63) and S = [K; Q] K^T (cols 64..127).
+//   1. TMA: K and Q (16-row boxes into the interleaved operand, 128-byte
+//      swizzle), V, eta.
+//   2. tcgen05: P = [K;Q] W_c (TMEM cols 0..63), S = [K;Q] K^T (cols 64..127).
 //   3. Every thread masks its own row of S in TMEM into the A operand of step 4:
 //      K rows keep the columns of earlier mini-batches, Q rows keep s <= t (the
-//      causal mask of the dual form, diagonal included), stored as bf16 hi + lo.
-//   4. For m = 0..3: the warp owning mini-batch m reads its 16 rows of P (already
-//      corrected for mini-batches < m), computes G_m (LN backward fused in
-//      registers), writes eta*G_m as bf16 hi + lo, and issues
-//      P -= A[:, m] (eta G_m) on the tensor core, which applies mini-batch m's
-//      update to every later K row and to every Q row at once.
-//   5. After the last mini-batch the Q rows of P hold Q W - tril(Q K^T) diag(eta) G:
-//      warps 2-3 apply LN + residual and store Z while the tensor core computes
+//      causal mask of the dual form, diagonal included), as bf16 hi + lo.
+//   4. For m = 0..3, warp m: reads its 16 K rows of P (already corrected for
+//      mini-batches < m), computes G_m (LN backward in registers), writes
+//      eta*G_m as bf16 hi + lo, and issues P -= A[:, m] (eta G_m), which applies
+//      mini-batch m's update to every later K row and every Q row at once.
+//   5. Then the Q rows of P hold Q W - tril(Q K^T) diag(eta) G: each warp applies
+//      LN + residual to its 16 Q rows and stores Z while the tensor core computes
 //      dW = K^T (eta G); every thread then updates its 32 fp32 state elements and
 //      rewrites the bf16 hi + lo operand copy of W for the next chunk.
 // Precision: every fp32 operand (W, eta*G, the masked Q K^T) enters the tensor
@@ -56,22 +57,26 @@ constexpr int THREADS = 128;
 constexpr uint32_t TMEM_COLS = 128;
 
 // Shared-memory map (bytes from a 1024-byte aligned base).
-constexpr uint32_t OFF_K = 0;         // K tile [64][64] bf16, 128B swizzle
-constexpr uint32_t OFF_Q = 8192;      // Q tile, directly after K: [K; Q] is one 128-row operand
-constexpr uint32_t OFF_WHI = 16384;   // W hi [d_in][d_out] bf16
-constexpr uint32_t OFF_WLO = 24576;   // W lo
-constexpr uint32_t OFF_GHI = 32768;   // eta*G hi [token][d_out] bf16
-constexpr uint32_t OFF_GLO = 40960;   // V tile on arrival; eta*G lo once mini-batch m is done
-constexpr uint32_t OFF_ETA = 49152;   // eta of the chunk, 64 floats
-constexpr uint32_t OFF_GAMMA = 49408; // LN gamma, 64 floats
-constexpr uint32_t OFF_BETA = 49664;  // LN beta, 64 floats
-constexpr uint32_t OFF_BAR = 49920;   // mbarriers
-constexpr uint32_t OFF_TSLOT = 49984; // TMEM base address
-constexpr uint32_t OFF_ABORT = 49988; // set when a bounded wait expired
-constexpr uint32_t SMEM_USED = 50000;
+constexpr uint32_t OFF_A = 0;          // [K0;Q0;K1;Q1;K2;Q2;K3;Q3], 16 rows x 128 B each
+constexpr uint32_t OFF_WHI = 16384;    // W hi [d_in][d_out] bf16
+constexpr uint32_t OFF_WLO = 24576;    // W lo
+constexpr uint32_t OFF_GHI = 32768;    // eta*G hi [token][d_out] bf16
+constexpr uint32_t OFF_GLO = 40960;    // V tile on arrival; eta*G lo once a mini-batch is done
+constexpr uint32_t OFF_ETA = 49152;    // eta of the chunk, 64 floats
+constexpr uint32_t OFF_GAMMA = 49408;  // LN gamma, 64 floats
+constexpr uint32_t OFF_BETA = 49664;   // LN beta, 64 floats
+constexpr uint32_t OFF_W2 = 49920;     // 2 gamma^2, 64 floats
+constexpr uint32_t OFF_BAR = 50176;    // mbarriers
+constexpr uint32_t OFF_TSLOT = 50240;  // TMEM base address
+constexpr uint32_t OFF_ABORT = 50244;  // set when a bounded wait expired
+constexpr uint32_t SMEM_USED = 50256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
-// mbarriers: K/V/eta loads; Q load; MMA P,S; mini-batch 0,1,2 updates; last update; dW.
+__host__ __device__ constexpr uint32_t k_block(int m) { return OFF_A + 4096u * m; }
+__host__ __device__ constexpr uint32_t q_block(int m) { return OFF_A + 4096u * m + 2048u; }
+
+// mbarriers: K/V/eta loads; MMA P,S; updates of mini-batches 0,1,2; last update;
+// dW; Q loads.
 enum { BAR_LOAD = 0, BAR_PS = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, BAR_LOADQ = 7, NUM_BARS = 8 };
 
 struct Params {
@@ -84,6 +89,16 @@ struct Params {
   float *Z;
   float *W_out;
 };
+
+// Sum of 16 values as a balanced tree (independent adds for instruction-level parallelism).
+__device__ __forceinline__ float tree_sum16(const float (&x)[16]) {
+  float a[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = x[2 * i] + x[2 * i + 1];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) a[i] += a[i + 4];
+  return (a[0] + a[2]) + (a[1] + a[3]);
+}
 
 __device__ __forceinline__ float quad_sum(float x) {
   x += __shfl_xor_sync(0xffffffffu, x, 1);
@@ -116,11 +131,10 @@ __global__ void __launch_bounds__(THREADS, 4)
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_TSLOT);
   volatile int *abort = reinterpret_cast<volatile int *>(sm + OFF_ABORT);
   float *eta_s = reinterpret_cast<float *>(sm + OFF_ETA);
-  float *gam_s = reinterpret_cast<float *>(sm + OFF_GAMMA);
-  float *bet_s = reinterpret_cast<float *>(sm + OFF_BETA);
-  const uint32_t aK = smem_u32(sm + OFF_K);
-  const uint32_t aWhi = smem_u32(sm + OFF_WHI), aWlo = smem_u32(sm + OFF_WLO);
-  const uint32_t aGhi = smem_u32(sm + OFF_GHI), aGlo = smem_u32(sm + OFF_GLO);
+  const uint32_t sbase = smem_u32(sm);
+  const uint32_t aA = sbase + OFF_A;
+  const uint32_t aWhi = sbase + OFF_WHI, aWlo = sbase + OFF_WLO;
+  const uint32_t aGhi = sbase + OFF_GHI, aGlo = sbase + OFF_GLO;
 
   if (tid == 0) {
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], 1);
@@ -135,8 +149,10 @@ __global__ void __launch_bounds__(THREADS, 4)
     tmem_relinquish();
   }
   if (LN && tid < D) {
-    gam_s[tid] = p.gamma[head * D + tid];
-    bet_s[tid] = p.beta[head * D + tid];
+    const float g = p.gamma[head * D + tid];
+    reinterpret_cast<float *>(sm + OFF_GAMMA)[tid] = g;
+    reinterpret_cast<float *>(sm + OFF_BETA)[tid] = p.beta[head * D + tid];
+    reinterpret_cast<float *>(sm + OFF_W2)[tid] = 2.f * g * g;
   }
 
   // Each thread owns 32 elements of the fp32 state: row wi, columns wc0..wc0+31.
@@ -175,14 +191,16 @@ __global__ void __launch_bounds__(THREADS, 4)
   // Q once P and S are computed, K / V / eta once dW is computed.
   auto issue_loads_kv = [&](int c) {
     const int ntok = min(CHUNK, T - c * CHUNK);
-    mbar_arrive_expect_tx(&bars[BAR_LOAD], 2u * 8192u + (uint32_t)ntok * 4u);
-    tma_load_3d(sm + OFF_K, &tmK, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
+    mbar_arrive_expect_tx(&bars[BAR_LOAD], 4u * 2048u + 8192u + (uint32_t)ntok * 4u);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tma_load_3d(sm + k_block(m), &tmK, 0, c * CHUNK + MB * m, unit, &bars[BAR_LOAD]);
     tma_load_3d(sm + OFF_GLO, &tmV, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
     bulk_load(eta_s, p.eta + tok_base + (size_t)c * CHUNK, (uint32_t)ntok * 4u, &bars[BAR_LOAD]);
   };
   auto issue_load_q = [&](int c) {
-    mbar_arrive_expect_tx(&bars[BAR_LOADQ], 8192u);
-    tma_load_3d(sm + OFF_Q, &tmQ, 0, c * CHUNK, unit, &bars[BAR_LOADQ]);
+    mbar_arrive_expect_tx(&bars[BAR_LOADQ], 4u * 2048u);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) tma_load_3d(sm + q_block(m), &tmQ, 0, c * CHUNK + MB * m, unit, &bars[BAR_LOADQ]);
   };
 
   fence_proxy_async_smem();
@@ -196,33 +214,38 @@ __global__ void __launch_bounds__(THREADS, 4)
     issue_load_q(0);
   }
 
-  constexpr uint32_t ID_PW = idesc_bf16_f32(128, 64, false, true, false);   // [K;Q] x W
-  constexpr uint32_t ID_S = idesc_bf16_f32(128, 64, false, false, false);   // [K;Q] x K^T
-  constexpr uint32_t ID_UPD = idesc_bf16_f32(128, 64, false, true, true);   // P -= A x (eta G)
-  constexpr uint32_t ID_DW = idesc_bf16_f32(128, 64, true, true, false);    // [K^T;K^T] x (eta G)
+  constexpr uint32_t ID_PW = idesc_bf16_f32(128, 64, false, true, false);  // [K;Q] x W
+  constexpr uint32_t ID_S = idesc_bf16_f32(128, 16, false, false, false);  // [K;Q] x K_m^T
+  constexpr uint32_t ID_UPD = idesc_bf16_f32(128, 64, false, true, true);  // P -= A x (eta G)
+  constexpr uint32_t ID_DW = idesc_bf16_f32(128, 64, true, true, false);   // [K^T;K^T] x (eta G)
+
+  const int q4 = lane & 3;
+  const int fr = lane >> 2;  // row within a 16-row group (and +8) in the 16x256b layout
 
   for (int c = 0; c < nchunks; ++c) {
     const int ntok = min(CHUNK, T - c * CHUNK);
     const int nmb = ntok / MB;
     const uint32_t par = (uint32_t)c & 1u;
 
-    // ---- 1-2: tiles in, P = [K;Q] W and S = [K;Q] K^T ----------------------------
+    // ---- 1-2: tiles in, P = [K;Q] W and S = [K;Q] K^T ------------------------------
     wait_or_abort(&bars[BAR_LOAD], par, abort);
     wait_or_abort(&bars[BAR_LOADQ], par, abort);
     if (tid == 0 && !*abort) {
       tc_fence_after_sync();
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        umma_ss(tP, smem_desc_sw128(aK + 32 * k, 16, 1024), smem_desc_sw128(aWhi + 2048 * k, 8192, 1024),
+        umma_ss(tP, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aWhi + 2048 * k, 8192, 1024),
                 ID_PW, k > 0);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        umma_ss(tP, smem_desc_sw128(aK + 32 * k, 16, 1024), smem_desc_sw128(aWlo + 2048 * k, 8192, 1024),
+        umma_ss(tP, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aWlo + 2048 * k, 8192, 1024),
                 ID_PW, true);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        umma_ss(tS, smem_desc_sw128(aK + 32 * k, 16, 1024), smem_desc_sw128(aK + 32 * k, 16, 1024),
-                ID_S, k > 0);
+      for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_ss(tS + 16 * n, smem_desc_sw128(aA + 32 * k, 16, 1024),
+                  smem_desc_sw128(sbase + k_block(n) + 32 * k, 16, 1024), ID_S, k > 0);
       umma_commit(&bars[BAR_PS]);
     }
     if (ntok < CHUNK) {  // ragged last chunk: absent tokens contribute nothing to dW
@@ -234,32 +257,42 @@ __global__ void __launch_bounds__(THREADS, 4)
     }
     wait_or_abort(&bars[BAR_PS], par, abort);
     tc_fence_after_sync();
+    __syncwarp();  // lanes leave the wait loop independently; TMEM access is warp-collective
 
-    // ---- 3: mask this thread's row of S into the A operand (in place, per block) ----
+    // ---- 3: mask this thread's row of S into the A operand (in place, per block) ------
     {
-      const int r = 32 * warp + lane;  // TMEM lane = row: K rows 0..63, Q rows 64..127
+      const bool qrow = lane >= 16;
+      const int t = MB * warp + (lane & 15);  // token of this row within the chunk
+      // Column blocks j > warp are zero for every row of this warp (K rows keep
+      // blocks < warp, Q rows blocks <= warp); TMEM loads and stores are
+      // warp-collective, so the skip is decided per warp.
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem_addr(tS, 32 * warp, 16 * j), v);
-        tmem_wait_ld();
-        uint32_t hi[8], lo[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int s0 = 16 * j + 2 * e;
-          bool keep0, keep1;
-          if (r < CHUNK) {
-            keep0 = keep1 = j < (r >> 4);  // earlier mini-batches only
-          } else {
-            keep0 = s0 <= r - CHUNK;  // causal, diagonal included
-            keep1 = s0 + 1 <= r - CHUNK;
-          }
-          const float a = keep0 ? __uint_as_float(v[2 * e]) : 0.f;
-          const float b = keep1 ? __uint_as_float(v[2 * e + 1]) : 0.f;
-          split_bf16x2(a, b, hi[e], lo[e]);
+      for (int jj = 0; jj < 2; ++jj) {
+        uint32_t v[32];
+        if (2 * jj <= warp) {
+          tmem_ld_32x32b_x32(tmem_addr(tS, 32 * warp, 32 * jj), v);
+          tmem_wait_ld();
         }
-        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j), hi);
-        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j + 8), lo);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int j = 2 * jj + h;
+          uint32_t hi[8], lo[8];
+          const bool all_zero = qrow ? (j > warp) : (j >= warp);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int s0 = MB * j + 2 * e;
+            const float a = (!all_zero && (!qrow || s0 <= t)) ? __uint_as_float(v[16 * h + 2 * e]) : 0.f;
+            const float b = (!all_zero && (!qrow || s0 + 1 <= t)) ? __uint_as_float(v[16 * h + 2 * e + 1]) : 0.f;
+            split_bf16x2(a, b, hi[e], lo[e]);
+          }
+          if (j <= warp) {
+            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j), hi);
+            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j + 8), lo);
+          } else {
+            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j), hi);  // zeros
+            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j + 8), hi);
+          }
+        }
       }
       tmem_wait_st();
     }
@@ -267,212 +300,238 @@ __global__ void __launch_bounds__(THREADS, 4)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
-    // The Q buffer is free (P and S are done).  Issued only after this barrier:
-    // every thread has then passed its wait on this chunk's Q phase, so the Q
-    // barrier cannot complete twice while a thread still waits on it.
-    if (tid == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
 
-    // ---- 4: the mini-batch chain (warp 0: mini-batches 0-1, warp 1: 2-3) ---------
-    if (warp < 2) {
-      const int q4 = lane & 3;
-#pragma unroll 1
-      for (int m = 2 * warp; m < 2 * warp + 2 && m < nmb; ++m) {
-        if (m > 0) wait_or_abort(&bars[BAR_C0 + m - 1], par, abort);
-        tc_fence_after_sync();
-        uint32_t yr[32];
-        tmem_ld_16x256b_x8(tmem_addr(tP, 32 * warp + 16 * (m & 1), 0), yr);
-        tmem_wait_ld();
-        const int r0 = 16 * m + (lane >> 2), r1 = r0 + 8;
-        float g0[16], g1[16];  // y = the P rows, then the gradient w.r.t. y
+    // ---- 4: the mini-batch chain: warp m handles mini-batch m ------------------------
+    if (warp < nmb) {
+      const int m = warp;
+      const int r0 = MB * m + fr, r1 = r0 + 8;  // tokens of this thread's two rows
+      const uint32_t kb = sbase + k_block(m);
+      // Everything of the LN backward that does not depend on P, computed before
+      // waiting for the previous mini-batch: u = 2 gamma (k + beta - v), its mean.
+      float u0[16], u1[16];
+      float um0 = 0.f, um1 = 0.f;
+      if (LN) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          g0[2 * j] = __uint_as_float(yr[4 * j + 0]);
-          g0[2 * j + 1] = __uint_as_float(yr[4 * j + 1]);
-          g1[2 * j] = __uint_as_float(yr[4 * j + 2]);
-          g1[2 * j + 1] = __uint_as_float(yr[4 * j + 3]);
+          const int col = 8 * j + 2 * q4;
+          const float2 ka = unpack_bf16x2(lds_u32(kb + sw128_offset(fr, col)));
+          const float2 kc = unpack_bf16x2(lds_u32(kb + sw128_offset(fr + 8, col)));
+          const float2 va = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r0, col)));
+          const float2 vc = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r1, col)));
+          const float2 gm = lds_f2(sbase + OFF_GAMMA + 4 * col);
+          const float2 bt = lds_f2(sbase + OFF_BETA + 4 * col);
+          u0[2 * j] = 2.f * gm.x * (ka.x + bt.x - va.x);
+          u0[2 * j + 1] = 2.f * gm.y * (ka.y + bt.y - va.y);
+          u1[2 * j] = 2.f * gm.x * (kc.x + bt.x - vc.x);
+          u1[2 * j + 1] = 2.f * gm.y * (kc.y + bt.y - vc.y);
+          um0 += u0[2 * j] + u0[2 * j + 1];
+          um1 += u1[2 * j] + u1[2 * j + 1];
         }
-        const uint32_t sbase = smem_u32(sm);
-        auto ld2 = [&](uint32_t off, int row, int col) {
-          return unpack_bf16x2(lds_u32(sbase + off + sw128_offset(row, col)));
-        };
-        const float e0 = eta_s[r0], e1 = eta_s[r1];
-        // Stores eta * (dl/dy) of one column pair of both rows as bf16 hi + lo; the
-        // lo half overwrites V, which this thread has read for exactly these cells.
-        auto store_grad = [&](int col, float ga0, float ga1, float gb0, float gb1) {
-          uint32_t h0, l0, h1, l1;
-          split_bf16x2(e0 * ga0, e0 * ga1, h0, l0);
-          split_bf16x2(e1 * gb0, e1 * gb1, h1, l1);
-          *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r0, col)) = h0;
-          *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r0, col)) = l0;
-          *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r1, col)) = h1;
-          *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r1, col)) = l1;
-        };
-        if (!LN) {
+        um0 = quad_sum(um0) * (1.f / D);
+        um1 = quad_sum(um1) * (1.f / D);
+      } else {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int col = 8 * j + 2 * q4;
-            const float2 va = ld2(OFF_GLO, r0, col), vb = ld2(OFF_GLO, r1, col);
-            store_grad(col, 2.f * (g0[2 * j] - va.x), 2.f * (g0[2 * j + 1] - va.y),
-                       2.f * (g1[2 * j] - vb.x), 2.f * (g1[2 * j + 1] - vb.y));
-          }
-        } else {
-          // LN backward of ||k + gamma*xhat + beta - v||^2 w.r.t. y: with
-          // dx = dl/dxhat = 2 (k + gamma xhat + beta - v) gamma,
-          // dl/dy = rstd (dx - mean(dx) - xhat mean(dx xhat)).
-          float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            s0 += g0[e];
-            s1 += g1[e];
-          }
-          const float mean0 = quad_sum(s0) * (1.f / D), mean1 = quad_sum(s1) * (1.f / D);
-          float q0 = 0.f, q1 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            g0[e] -= mean0;
-            g1[e] -= mean1;
-            q0 += g0[e] * g0[e];
-            q1 += g1[e] * g1[e];
-          }
-          const float rstd0 = rsqrtf(quad_sum(q0) * (1.f / D) + p.eps);
-          const float rstd1 = rsqrtf(quad_sum(q1) * (1.f / D) + p.eps);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            g0[e] *= rstd0;  // xhat
-            g1[e] *= rstd1;
-          }
-          auto dxhat = [&](int col, float xa0, float xa1, float xb0, float xb1, float &d00,
-                           float &d01, float &d10, float &d11) {
-            const float2 ka = ld2(OFF_K, r0, col), kb = ld2(OFF_K, r1, col);
-            const float2 va = ld2(OFF_GLO, r0, col), vb = ld2(OFF_GLO, r1, col);
-            const float2 gm = lds_f2(sbase + OFF_GAMMA + 4 * col);
-            const float2 bt = lds_f2(sbase + OFF_BETA + 4 * col);
-            d00 = 2.f * (ka.x + gm.x * xa0 + bt.x - va.x) * gm.x;
-            d01 = 2.f * (ka.y + gm.y * xa1 + bt.y - va.y) * gm.y;
-            d10 = 2.f * (kb.x + gm.x * xb0 + bt.x - vb.x) * gm.x;
-            d11 = 2.f * (kb.y + gm.y * xb1 + bt.y - vb.y) * gm.y;
-          };
-          float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float d00, d01, d10, d11;
-            dxhat(8 * j + 2 * q4, g0[2 * j], g0[2 * j + 1], g1[2 * j], g1[2 * j + 1], d00, d01, d10, d11);
-            a0 += d00 + d01;
-            a1 += d10 + d11;
-            b0 += d00 * g0[2 * j] + d01 * g0[2 * j + 1];
-            b1 += d10 * g1[2 * j] + d11 * g1[2 * j + 1];
-          }
-          const float mg0 = quad_sum(a0) * (1.f / D), mg1 = quad_sum(a1) * (1.f / D);
-          const float mx0 = quad_sum(b0) * (1.f / D), mx1 = quad_sum(b1) * (1.f / D);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {  // second pass: recompute dx, finish and store
-            const int col = 8 * j + 2 * q4;
-            float d00, d01, d10, d11;
-            dxhat(col, g0[2 * j], g0[2 * j + 1], g1[2 * j], g1[2 * j + 1], d00, d01, d10, d11);
-            store_grad(col, rstd0 * (d00 - mg0 - g0[2 * j] * mx0),
-                       rstd0 * (d01 - mg0 - g0[2 * j + 1] * mx0),
-                       rstd1 * (d10 - mg1 - g1[2 * j] * mx1),
-                       rstd1 * (d11 - mg1 - g1[2 * j + 1] * mx1));
-          }
+        for (int j = 0; j < 8; ++j) {
+          const int col = 8 * j + 2 * q4;
+          const float2 va = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r0, col)));
+          const float2 vc = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r1, col)));
+          u0[2 * j] = va.x;
+          u0[2 * j + 1] = va.y;
+          u1[2 * j] = vc.x;
+          u1[2 * j + 1] = vc.y;
         }
-        fence_proxy_async_smem();
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0 && !*abort) {
-          tc_fence_after_sync();
-          const uint64_t bhi = smem_desc_sw128(aGhi + 2048 * m, 8192, 1024);
-          const uint64_t blo = smem_desc_sw128(aGlo + 2048 * m, 8192, 1024);
-          umma_ts(tP, tS + 16 * m, bhi, ID_UPD, true);
-          umma_ts(tP, tS + 16 * m, blo, ID_UPD, true);
-          umma_ts(tP, tS + 16 * m + 8, bhi, ID_UPD, true);
-          umma_commit(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
-        }
-        __syncwarp();
       }
+      const float e0 = eta_s[r0], e1 = eta_s[r1];
+
+      if (m > 0) wait_or_abort(&bars[BAR_C0 + m - 1], par, abort);
+      tc_fence_after_sync();
+      __syncwarp();
+      uint32_t yr[32];
+      tmem_ld_16x256b_x8(tmem_addr(tP, 32 * m, 0), yr);
+      tmem_wait_ld();
+      float y0[16], y1[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        y0[2 * j] = __uint_as_float(yr[4 * j + 0]);
+        y0[2 * j + 1] = __uint_as_float(yr[4 * j + 1]);
+        y1[2 * j] = __uint_as_float(yr[4 * j + 2]);
+        y1[2 * j + 1] = __uint_as_float(yr[4 * j + 3]);
+      }
+      // Stores eta * (dl/dy) of one column pair of both rows as bf16 hi + lo; the
+      // lo half overwrites V, which this thread has read for exactly these cells.
+      auto store_grad = [&](int col, float ga0, float ga1, float gb0, float gb1) {
+        uint32_t h0, l0, h1, l1;
+        split_bf16x2(ga0, ga1, h0, l0);
+        split_bf16x2(gb0, gb1, h1, l1);
+        *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r0, col)) = h0;
+        *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r0, col)) = l0;
+        *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r1, col)) = h1;
+        *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r1, col)) = l1;
+      };
+      if (!LN) {
+        // dl/dy = 2 (y - v)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          store_grad(8 * j + 2 * q4, 2.f * e0 * (y0[2 * j] - u0[2 * j]),
+                     2.f * e0 * (y0[2 * j + 1] - u0[2 * j + 1]), 2.f * e1 * (y1[2 * j] - u1[2 * j]),
+                     2.f * e1 * (y1[2 * j + 1] - u1[2 * j + 1]));
+      } else {
+        // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y.  With
+        // dx = dl/dxhat = u + w xhat (w = 2 gamma^2), A = mean(dx), B = mean(dx xhat):
+        // dl/dy = rstd (dx - A - xhat B) = rstd (u + xhat (w - B) - A).
+        const float mean0 = quad_sum(tree_sum16(y0)) * (1.f / D);
+        const float mean1 = quad_sum(tree_sum16(y1)) * (1.f / D);
+        float sq0[16], sq1[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          y0[e] -= mean0;
+          y1[e] -= mean1;
+          sq0[e] = y0[e] * y0[e];
+          sq1[e] = y1[e] * y1[e];
+        }
+        const float v0 = tree_sum16(sq0), v1 = tree_sum16(sq1);
+        const float rstd0 = rsqrtf(quad_sum(v0) * (1.f / D) + p.eps);
+        const float rstd1 = rsqrtf(quad_sum(v1) * (1.f / D) + p.eps);
+        float wx0 = 0.f, wx1 = 0.f, ux0 = 0.f, ux1 = 0.f, wxx0 = 0.f, wxx1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 w2 = lds_f2(sbase + OFF_W2 + 4 * (8 * j + 2 * q4));
+          const float wv[2] = {w2.x, w2.y};
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int e = 2 * j + h;
+            const float xa = y0[e] * rstd0, xb = y1[e] * rstd1;
+            y0[e] = xa;
+            y1[e] = xb;
+            wx0 = fmaf(wv[h], xa, wx0);
+            wx1 = fmaf(wv[h], xb, wx1);
+            ux0 = fmaf(u0[e], xa, ux0);
+            ux1 = fmaf(u1[e], xb, ux1);
+            wxx0 = fmaf(wv[h] * xa, xa, wxx0);
+            wxx1 = fmaf(wv[h] * xb, xb, wxx1);
+          }
+        }
+        const float A0 = um0 + quad_sum(wx0) * (1.f / D), A1 = um1 + quad_sum(wx1) * (1.f / D);
+        const float B0 = (quad_sum(ux0) + quad_sum(wxx0)) * (1.f / D);
+        const float B1 = (quad_sum(ux1) + quad_sum(wxx1)) * (1.f / D);
+        const float f0 = e0 * rstd0, f1 = e1 * rstd1;  // eta folded into the scale
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 w2 = lds_f2(sbase + OFF_W2 + 4 * (8 * j + 2 * q4));
+          store_grad(8 * j + 2 * q4, f0 * (fmaf(y0[2 * j], w2.x - B0, u0[2 * j]) - A0),
+                     f0 * (fmaf(y0[2 * j + 1], w2.y - B0, u0[2 * j + 1]) - A0),
+                     f1 * (fmaf(y1[2 * j], w2.x - B1, u1[2 * j]) - A1),
+                     f1 * (fmaf(y1[2 * j + 1], w2.y - B1, u1[2 * j + 1]) - A1));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0 && !*abort) {
+        tc_fence_after_sync();
+        const uint64_t bhi = smem_desc_sw128(aGhi + 2048 * m, 8192, 1024);
+        const uint64_t blo = smem_desc_sw128(aGlo + 2048 * m, 8192, 1024);
+        umma_ts(tP, tS + 16 * m, bhi, ID_UPD, true);
+        umma_ts(tP, tS + 16 * m, blo, ID_UPD, true);
+        umma_ts(tP, tS + 16 * m + 8, bhi, ID_UPD, true);
+        umma_commit(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
+      }
+      __syncwarp();
     }
 
-    // ---- 5: the last update done -> dW on the tensor core, output on CUDA cores ----
+    // This warp's Q rows, kept in registers for the residual of the output; then
+    // the Q buffer is refilled with the next chunk.  The prefetch is issued after a
+    // CTA-wide barrier: every thread has then read its Q rows and passed its wait
+    // on this chunk's Q phase (so that phase cannot be overtaken).
+    uint32_t qres[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int col = 8 * j + 2 * q4;
+      qres[2 * j] = lds_u32(sbase + q_block(warp) + sw128_offset(fr, col));
+      qres[2 * j + 1] = lds_u32(sbase + q_block(warp) + sw128_offset(fr + 8, col));
+    }
+    named_barrier_sync(1, THREADS);
+    if (tid == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
+
+    // ---- 5: the last update done -> dW on the tensor core, output on CUDA cores --------
     wait_or_abort(&bars[BAR_LAST], par, abort);
     tc_fence_after_sync();
+    __syncwarp();
     if (tid == 0 && !*abort) {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        umma_ss(tS, smem_desc_sw128(aK + 2048 * k, 0, 1024), smem_desc_sw128(aGhi + 2048 * k, 8192, 1024),
+        umma_ss(tS, smem_desc_sw128(sbase + k_block(k), 0, 1024), smem_desc_sw128(aGhi + 2048 * k, 8192, 1024),
                 ID_DW, k > 0);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        umma_ss(tS, smem_desc_sw128(aK + 2048 * k, 0, 1024), smem_desc_sw128(aGlo + 2048 * k, 8192, 1024),
+        umma_ss(tS, smem_desc_sw128(sbase + k_block(k), 0, 1024), smem_desc_sw128(aGlo + 2048 * k, 8192, 1024),
                 ID_DW, true);
       umma_commit(&bars[BAR_DW]);
     }
-    if (warp >= 2) {
-      const int q4 = lane & 3;
+    {
+      // Q rows of mini-batch `warp`: lanes 32 warp + 16 .. +31.
+      uint32_t zr[32];
+      tmem_ld_16x256b_x8(tmem_addr(tP, 32 * warp + 16, 0), zr);
+      tmem_wait_ld();
+      const int t0 = MB * warp + fr, t1 = t0 + 8;
+      float z0[16], z1[16];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        z0[2 * j] = __uint_as_float(zr[4 * j + 0]);
+        z0[2 * j + 1] = __uint_as_float(zr[4 * j + 1]);
+        z1[2 * j] = __uint_as_float(zr[4 * j + 2]);
+        z1[2 * j + 1] = __uint_as_float(zr[4 * j + 3]);
+      }
       float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
-      const __nv_bfloat16 *Qc = p.Q + (tok_base + (size_t)c * CHUNK) * D;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        uint32_t zr[32];
-        tmem_ld_16x256b_x8(tmem_addr(tP, 32 * warp + 16 * h, 0), zr);
-        tmem_wait_ld();
-        const int t0 = 32 * (warp - 2) + 16 * h + (lane >> 2), t1 = t0 + 8;
-        float z0[16], z1[16];
+      const bool ok0 = t0 < ntok, ok1 = t1 < ntok;
+      if (LN) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          s0 += z0[e];
+          s1 += z1[e];
+        }
+        const float mean0 = quad_sum(s0) * (1.f / D), mean1 = quad_sum(s1) * (1.f / D);
+        float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          z0[e] -= mean0;
+          z1[e] -= mean1;
+          v0 += z0[e] * z0[e];
+          v1 += z1[e] * z1[e];
+        }
+        const float rstd0 = rsqrtf(quad_sum(v0) * (1.f / D) + p.eps);
+        const float rstd1 = rsqrtf(quad_sum(v1) * (1.f / D) + p.eps);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          z0[2 * j] = __uint_as_float(zr[4 * j + 0]);
-          z0[2 * j + 1] = __uint_as_float(zr[4 * j + 1]);
-          z1[2 * j] = __uint_as_float(zr[4 * j + 2]);
-          z1[2 * j + 1] = __uint_as_float(zr[4 * j + 3]);
+          const int col = 8 * j + 2 * q4;
+          const float2 gm = lds_f2(sbase + OFF_GAMMA + 4 * col);
+          const float2 bt = lds_f2(sbase + OFF_BETA + 4 * col);
+          if (ok0) {
+            const float2 qa = unpack_bf16x2(qres[2 * j]);
+            *reinterpret_cast<float2 *>(Zc + t0 * D + col) =
+                make_float2(qa.x + fmaf(gm.x, z0[2 * j] * rstd0, bt.x), qa.y + fmaf(gm.y, z0[2 * j + 1] * rstd0, bt.y));
+          }
+          if (ok1) {
+            const float2 qb = unpack_bf16x2(qres[2 * j + 1]);
+            *reinterpret_cast<float2 *>(Zc + t1 * D + col) =
+                make_float2(qb.x + fmaf(gm.x, z1[2 * j] * rstd1, bt.x), qb.y + fmaf(gm.y, z1[2 * j + 1] * rstd1, bt.y));
+          }
         }
-        if (LN) {
-          float s0 = 0.f, s1 = 0.f;
+      } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            s0 += z0[e];
-            s1 += z1[e];
-          }
-          const float mean0 = quad_sum(s0) * (1.f / D), mean1 = quad_sum(s1) * (1.f / D);
-          float q0 = 0.f, q1 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            z0[e] -= mean0;
-            z1[e] -= mean1;
-            q0 += z0[e] * z0[e];
-            q1 += z1[e] * z1[e];
-          }
-          const float rstd0 = rsqrtf(quad_sum(q0) * (1.f / D) + p.eps);
-          const float rstd1 = rsqrtf(quad_sum(q1) * (1.f / D) + p.eps);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int col = 8 * j + 2 * q4;
-            const float2 qa = t0 < ntok ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(Qc + t0 * D + col))
-                                        : make_float2(0.f, 0.f);
-            const float2 qb = t1 < ntok ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(Qc + t1 * D + col))
-                                        : make_float2(0.f, 0.f);
-            const float2 gm = lds_f2(smem_u32(sm) + OFF_GAMMA + 4 * col);
-            const float2 bt = lds_f2(smem_u32(sm) + OFF_BETA + 4 * col);
-            if (t0 < ntok)
-              *reinterpret_cast<float2 *>(Zc + t0 * D + col) =
-                  make_float2(qa.x + gm.x * (z0[2 * j] * rstd0) + bt.x,
-                              qa.y + gm.y * (z0[2 * j + 1] * rstd0) + bt.y);
-            if (t1 < ntok)
-              *reinterpret_cast<float2 *>(Zc + t1 * D + col) =
-                  make_float2(qb.x + gm.x * (z1[2 * j] * rstd1) + bt.x,
-                              qb.y + gm.y * (z1[2 * j + 1] * rstd1) + bt.y);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int col = 8 * j + 2 * q4;
-            if (t0 < ntok) *reinterpret_cast<float2 *>(Zc + t0 * D + col) = make_float2(z0[2 * j], z0[2 * j + 1]);
-            if (t1 < ntok) *reinterpret_cast<float2 *>(Zc + t1 * D + col) = make_float2(z1[2 * j], z1[2 * j + 1]);
-          }
+        for (int j = 0; j < 8; ++j) {
+          const int col = 8 * j + 2 * q4;
+          if (ok0) *reinterpret_cast<float2 *>(Zc + t0 * D + col) = make_float2(z0[2 * j], z0[2 * j + 1]);
+          if (ok1) *reinterpret_cast<float2 *>(Zc + t1 * D + col) = make_float2(z1[2 * j], z1[2 * j + 1]);
         }
       }
     }
 
-    // ---- 6: state update W -= dW and the next chunk's operand copy --------------
+    // ---- 6: state update W -= dW and the next chunk's operand copy ------------------
     wait_or_abort(&bars[BAR_DW], par, abort);
     tc_fence_after_sync();
+    __syncwarp();
     // K, V (lo half of eta*G) and eta are free once dW is done; every thread passed
     // this chunk's wait on their barrier before the A-operand barrier above.
     if (tid == 0 && c + 1 < nchunks && !*abort) issue_loads_kv(c + 1);

@@ -175,14 +175,14 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [units][T][64] bf16 viewed as a 3-D tensor; boxes of 64 tokens x 64 features
-// with the 128-byte swizzle.  Rows past T read as zeros.
-bool make_qkv_map(CUtensorMap *map, const void *base, int T, long long units) {
+// [units][T][64] bf16 viewed as a 3-D tensor; boxes of `box_rows` tokens x 64
+// features with the 128-byte swizzle.  Rows past T read as zeros.
+bool make_qkv_map(CUtensorMap *map, const void *base, int T, long long units, int box_rows) {
   auto encode = tensor_map_encoder();
   if (!encode) return false;
   cuuint64_t dims[3] = {64, (cuuint64_t)T, (cuuint64_t)units};
   cuuint64_t strides[2] = {64 * 2, (cuuint64_t)T * 64 * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -198,8 +198,10 @@ template <bool LN>
 int launch_linear_tc(const Call &c) {
   const long long units = (long long)c.B * c.H;
   CUtensorMap mq, mk, mv;
-  if (!make_qkv_map(&mq, c.Q, c.T, units) || !make_qkv_map(&mk, c.K, c.T, units) ||
-      !make_qkv_map(&mv, c.V, c.T, units))
+  // Q and K arrive as one 16-token box per mini-batch (interleaved operand), V as
+  // one 64-token box per chunk.
+  if (!make_qkv_map(&mq, c.Q, c.T, units, tc::MB) || !make_qkv_map(&mk, c.K, c.T, units, tc::MB) ||
+      !make_qkv_map(&mv, c.V, c.T, units, tc::CHUNK))
     return TTT_ERR_CUDA;
   tc::Params p;
   p.Q = static_cast<const __nv_bfloat16 *>(c.Q);
