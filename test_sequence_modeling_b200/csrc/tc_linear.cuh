@@ -66,18 +66,18 @@ constexpr uint32_t OFF_ETA = 49152;    // eta of the chunk, 64 floats
 constexpr uint32_t OFF_GAMMA = 49408;  // LN gamma, 64 floats
 constexpr uint32_t OFF_BETA = 49664;   // LN beta, 64 floats
 constexpr uint32_t OFF_W2 = 49920;     // 2 gamma^2, 64 floats
-constexpr uint32_t OFF_BAR = 50176;    // mbarriers
-constexpr uint32_t OFF_TSLOT = 50240;  // TMEM base address
-constexpr uint32_t OFF_ABORT = 50244;  // set when a bounded wait expired
+constexpr uint32_t OFF_BAR = 50176;    // mbarriers (9 x 8 bytes)
+constexpr uint32_t OFF_TSLOT = 50248;  // TMEM base address
+constexpr uint32_t OFF_ABORT = 50252;  // set when a bounded wait expired
 constexpr uint32_t SMEM_USED = 50256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 __host__ __device__ constexpr uint32_t k_block(int m) { return OFF_A + 4096u * m; }
 __host__ __device__ constexpr uint32_t q_block(int m) { return OFF_A + 4096u * m + 2048u; }
 
-// mbarriers: K/V/eta loads; MMA P,S; updates of mini-batches 0,1,2; last update;
-// dW; Q loads.
-enum { BAR_LOAD = 0, BAR_PS = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, BAR_LOADQ = 7, NUM_BARS = 8 };
+// mbarriers: K/V/eta loads; MMA S; updates of mini-batches 0,1,2; last update;
+// dW; Q loads (four arrivals: one per warp and Q block); MMA P.
+enum { BAR_LOAD = 0, BAR_S = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, BAR_LOADQ = 7, BAR_P = 8, NUM_BARS = 9 };
 
 struct Params {
   const __nv_bfloat16 *Q;  // for the residual of the output (read back from L2)
@@ -90,14 +90,15 @@ struct Params {
   float *W_out;
 };
 
-// Sum of 16 values as a balanced tree (independent adds for instruction-level parallelism).
-__device__ __forceinline__ float tree_sum16(const float (&x)[16]) {
-  float a[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a[i] = x[2 * i] + x[2 * i + 1];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) a[i] += a[i + 4];
-  return (a[0] + a[2]) + (a[1] + a[3]);
+__device__ __forceinline__ float sum8(const float2 (&x)[8]) {
+  const float2 a = __fadd2_rn(__fadd2_rn(x[0], x[1]), __fadd2_rn(x[2], x[3]));
+  const float2 b = __fadd2_rn(__fadd2_rn(x[4], x[5]), __fadd2_rn(x[6], x[7]));
+  const float2 c = __fadd2_rn(a, b);
+  return c.x + c.y;
+}
+
+__device__ __forceinline__ float2 __fsub2(float2 a, float2 b) {
+  return __fadd2_rn(a, make_float2(-b.x, -b.y));
 }
 
 __device__ __forceinline__ float quad_sum(float x) {
@@ -137,7 +138,7 @@ __global__ void __launch_bounds__(THREADS, 4)
   const uint32_t aGhi = sbase + OFF_GHI, aGlo = sbase + OFF_GLO;
 
   if (tid == 0) {
-    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], i == BAR_LOADQ ? 4 : 1);
     *abort = 0;
     fence_mbarrier_init();
     prefetch_tensormap(&tmQ);
@@ -186,9 +187,12 @@ __global__ void __launch_bounds__(THREADS, 4)
 
   const int nchunks = (T + CHUNK - 1) / CHUNK;
   const size_t tok_base = (size_t)unit * T;
+  const int q4 = lane & 3;
+  const int fr = lane >> 2;  // row within a 16-row group (and +8) in the 16x256b layout
 
   // Loads are split so that each tile is fetched as soon as its buffer is free:
-  // Q once P and S are computed, K / V / eta once dW is computed.
+  // each warp refills its own Q block once it has written its output, thread 0
+  // refills K / V / eta once dW is computed.
   auto issue_loads_kv = [&](int c) {
     const int ntok = min(CHUNK, T - c * CHUNK);
     mbar_arrive_expect_tx(&bars[BAR_LOAD], 4u * 2048u + 8192u + (uint32_t)ntok * 4u);
@@ -197,10 +201,10 @@ __global__ void __launch_bounds__(THREADS, 4)
     tma_load_3d(sm + OFF_GLO, &tmV, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
     bulk_load(eta_s, p.eta + tok_base + (size_t)c * CHUNK, (uint32_t)ntok * 4u, &bars[BAR_LOAD]);
   };
-  auto issue_load_q = [&](int c) {
-    mbar_arrive_expect_tx(&bars[BAR_LOADQ], 4u * 2048u);
-#pragma unroll
-    for (int m = 0; m < 4; ++m) tma_load_3d(sm + q_block(m), &tmQ, 0, c * CHUNK + MB * m, unit, &bars[BAR_LOADQ]);
+  // One of the four arrivals of the Q barrier: Q block m of chunk c.
+  auto issue_load_q_block = [&](int c, int m) {
+    mbar_arrive_expect_tx(&bars[BAR_LOADQ], 2048u);
+    tma_load_3d(sm + q_block(m), &tmQ, 0, c * CHUNK + MB * m, unit, &bars[BAR_LOADQ]);
   };
 
   fence_proxy_async_smem();
@@ -209,29 +213,31 @@ __global__ void __launch_bounds__(THREADS, 4)
   tc_fence_after_sync();
   const uint32_t tb = *tslot;
   const uint32_t tP = tb, tS = tb + 64;  // column bases of P and S (lane 0)
-  if (tid == 0 && nchunks > 0) {
-    issue_loads_kv(0);
-    issue_load_q(0);
-  }
+  if (tid == 0 && nchunks > 0) issue_loads_kv(0);
+  if (lane == 0 && nchunks > 0) issue_load_q_block(0, warp);
 
   constexpr uint32_t ID_PW = idesc_bf16_f32(128, 64, false, true, false);  // [K;Q] x W
   constexpr uint32_t ID_S = idesc_bf16_f32(128, 16, false, false, false);  // [K;Q] x K_m^T
   constexpr uint32_t ID_UPD = idesc_bf16_f32(128, 64, false, true, true);  // P -= A x (eta G)
   constexpr uint32_t ID_DW = idesc_bf16_f32(128, 64, true, true, false);   // [K^T;K^T] x (eta G)
 
-  const int q4 = lane & 3;
-  const int fr = lane >> 2;  // row within a 16-row group (and +8) in the 16x256b layout
-
   for (int c = 0; c < nchunks; ++c) {
     const int ntok = min(CHUNK, T - c * CHUNK);
     const int nmb = ntok / MB;
     const uint32_t par = (uint32_t)c & 1u;
 
-    // ---- 1-2: tiles in, P = [K;Q] W and S = [K;Q] K^T ------------------------------
+    // ---- 1-2: tiles in; S = [K;Q] K^T first (the masking needs it), then P = [K;Q] W
     wait_or_abort(&bars[BAR_LOAD], par, abort);
     wait_or_abort(&bars[BAR_LOADQ], par, abort);
     if (tid == 0 && !*abort) {
       tc_fence_after_sync();
+#pragma unroll
+      for (int n = 0; n < 4; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          umma_ss(tS + 16 * n, smem_desc_sw128(aA + 32 * k, 16, 1024),
+                  smem_desc_sw128(sbase + k_block(n) + 32 * k, 16, 1024), ID_S, k > 0);
+      umma_commit(&bars[BAR_S]);
 #pragma unroll
       for (int k = 0; k < 4; ++k)
         umma_ss(tP, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aWhi + 2048 * k, 8192, 1024),
@@ -240,13 +246,7 @@ __global__ void __launch_bounds__(THREADS, 4)
       for (int k = 0; k < 4; ++k)
         umma_ss(tP, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aWlo + 2048 * k, 8192, 1024),
                 ID_PW, true);
-#pragma unroll
-      for (int n = 0; n < 4; ++n)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_ss(tS + 16 * n, smem_desc_sw128(aA + 32 * k, 16, 1024),
-                  smem_desc_sw128(sbase + k_block(n) + 32 * k, 16, 1024), ID_S, k > 0);
-      umma_commit(&bars[BAR_PS]);
+      umma_commit(&bars[BAR_P]);
     }
     if (ntok < CHUNK) {  // ragged last chunk: absent tokens contribute nothing to dW
       for (int x = tid; x < (CHUNK - ntok) * 32; x += THREADS) {
@@ -255,7 +255,44 @@ __global__ void __launch_bounds__(THREADS, 4)
         *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(row, col)) = 0u;
       }
     }
-    wait_or_abort(&bars[BAR_PS], par, abort);
+
+    // Everything of mini-batch `warp`'s LN backward that does not depend on P,
+    // computed while the tensor core works: u = 2 gamma (k + beta - v) (or v for
+    // the plain linear model) for this thread's two rows, and mean(u).
+    const int m = warp;
+    const int r0 = MB * m + fr, r1 = r0 + 8;  // tokens of this thread's two rows
+    float2 u0[8], u1[8];
+    float um0 = 0.f, um1 = 0.f;
+    if (m < nmb) {
+      const uint32_t kb = sbase + k_block(m);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int col = 8 * j + 2 * q4;
+        const float2 va = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r0, col)));
+        const float2 vc = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r1, col)));
+        if (LN) {
+          const float2 ka = unpack_bf16x2(lds_u32(kb + sw128_offset(fr, col)));
+          const float2 kc = unpack_bf16x2(lds_u32(kb + sw128_offset(fr + 8, col)));
+          const float2 gm = *reinterpret_cast<const float2 *>(sm + OFF_GAMMA + 4 * col);
+          const float2 bt = *reinterpret_cast<const float2 *>(sm + OFF_BETA + 4 * col);
+          const float2 g2 = __fadd2_rn(gm, gm);
+          u0[j] = __fmul2_rn(g2, __fadd2_rn(ka, __fsub2(bt, va)));
+          u1[j] = __fmul2_rn(g2, __fadd2_rn(kc, __fsub2(bt, vc)));
+          um0 += u0[j].x + u0[j].y;
+          um1 += u1[j].x + u1[j].y;
+        } else {
+          u0[j] = va;
+          u1[j] = vc;
+        }
+      }
+      if (LN) {
+        um0 = quad_sum(um0) * (1.f / D);
+        um1 = quad_sum(um1) * (1.f / D);
+      }
+    }
+    const float e0 = eta_s[r0], e1 = eta_s[r1];
+
+    wait_or_abort(&bars[BAR_S], par, abort);
     tc_fence_after_sync();
     __syncwarp();  // lanes leave the wait loop independently; TMEM access is warp-collective
 
@@ -267,32 +304,22 @@ __global__ void __launch_bounds__(THREADS, 4)
       // blocks < warp, Q rows blocks <= warp); TMEM loads and stores are
       // warp-collective, so the skip is decided per warp.
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        uint32_t v[32];
-        if (2 * jj <= warp) {
-          tmem_ld_32x32b_x32(tmem_addr(tS, 32 * warp, 32 * jj), v);
+      for (int j = 0; j < 4; ++j) {
+        uint32_t v[16], hi[8], lo[8];
+        if (j <= warp) {
+          tmem_ld_32x32b_x16(tmem_addr(tS, 32 * warp, 16 * j), v);
           tmem_wait_ld();
         }
+        const bool all_zero = qrow ? (j > warp) : (j >= warp);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int j = 2 * jj + h;
-          uint32_t hi[8], lo[8];
-          const bool all_zero = qrow ? (j > warp) : (j >= warp);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int s0 = MB * j + 2 * e;
-            const float a = (!all_zero && (!qrow || s0 <= t)) ? __uint_as_float(v[16 * h + 2 * e]) : 0.f;
-            const float b = (!all_zero && (!qrow || s0 + 1 <= t)) ? __uint_as_float(v[16 * h + 2 * e + 1]) : 0.f;
-            split_bf16x2(a, b, hi[e], lo[e]);
-          }
-          if (j <= warp) {
-            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j), hi);
-            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j + 8), lo);
-          } else {
-            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j), hi);  // zeros
-            tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j + 8), hi);
-          }
+        for (int e = 0; e < 8; ++e) {
+          const int s0 = MB * j + 2 * e;
+          const float a = (!all_zero && (!qrow || s0 <= t)) ? __uint_as_float(v[2 * e]) : 0.f;
+          const float b = (!all_zero && (!qrow || s0 + 1 <= t)) ? __uint_as_float(v[2 * e + 1]) : 0.f;
+          split_bf16x2(a, b, hi[e], lo[e]);
         }
+        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j), hi);
+        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j + 8), lo);
       }
       tmem_wait_st();
     }
@@ -302,67 +329,25 @@ __global__ void __launch_bounds__(THREADS, 4)
     tc_fence_after_sync();
 
     // ---- 4: the mini-batch chain: warp m handles mini-batch m ------------------------
-    if (warp < nmb) {
-      const int m = warp;
-      const int r0 = MB * m + fr, r1 = r0 + 8;  // tokens of this thread's two rows
-      const uint32_t kb = sbase + k_block(m);
-      // Everything of the LN backward that does not depend on P, computed before
-      // waiting for the previous mini-batch: u = 2 gamma (k + beta - v), its mean.
-      float u0[16], u1[16];
-      float um0 = 0.f, um1 = 0.f;
-      if (LN) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          const float2 ka = unpack_bf16x2(lds_u32(kb + sw128_offset(fr, col)));
-          const float2 kc = unpack_bf16x2(lds_u32(kb + sw128_offset(fr + 8, col)));
-          const float2 va = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r0, col)));
-          const float2 vc = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r1, col)));
-          const float2 gm = lds_f2(sbase + OFF_GAMMA + 4 * col);
-          const float2 bt = lds_f2(sbase + OFF_BETA + 4 * col);
-          u0[2 * j] = 2.f * gm.x * (ka.x + bt.x - va.x);
-          u0[2 * j + 1] = 2.f * gm.y * (ka.y + bt.y - va.y);
-          u1[2 * j] = 2.f * gm.x * (kc.x + bt.x - vc.x);
-          u1[2 * j + 1] = 2.f * gm.y * (kc.y + bt.y - vc.y);
-          um0 += u0[2 * j] + u0[2 * j + 1];
-          um1 += u1[2 * j] + u1[2 * j + 1];
-        }
-        um0 = quad_sum(um0) * (1.f / D);
-        um1 = quad_sum(um1) * (1.f / D);
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          const float2 va = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r0, col)));
-          const float2 vc = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r1, col)));
-          u0[2 * j] = va.x;
-          u0[2 * j + 1] = va.y;
-          u1[2 * j] = vc.x;
-          u1[2 * j + 1] = vc.y;
-        }
-      }
-      const float e0 = eta_s[r0], e1 = eta_s[r1];
-
-      if (m > 0) wait_or_abort(&bars[BAR_C0 + m - 1], par, abort);
+    if (m < nmb) {
+      wait_or_abort(&bars[m == 0 ? BAR_P : BAR_C0 + m - 1], par, abort);
       tc_fence_after_sync();
       __syncwarp();
       uint32_t yr[32];
       tmem_ld_16x256b_x8(tmem_addr(tP, 32 * m, 0), yr);
       tmem_wait_ld();
-      float y0[16], y1[16];
+      float2 y0[8], y1[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        y0[2 * j] = __uint_as_float(yr[4 * j + 0]);
-        y0[2 * j + 1] = __uint_as_float(yr[4 * j + 1]);
-        y1[2 * j] = __uint_as_float(yr[4 * j + 2]);
-        y1[2 * j + 1] = __uint_as_float(yr[4 * j + 3]);
+        y0[j] = make_float2(__uint_as_float(yr[4 * j + 0]), __uint_as_float(yr[4 * j + 1]));
+        y1[j] = make_float2(__uint_as_float(yr[4 * j + 2]), __uint_as_float(yr[4 * j + 3]));
       }
       // Stores eta * (dl/dy) of one column pair of both rows as bf16 hi + lo; the
       // lo half overwrites V, which this thread has read for exactly these cells.
-      auto store_grad = [&](int col, float ga0, float ga1, float gb0, float gb1) {
+      auto store_grad = [&](int col, float2 g0, float2 g1) {
         uint32_t h0, l0, h1, l1;
-        split_bf16x2(ga0, ga1, h0, l0);
-        split_bf16x2(gb0, gb1, h1, l1);
+        split_bf16x2(g0.x, g0.y, h0, l0);
+        split_bf16x2(g1.x, g1.y, h1, l1);
         *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r0, col)) = h0;
         *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r0, col)) = l0;
         *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r1, col)) = h1;
@@ -370,58 +355,60 @@ __global__ void __launch_bounds__(THREADS, 4)
       };
       if (!LN) {
         // dl/dy = 2 (y - v)
+        const float2 f0 = make_float2(2.f * e0, 2.f * e0), f1 = make_float2(2.f * e1, 2.f * e1);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          store_grad(8 * j + 2 * q4, 2.f * e0 * (y0[2 * j] - u0[2 * j]),
-                     2.f * e0 * (y0[2 * j + 1] - u0[2 * j + 1]), 2.f * e1 * (y1[2 * j] - u1[2 * j]),
-                     2.f * e1 * (y1[2 * j + 1] - u1[2 * j + 1]));
+          store_grad(8 * j + 2 * q4, __fmul2_rn(f0, __fsub2(y0[j], u0[j])),
+                     __fmul2_rn(f1, __fsub2(y1[j], u1[j])));
       } else {
         // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y.  With
         // dx = dl/dxhat = u + w xhat (w = 2 gamma^2), A = mean(dx), B = mean(dx xhat):
         // dl/dy = rstd (dx - A - xhat B) = rstd (u + xhat (w - B) - A).
-        const float mean0 = quad_sum(tree_sum16(y0)) * (1.f / D);
-        const float mean1 = quad_sum(tree_sum16(y1)) * (1.f / D);
-        float sq0[16], sq1[16];
+        const float mean0 = quad_sum(sum8(y0)) * (1.f / D);
+        const float mean1 = quad_sum(sum8(y1)) * (1.f / D);
+        const float2 nm0 = make_float2(-mean0, -mean0), nm1 = make_float2(-mean1, -mean1);
+        float2 q0a = make_float2(0.f, 0.f), q0b = q0a, q1a = q0a, q1b = q0a;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          y0[e] -= mean0;
-          y1[e] -= mean1;
-          sq0[e] = y0[e] * y0[e];
-          sq1[e] = y1[e] * y1[e];
+        for (int j = 0; j < 8; j += 2) {
+          y0[j] = __fadd2_rn(y0[j], nm0);
+          y0[j + 1] = __fadd2_rn(y0[j + 1], nm0);
+          y1[j] = __fadd2_rn(y1[j], nm1);
+          y1[j + 1] = __fadd2_rn(y1[j + 1], nm1);
+          q0a = __ffma2_rn(y0[j], y0[j], q0a);
+          q0b = __ffma2_rn(y0[j + 1], y0[j + 1], q0b);
+          q1a = __ffma2_rn(y1[j], y1[j], q1a);
+          q1b = __ffma2_rn(y1[j + 1], y1[j + 1], q1b);
         }
-        const float v0 = tree_sum16(sq0), v1 = tree_sum16(sq1);
-        const float rstd0 = rsqrtf(quad_sum(v0) * (1.f / D) + p.eps);
-        const float rstd1 = rsqrtf(quad_sum(v1) * (1.f / D) + p.eps);
-        float wx0 = 0.f, wx1 = 0.f, ux0 = 0.f, ux1 = 0.f, wxx0 = 0.f, wxx1 = 0.f;
+        const float rstd0 = rsqrtf(quad_sum((q0a.x + q0b.x) + (q0a.y + q0b.y)) * (1.f / D) + p.eps);
+        const float rstd1 = rsqrtf(quad_sum((q1a.x + q1b.x) + (q1a.y + q1b.y)) * (1.f / D) + p.eps);
+        const float2 rs0 = make_float2(rstd0, rstd0), rs1 = make_float2(rstd1, rstd1);
+        float2 wx0 = make_float2(0.f, 0.f), wx1 = wx0, ux0 = wx0, ux1 = wx0, wxx0 = wx0, wxx1 = wx0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float2 w2 = lds_f2(sbase + OFF_W2 + 4 * (8 * j + 2 * q4));
-          const float wv[2] = {w2.x, w2.y};
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int e = 2 * j + h;
-            const float xa = y0[e] * rstd0, xb = y1[e] * rstd1;
-            y0[e] = xa;
-            y1[e] = xb;
-            wx0 = fmaf(wv[h], xa, wx0);
-            wx1 = fmaf(wv[h], xb, wx1);
-            ux0 = fmaf(u0[e], xa, ux0);
-            ux1 = fmaf(u1[e], xb, ux1);
-            wxx0 = fmaf(wv[h] * xa, xa, wxx0);
-            wxx1 = fmaf(wv[h] * xb, xb, wxx1);
-          }
+          const float2 w2 = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
+          y0[j] = __fmul2_rn(y0[j], rs0);  // xhat
+          y1[j] = __fmul2_rn(y1[j], rs1);
+          const float2 wa = __fmul2_rn(w2, y0[j]), wb = __fmul2_rn(w2, y1[j]);
+          wx0 = __fadd2_rn(wx0, wa);
+          wx1 = __fadd2_rn(wx1, wb);
+          wxx0 = __ffma2_rn(wa, y0[j], wxx0);
+          wxx1 = __ffma2_rn(wb, y1[j], wxx1);
+          ux0 = __ffma2_rn(u0[j], y0[j], ux0);
+          ux1 = __ffma2_rn(u1[j], y1[j], ux1);
         }
-        const float A0 = um0 + quad_sum(wx0) * (1.f / D), A1 = um1 + quad_sum(wx1) * (1.f / D);
-        const float B0 = (quad_sum(ux0) + quad_sum(wxx0)) * (1.f / D);
-        const float B1 = (quad_sum(ux1) + quad_sum(wxx1)) * (1.f / D);
-        const float f0 = e0 * rstd0, f1 = e1 * rstd1;  // eta folded into the scale
+        const float A0 = um0 + quad_sum(wx0.x + wx0.y) * (1.f / D);
+        const float A1 = um1 + quad_sum(wx1.x + wx1.y) * (1.f / D);
+        const float B0 = quad_sum((ux0.x + ux0.y) + (wxx0.x + wxx0.y)) * (1.f / D);
+        const float B1 = quad_sum((ux1.x + ux1.y) + (wxx1.x + wxx1.y)) * (1.f / D);
+        const float2 f0 = make_float2(e0 * rstd0, e0 * rstd0), f1 = make_float2(e1 * rstd1, e1 * rstd1);
+        const float2 nA0 = make_float2(-A0, -A0), nA1 = make_float2(-A1, -A1);
+        const float2 nB0 = make_float2(-B0, -B0), nB1 = make_float2(-B1, -B1);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float2 w2 = lds_f2(sbase + OFF_W2 + 4 * (8 * j + 2 * q4));
-          store_grad(8 * j + 2 * q4, f0 * (fmaf(y0[2 * j], w2.x - B0, u0[2 * j]) - A0),
-                     f0 * (fmaf(y0[2 * j + 1], w2.y - B0, u0[2 * j + 1]) - A0),
-                     f1 * (fmaf(y1[2 * j], w2.x - B1, u1[2 * j]) - A1),
-                     f1 * (fmaf(y1[2 * j + 1], w2.y - B1, u1[2 * j + 1]) - A1));
+          const float2 w2 = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
+          const float2 ga = __fmul2_rn(f0, __fadd2_rn(__ffma2_rn(y0[j], __fadd2_rn(w2, nB0), u0[j]), nA0));
+          const float2 gb = __fmul2_rn(f1, __fadd2_rn(__ffma2_rn(y1[j], __fadd2_rn(w2, nB1), u1[j]), nA1));
+          store_grad(8 * j + 2 * q4, ga, gb);
         }
       }
       fence_proxy_async_smem();
@@ -437,26 +424,75 @@ __global__ void __launch_bounds__(THREADS, 4)
         umma_commit(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
       }
       __syncwarp();
-    }
 
-    // This warp's Q rows, kept in registers for the residual of the output; then
-    // the Q buffer is refilled with the next chunk.  The prefetch is issued after a
-    // CTA-wide barrier: every thread has then read its Q rows and passed its wait
-    // on this chunk's Q phase (so that phase cannot be overtaken).
-    uint32_t qres[16];
+      // ---- 5: output of this mini-batch's Q rows.  After update m their value is
+      // final: later updates add exactly zero to them (A is zero there).
+      wait_or_abort(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m], par, abort);
+      tc_fence_after_sync();
+      __syncwarp();
+      uint32_t zr[32];
+      tmem_ld_16x256b_x8(tmem_addr(tP, 32 * m + 16, 0), zr);
+      tmem_wait_ld();
+      float2 z0[8], z1[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int col = 8 * j + 2 * q4;
-      qres[2 * j] = lds_u32(sbase + q_block(warp) + sw128_offset(fr, col));
-      qres[2 * j + 1] = lds_u32(sbase + q_block(warp) + sw128_offset(fr + 8, col));
+      for (int j = 0; j < 8; ++j) {
+        z0[j] = make_float2(__uint_as_float(zr[4 * j + 0]), __uint_as_float(zr[4 * j + 1]));
+        z1[j] = make_float2(__uint_as_float(zr[4 * j + 2]), __uint_as_float(zr[4 * j + 3]));
+      }
+      float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
+      const bool ok0 = r0 < ntok, ok1 = r1 < ntok;
+      const uint32_t qb = sbase + q_block(m);
+      if (LN) {
+        const float mean0 = quad_sum(sum8(z0)) * (1.f / D);
+        const float mean1 = quad_sum(sum8(z1)) * (1.f / D);
+        const float2 nm0 = make_float2(-mean0, -mean0), nm1 = make_float2(-mean1, -mean1);
+        float2 q0a = make_float2(0.f, 0.f), q0b = q0a, q1a = q0a, q1b = q0a;
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+          z0[j] = __fadd2_rn(z0[j], nm0);
+          z0[j + 1] = __fadd2_rn(z0[j + 1], nm0);
+          z1[j] = __fadd2_rn(z1[j], nm1);
+          z1[j + 1] = __fadd2_rn(z1[j + 1], nm1);
+          q0a = __ffma2_rn(z0[j], z0[j], q0a);
+          q0b = __ffma2_rn(z0[j + 1], z0[j + 1], q0b);
+          q1a = __ffma2_rn(z1[j], z1[j], q1a);
+          q1b = __ffma2_rn(z1[j + 1], z1[j + 1], q1b);
+        }
+        const float rstd0 = rsqrtf(quad_sum((q0a.x + q0b.x) + (q0a.y + q0b.y)) * (1.f / D) + p.eps);
+        const float rstd1 = rsqrtf(quad_sum((q1a.x + q1b.x) + (q1a.y + q1b.y)) * (1.f / D) + p.eps);
+        const float2 rs0 = make_float2(rstd0, rstd0), rs1 = make_float2(rstd1, rstd1);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int col = 8 * j + 2 * q4;
+          const float2 gm = *reinterpret_cast<const float2 *>(sm + OFF_GAMMA + 4 * col);
+          const float2 bt = *reinterpret_cast<const float2 *>(sm + OFF_BETA + 4 * col);
+          const float2 qa = unpack_bf16x2(lds_u32(qb + sw128_offset(fr, col)));
+          const float2 qc = unpack_bf16x2(lds_u32(qb + sw128_offset(fr + 8, col)));
+          if (ok0)
+            *reinterpret_cast<float2 *>(Zc + r0 * D + col) =
+                __fadd2_rn(qa, __ffma2_rn(gm, __fmul2_rn(z0[j], rs0), bt));
+          if (ok1)
+            *reinterpret_cast<float2 *>(Zc + r1 * D + col) =
+                __fadd2_rn(qc, __ffma2_rn(gm, __fmul2_rn(z1[j], rs1), bt));
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int col = 8 * j + 2 * q4;
+          if (ok0) *reinterpret_cast<float2 *>(Zc + r0 * D + col) = z0[j];
+          if (ok1) *reinterpret_cast<float2 *>(Zc + r1 * D + col) = z1[j];
+        }
+      }
+      // This warp's Q block is no longer needed: refill it with the next chunk.
+      // The Q barrier completes only when all four warps have arrived, i.e. after
+      // every thread has passed its wait on this chunk's Q phase.
+      __syncwarp();
+      if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q_block(c + 1, m);
     }
-    named_barrier_sync(1, THREADS);
-    if (tid == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
 
-    // ---- 5: the last update done -> dW on the tensor core, output on CUDA cores --------
+    // ---- 6: dW on the tensor core after the last update; state update -------------
     wait_or_abort(&bars[BAR_LAST], par, abort);
     tc_fence_after_sync();
-    __syncwarp();
     if (tid == 0 && !*abort) {
 #pragma unroll
       for (int k = 0; k < 4; ++k)
@@ -468,67 +504,6 @@ __global__ void __launch_bounds__(THREADS, 4)
                 ID_DW, true);
       umma_commit(&bars[BAR_DW]);
     }
-    {
-      // Q rows of mini-batch `warp`: lanes 32 warp + 16 .. +31.
-      uint32_t zr[32];
-      tmem_ld_16x256b_x8(tmem_addr(tP, 32 * warp + 16, 0), zr);
-      tmem_wait_ld();
-      const int t0 = MB * warp + fr, t1 = t0 + 8;
-      float z0[16], z1[16];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        z0[2 * j] = __uint_as_float(zr[4 * j + 0]);
-        z0[2 * j + 1] = __uint_as_float(zr[4 * j + 1]);
-        z1[2 * j] = __uint_as_float(zr[4 * j + 2]);
-        z1[2 * j + 1] = __uint_as_float(zr[4 * j + 3]);
-      }
-      float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
-      const bool ok0 = t0 < ntok, ok1 = t1 < ntok;
-      if (LN) {
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          s0 += z0[e];
-          s1 += z1[e];
-        }
-        const float mean0 = quad_sum(s0) * (1.f / D), mean1 = quad_sum(s1) * (1.f / D);
-        float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          z0[e] -= mean0;
-          z1[e] -= mean1;
-          v0 += z0[e] * z0[e];
-          v1 += z1[e] * z1[e];
-        }
-        const float rstd0 = rsqrtf(quad_sum(v0) * (1.f / D) + p.eps);
-        const float rstd1 = rsqrtf(quad_sum(v1) * (1.f / D) + p.eps);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          const float2 gm = lds_f2(sbase + OFF_GAMMA + 4 * col);
-          const float2 bt = lds_f2(sbase + OFF_BETA + 4 * col);
-          if (ok0) {
-            const float2 qa = unpack_bf16x2(qres[2 * j]);
-            *reinterpret_cast<float2 *>(Zc + t0 * D + col) =
-                make_float2(qa.x + fmaf(gm.x, z0[2 * j] * rstd0, bt.x), qa.y + fmaf(gm.y, z0[2 * j + 1] * rstd0, bt.y));
-          }
-          if (ok1) {
-            const float2 qb = unpack_bf16x2(qres[2 * j + 1]);
-            *reinterpret_cast<float2 *>(Zc + t1 * D + col) =
-                make_float2(qb.x + fmaf(gm.x, z1[2 * j] * rstd1, bt.x), qb.y + fmaf(gm.y, z1[2 * j + 1] * rstd1, bt.y));
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          if (ok0) *reinterpret_cast<float2 *>(Zc + t0 * D + col) = make_float2(z0[2 * j], z0[2 * j + 1]);
-          if (ok1) *reinterpret_cast<float2 *>(Zc + t1 * D + col) = make_float2(z1[2 * j], z1[2 * j + 1]);
-        }
-      }
-    }
-
-    // ---- 6: state update W -= dW and the next chunk's operand copy ------------------
     wait_or_abort(&bars[BAR_DW], par, abort);
     tc_fence_after_sync();
     __syncwarp();
