@@ -295,7 +295,9 @@ def main():
     lib = _lib.load()
     ttt.set_path({"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT, "tc": ttt.TTT_PATH_TC}[args.path])
 
-    data = I.make_inputs(cfg, batch_offset=rank * cfg.B)
+    from test_sequence_modeling_b200 import sharding
+    cfg, batch_offset = sharding.shard(cfg, world, rank)
+    data = I.make_inputs(cfg, batch_offset=batch_offset)
     if data["qkv_bits"]:
         host = {k: torch.from_numpy(data[k].view(np.int16)).view(torch.bfloat16) for k in "QKV"}
     else:
@@ -363,10 +365,7 @@ def main():
     status = ttt.last_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
-    t = torch.tensor([total_ms, statistics.mean(kernel_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, kernel_avg_ms = float(t[0]), float(t[1])
+    total_ms, kernel_avg_ms = sharding.max_over_ranks([total_ms, statistics.mean(kernel_ms)], dist, dev)
     ms_per_step = total_ms / args.steps
     value = world * cfg.head_tokens * args.steps / (total_ms / 1e3)
 
@@ -404,10 +403,9 @@ def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, 
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = world * cfg.head_tokens * args.e2e_steps / (float(te[0]) / 1e3)
+    from test_sequence_modeling_b200 import sharding
+    (te,) = sharding.max_over_ranks([e0.elapsed_time(e1)], dist, dev)
+    e2e_value = world * cfg.head_tokens * args.e2e_steps / (te / 1e3)
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps}
 
