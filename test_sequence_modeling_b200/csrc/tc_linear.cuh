@@ -8,31 +8,45 @@
 // Work decomposition.  One CTA of 4 warps owns one (batch, head) sequence for
 // its whole length and keeps the fp32 state W in registers.  Tokens are taken
 // in chunks of 64 (four mini-batches), so that every tensor-core product has
-// M = 128 rows: the 64 K rows and the 64 Q rows of the chunk, interleaved by
-// mini-batch as [K0; Q0; K1; Q1; K2; Q2; K3; Q3] (16 rows each).  TMEM lane =
-// operand row, so warp m (which can read TMEM lanes 32m..32m+31) holds exactly
-// the K and Q rows of mini-batch m.  With W_c the state at the start of the
-// chunk and G_m the gradient of the loss w.r.t. the pre-activation of
-// mini-batch m (taken at that mini-batch's own base state), the state at the
-// start of mini-batch m is W_m = W_c - sum_{j<m} K_j^T diag(eta_j) G_j, so that
+// M = 128 rows: the 64 K rows and the 64 Q rows of the chunk.  With W_c the
+// state at the start of the chunk and G_m the gradient of the loss w.r.t. the
+// pre-activation of mini-batch m (taken at that mini-batch's own base state),
+// W_m = W_c - sum_{j<m} K_j^T diag(eta_j) G_j, so that, exactly,
 //   K_m W_m = (K W_c)_m - sum_{j<m} (K_m K_j^T) diag(eta_j) G_j
 //   q_t W_t = (Q W_c)_t - sum_{s<=t} (q_t . k_s) eta_s G_s    (dual-form output)
 //   W_next  = W_c - K^T diag(eta) G.
+//
+// Row layout of [K;Q] (= TMEM lanes of the products).  8-row group
+// g = 8h + 2m + q holds tokens 16m + 8h + (0..7) of K (q = 0) or Q (q = 1): h
+// is the half of mini-batch m.  So TMEM lane quarter w (warp w) holds half
+// h = w / 2 of mini-batches 2(w % 2) and 2(w % 2) + 1, each as 8 K rows followed
+// by the 8 Q rows of the same tokens (one 16-lane access returns both), every
+// mini-batch is shared by two warps (m / 2 and 2 + m / 2), and the K rows alone
+// sit in every other group (a uniform-stride operand: column n = 8i + r of
+// S = [K;Q] K^T is token 16 (i % 4) + 8 (i / 4) + r).
+//
 // Per chunk:
-//   1. TMA: K and Q (16-row boxes into the interleaved operand, 128-byte
-//      swizzle), V, eta.
-//   2. tcgen05: P = [K;Q] W_c (TMEM cols 0..63), S = [K;Q] K^T (cols 64..127).
-//   3. Every thread masks its own row of S in TMEM into the A operand of step 4:
-//      K rows keep the columns of earlier mini-batches, Q rows keep s <= t (the
-//      causal mask of the dual form, diagonal included), as bf16 hi + lo.
-//   4. For m = 0..3, warp m: reads its 16 K rows of P (already corrected for
-//      mini-batches < m), computes G_m (LN backward in registers), writes
-//      eta*G_m as bf16 hi + lo, and issues P -= A[:, m] (eta G_m), which applies
-//      mini-batch m's update to every later K row and every Q row at once.
-//   5. Then the Q rows of P hold Q W - tril(Q K^T) diag(eta) G: each warp applies
-//      LN + residual to its 16 Q rows and stores Z while the tensor core computes
-//      dW = K^T (eta G); every thread then updates its 32 fp32 state elements and
-//      rewrites the bf16 hi + lo operand copy of W for the next chunk.
+//   1. TMA: K and Q (8-row boxes into that layout, 128-byte swizzle), V
+//      (64 x 64), eta.
+//   2. tcgen05: S = [K;Q] K^T (TMEM cols 64..127) and P = [K;Q] W_c (cols 0..63).
+//   3. Every thread masks its own row of S in TMEM, in place, into the A operand
+//      of step 4 (bf16 hi in the columns of the first half of each mini-batch,
+//      lo in those of the second): K rows keep the columns of earlier
+//      mini-batches, Q rows keep s <= t (the causal mask of the dual form,
+//      diagonal included).
+//   4. For m = 0..3, the two warps that hold mini-batch m read its K rows of P
+//      (already corrected for mini-batches < m), compute G_m (LN backward in
+//      registers, 16 elements per thread), write eta*G_m as bf16 hi + lo, meet
+//      at a named barrier, and one of them issues P -= A[:, m] (eta G_m) (A read
+//      from TMEM), which applies mini-batch m's update to every later K row and
+//      every Q row at once.  Once their chain steps are issued, the warps write
+//      the outputs of their Q rows, which are final after their mini-batch's
+//      update (later updates add exactly zero to them).
+//   5. dW = K^T (eta G) on the tensor core into the S columns (free again);
+//      every thread updates its 32 fp32 state elements and rewrites the bf16
+//      hi + lo operand copy of W; then steps 1-3 of the next chunk follow
+//      directly (the next K, V are fetched as soon as dW is done, each warp's Q
+//      rows as soon as it has written its outputs).
 // Precision: every fp32 operand (W, eta*G, the masked Q K^T) enters the tensor
 // core as a bf16 pair hi + lo (error ~2^-16 relative); K and Q are exact bf16;
 // accumulation is fp32.
@@ -57,7 +71,7 @@ constexpr int THREADS = 128;
 constexpr uint32_t TMEM_COLS = 128;
 
 // Shared-memory map (bytes from a 1024-byte aligned base).
-constexpr uint32_t OFF_A = 0;          // [K0;Q0;K1;Q1;K2;Q2;K3;Q3], 16 rows x 128 B each
+constexpr uint32_t OFF_A = 0;          // [K;Q] rows of the chunk in 8-row groups (see kq_group)
 constexpr uint32_t OFF_WHI = 16384;    // W hi [d_in][d_out] bf16
 constexpr uint32_t OFF_WLO = 24576;    // W lo
 constexpr uint32_t OFF_GHI = 32768;    // eta*G hi [token][d_out] bf16
@@ -72,15 +86,35 @@ constexpr uint32_t OFF_ABORT = 50252;  // set when a bounded wait expired
 constexpr uint32_t SMEM_USED = 50256;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
-__host__ __device__ constexpr uint32_t k_block(int m) { return OFF_A + 4096u * m; }
-__host__ __device__ constexpr uint32_t q_block(int m) { return OFF_A + 4096u * m + 2048u; }
+// 8-row group of token `row` of the chunk in the [K;Q] operand: K (q = 0) or Q
+// (q = 1) of half (row / 8) % 2 of mini-batch row / 16.
+__host__ __device__ __forceinline__ uint32_t kq_group(int row, int q) {
+  return 8u * ((row >> 3) & 1) + 2u * (row >> 4) + (uint32_t)q;
+}
+__device__ __forceinline__ uint32_t kq_offset(int row, int q, int col) {
+  return OFF_A + 1024u * kq_group(row, q) + sw128_offset(row & 7, col);
+}
+
+// One of the two lanes that a 16x256b load gives each thread (which = 0: lane
+// base + i/4, which = 1: lane base + 8 + i/4), all 64 columns, as column pairs
+// 8j + 2(i%4) + {0,1}; two 32-column loads keep the live registers low.
+__device__ __forceinline__ void tmem_rows_16x256b(uint32_t taddr, int which, float2 (&y)[8]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t r[16];
+    tmem_ld_16x256b_x4(taddr + 32 * h, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      y[4 * h + j] = make_float2(__uint_as_float(r[4 * j + 2 * which]), __uint_as_float(r[4 * j + 2 * which + 1]));
+  }
+}
 
 // mbarriers: K/V/eta loads; MMA S; updates of mini-batches 0,1,2; last update;
-// dW; Q loads (four arrivals: one per warp and Q block); MMA P.
+// dW; Q loads (four arrivals: one per warp); MMA P.
 enum { BAR_LOAD = 0, BAR_S = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, BAR_LOADQ = 7, BAR_P = 8, NUM_BARS = 9 };
 
 struct Params {
-  const __nv_bfloat16 *Q;  // for the residual of the output (read back from L2)
   const float *eta;
   const float *W0;
   const float *gamma, *beta;
@@ -136,6 +170,10 @@ __global__ void __launch_bounds__(THREADS, 4)
   const uint32_t aA = sbase + OFF_A;
   const uint32_t aWhi = sbase + OFF_WHI, aWlo = sbase + OFF_WLO;
   const uint32_t aGhi = sbase + OFF_GHI, aGlo = sbase + OFF_GLO;
+  const int q4 = lane & 3;
+  const int fr = lane >> 2;        // row within an 8-row group in the 16x256b layout
+  const int mb0 = 2 * (warp & 1);  // this warp holds mini-batches mb0 and mb0 + 1 ...
+  const int hh = warp >> 1;        // ... half hh of each
 
   if (tid == 0) {
     for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], i == BAR_LOADQ ? 4 : 1);
@@ -156,7 +194,8 @@ __global__ void __launch_bounds__(THREADS, 4)
     reinterpret_cast<float *>(sm + OFF_W2)[tid] = 2.f * g * g;
   }
 
-  // Each thread owns 32 elements of the fp32 state: row wi, columns wc0..wc0+31.
+  // Each thread owns 32 elements of the fp32 state: row wi, columns wc0..wc0+31
+  // (the layout in which dW comes back from TMEM).
   const int wi = 32 * (warp & 1) + lane;
   const int wc0 = 32 * (warp >> 1);
   float wm[32];
@@ -187,24 +226,28 @@ __global__ void __launch_bounds__(THREADS, 4)
 
   const int nchunks = (T + CHUNK - 1) / CHUNK;
   const size_t tok_base = (size_t)unit * T;
-  const int q4 = lane & 3;
-  const int fr = lane >> 2;  // row within a 16-row group (and +8) in the 16x256b layout
+  auto chunk_tokens = [&](int c) { return min(CHUNK, T - c * CHUNK); };
 
   // Loads are split so that each tile is fetched as soon as its buffer is free:
-  // each warp refills its own Q block once it has written its output, thread 0
+  // each warp refills its own Q rows once it has written its outputs, thread 0
   // refills K / V / eta once dW is computed.
   auto issue_loads_kv = [&](int c) {
-    const int ntok = min(CHUNK, T - c * CHUNK);
-    mbar_arrive_expect_tx(&bars[BAR_LOAD], 4u * 2048u + 8192u + (uint32_t)ntok * 4u);
+    const int ntok = chunk_tokens(c);
+    mbar_arrive_expect_tx(&bars[BAR_LOAD], 8u * 1024u + 8192u + (uint32_t)ntok * 4u);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) tma_load_3d(sm + k_block(m), &tmK, 0, c * CHUNK + MB * m, unit, &bars[BAR_LOAD]);
+    for (int g = 0; g < 8; ++g)
+      tma_load_3d(sm + OFF_A + 1024u * kq_group(8 * g, 0), &tmK, 0, c * CHUNK + 8 * g, unit, &bars[BAR_LOAD]);
     tma_load_3d(sm + OFF_GLO, &tmV, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
     bulk_load(eta_s, p.eta + tok_base + (size_t)c * CHUNK, (uint32_t)ntok * 4u, &bars[BAR_LOAD]);
   };
-  // One of the four arrivals of the Q barrier: Q block m of chunk c.
-  auto issue_load_q_block = [&](int c, int m) {
+  // One of the four arrivals of the Q barrier: this warp's 16 Q rows of chunk c.
+  auto issue_load_q = [&](int c) {
     mbar_arrive_expect_tx(&bars[BAR_LOADQ], 2048u);
-    tma_load_3d(sm + q_block(m), &tmQ, 0, c * CHUNK + MB * m, unit, &bars[BAR_LOADQ]);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int t0 = MB * (mb0 + i) + 8 * hh;
+      tma_load_3d(sm + OFF_A + 1024u * kq_group(t0, 1), &tmQ, 0, c * CHUNK + t0, unit, &bars[BAR_LOADQ]);
+    }
   };
 
   fence_proxy_async_smem();
@@ -214,39 +257,45 @@ __global__ void __launch_bounds__(THREADS, 4)
   const uint32_t tb = *tslot;
   const uint32_t tP = tb, tS = tb + 64;  // column bases of P and S (lane 0)
   if (tid == 0 && nchunks > 0) issue_loads_kv(0);
-  if (lane == 0 && nchunks > 0) issue_load_q_block(0, warp);
+  if (lane == 0 && nchunks > 0) issue_load_q(0);
 
-  constexpr uint32_t ID_PW = idesc_bf16_f32(128, 64, false, true, false);  // [K;Q] x W
-  constexpr uint32_t ID_S = idesc_bf16_f32(128, 16, false, false, false);  // [K;Q] x K_m^T
+  constexpr uint32_t ID_P = idesc_bf16_f32(128, 64, false, true, false);   // [K;Q] x W
+  constexpr uint32_t ID_S = idesc_bf16_f32(128, 64, false, false, false);  // [K;Q] x K^T
   constexpr uint32_t ID_UPD = idesc_bf16_f32(128, 64, false, true, true);  // P -= A x (eta G)
   constexpr uint32_t ID_DW = idesc_bf16_f32(128, 64, true, true, false);   // [K^T;K^T] x (eta G)
 
-  for (int c = 0; c < nchunks; ++c) {
-    const int ntok = min(CHUNK, T - c * CHUNK);
+  // Steps 1-3 of chunk c: wait for its tiles, issue S then P, precompute the
+  // P-independent part of this thread's LN backward, mask S into the A operand.
+  // This thread's K and Q rows: token MB (mb0 + i) + 8 hh + fr, i = 0, 1.
+  float2 u[2][8];
+  float um[2] = {0.f, 0.f};
+  auto chunk_head = [&](int c) {
+    const int ntok = chunk_tokens(c);
     const int nmb = ntok / MB;
     const uint32_t par = (uint32_t)c & 1u;
-
-    // ---- 1-2: tiles in; S = [K;Q] K^T first (the masking needs it), then P = [K;Q] W
     wait_or_abort(&bars[BAR_LOAD], par, abort);
     wait_or_abort(&bars[BAR_LOADQ], par, abort);
-    if (tid == 0 && !*abort) {
+    // Products are issued by one elected lane of a converged warp (the whole warp
+    // computes the operand descriptors).
+    if (warp == 0) {
+      __syncwarp();
+      const bool issue = elect_one_sync() && !*abort;
       tc_fence_after_sync();
-#pragma unroll
-      for (int n = 0; n < 4; ++n)
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          umma_ss(tS + 16 * n, smem_desc_sw128(aA + 32 * k, 16, 1024),
-                  smem_desc_sw128(sbase + k_block(n) + 32 * k, 16, 1024), ID_S, k > 0);
-      umma_commit(&bars[BAR_S]);
+      // S = [K;Q] K^T: B = the K rows alone (every other 8-row group, 2 KB apart).
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        umma_ss(tP, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aWhi + 2048 * k, 8192, 1024),
-                ID_PW, k > 0);
+        if (issue)
+          umma_ss(tS, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aA + 32 * k, 16, 2048), ID_S,
+                  k > 0);
+      if (issue) umma_commit(&bars[BAR_S]);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        umma_ss(tP, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aWlo + 2048 * k, 8192, 1024),
-                ID_PW, true);
-      umma_commit(&bars[BAR_P]);
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ak = smem_desc_sw128(aA + 32 * k, 16, 1024);
+        if (issue) umma_ss(tP, ak, smem_desc_sw128(aWhi + 2048 * k, 8192, 1024), ID_P, k > 0);
+        if (issue) umma_ss(tP, ak, smem_desc_sw128(aWlo + 2048 * k, 8192, 1024), ID_P, true);
+      }
+      if (issue) umma_commit(&bars[BAR_P]);
+      __syncwarp();
     }
     if (ntok < CHUNK) {  // ragged last chunk: absent tokens contribute nothing to dW
       for (int x = tid; x < (CHUNK - ntok) * 32; x += THREADS) {
@@ -255,71 +304,68 @@ __global__ void __launch_bounds__(THREADS, 4)
         *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(row, col)) = 0u;
       }
     }
-
-    // Everything of mini-batch `warp`'s LN backward that does not depend on P,
-    // computed while the tensor core works: u = 2 gamma (k + beta - v) (or v for
-    // the plain linear model) for this thread's two rows, and mean(u).
-    const int m = warp;
-    const int r0 = MB * m + fr, r1 = r0 + 8;  // tokens of this thread's two rows
-    float2 u0[8], u1[8];
-    float um0 = 0.f, um1 = 0.f;
-    if (m < nmb) {
-      const uint32_t kb = sbase + k_block(m);
+    // u = 2 gamma (k + beta - v) (or v for the plain linear model) and mean(u)
+    // for this thread's two K rows, while the tensor core works.
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = 8 * j + 2 * q4;
-        const float2 va = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r0, col)));
-        const float2 vc = unpack_bf16x2(lds_u32(aGlo + sw128_offset(r1, col)));
-        if (LN) {
-          const float2 ka = unpack_bf16x2(lds_u32(kb + sw128_offset(fr, col)));
-          const float2 kc = unpack_bf16x2(lds_u32(kb + sw128_offset(fr + 8, col)));
-          const float2 gm = *reinterpret_cast<const float2 *>(sm + OFF_GAMMA + 4 * col);
-          const float2 bt = *reinterpret_cast<const float2 *>(sm + OFF_BETA + 4 * col);
-          const float2 g2 = __fadd2_rn(gm, gm);
-          u0[j] = __fmul2_rn(g2, __fadd2_rn(ka, __fsub2(bt, va)));
-          u1[j] = __fmul2_rn(g2, __fadd2_rn(kc, __fsub2(bt, vc)));
-          um0 += u0[j].x + u0[j].y;
-          um1 += u1[j].x + u1[j].y;
-        } else {
-          u0[j] = va;
-          u1[j] = vc;
+    for (int i = 0; i < 2; ++i) {
+      const int tk = MB * (mb0 + i) + 8 * hh + fr;
+      um[i] = 0.f;
+      if (mb0 + i < nmb) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int col = 8 * j + 2 * q4;
+          const float2 v = unpack_bf16x2(lds_u32(aGlo + sw128_offset(tk, col)));
+          if (LN) {
+            const float2 k = unpack_bf16x2(lds_u32(sbase + kq_offset(tk, 0, col)));
+            const float2 gm = *reinterpret_cast<const float2 *>(sm + OFF_GAMMA + 4 * col);
+            const float2 bt = *reinterpret_cast<const float2 *>(sm + OFF_BETA + 4 * col);
+            u[i][j] = __fmul2_rn(__fadd2_rn(gm, gm), __fadd2_rn(k, __fsub2(bt, v)));
+            um[i] += u[i][j].x + u[i][j].y;
+          } else {
+            u[i][j] = v;
+          }
         }
-      }
-      if (LN) {
-        um0 = quad_sum(um0) * (1.f / D);
-        um1 = quad_sum(um1) * (1.f / D);
+        if (LN) um[i] = quad_sum(um[i]) * (1.f / D);
       }
     }
-    const float e0 = eta_s[r0], e1 = eta_s[r1];
-
     wait_or_abort(&bars[BAR_S], par, abort);
     tc_fence_after_sync();
     __syncwarp();  // lanes leave the wait loop independently; TMEM access is warp-collective
-
-    // ---- 3: mask this thread's row of S into the A operand (in place, per block) ------
     {
-      const bool qrow = lane >= 16;
-      const int t = MB * warp + (lane & 15);  // token of this row within the chunk
-      // Column blocks j > warp are zero for every row of this warp (K rows keep
-      // blocks < warp, Q rows blocks <= warp); TMEM loads and stores are
-      // warp-collective, so the skip is decided per warp.
+      // This thread's row of [K;Q]: group 4 warp + lane / 8.
+      const bool qrow = (lane >> 3) & 1;
+      const int mrow = mb0 + (lane >> 4);             // its mini-batch
+      const int t = MB * mrow + 8 * hh + (lane & 7);  // its token
+      // A block j (tokens 16j..16j+15, natural order) is read from S columns
+      // 8j..8j+7 (first half) and 32+8j..32+8j+7 (second half) and written back
+      // in place: hi over the first, lo over the second.  Blocks j > mb0 + 1 are
+      // zero for every row of this warp (the choice is per warp: TMEM access is
+      // warp-collective).
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        uint32_t v[16], hi[8], lo[8];
-        if (j <= warp) {
-          tmem_ld_32x32b_x16(tmem_addr(tS, 32 * warp, 16 * j), v);
+        uint32_t hi[8], lo[8];
+        if (j <= mb0 + 1) {
+          uint32_t v0[8], v1[8];
+          tmem_ld_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), v0);
+          tmem_ld_32x32b_x8(tmem_addr(tS, 32 * warp, 32 + 8 * j), v1);
           tmem_wait_ld();
-        }
-        const bool all_zero = qrow ? (j > warp) : (j >= warp);
+          const bool full = j < mrow;           // an earlier mini-batch: every column
+          const bool diag = qrow && j == mrow;  // own mini-batch of a Q row: s <= t
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int s0 = MB * j + 2 * e;
-          const float a = (!all_zero && (!qrow || s0 <= t)) ? __uint_as_float(v[2 * e]) : 0.f;
-          const float b = (!all_zero && (!qrow || s0 + 1 <= t)) ? __uint_as_float(v[2 * e + 1]) : 0.f;
-          split_bf16x2(a, b, hi[e], lo[e]);
+          for (int e = 0; e < 8; ++e) {
+            const int s0 = MB * j + 2 * e;
+            const uint32_t b0 = e < 4 ? v0[2 * e] : v1[2 * e - 8];
+            const uint32_t b1 = e < 4 ? v0[2 * e + 1] : v1[2 * e - 7];
+            const float a0 = (full || (diag && s0 <= t)) ? __uint_as_float(b0) : 0.f;
+            const float a1 = (full || (diag && s0 + 1 <= t)) ? __uint_as_float(b1) : 0.f;
+            split_bf16x2(a0, a1, hi[e], lo[e]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) hi[e] = lo[e] = 0u;
         }
-        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j), hi);
-        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 16 * j + 8), lo);
+        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), hi);
+        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 32 + 8 * j), lo);
       }
       tmem_wait_st();
     }
@@ -327,202 +373,183 @@ __global__ void __launch_bounds__(THREADS, 4)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
+  };
 
-    // ---- 4: the mini-batch chain: warp m handles mini-batch m ------------------------
-    if (m < nmb) {
+  if (nchunks > 0) chunk_head(0);
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int ntok = chunk_tokens(c);
+    const int nmb = ntok / MB;
+    const uint32_t par = (uint32_t)c & 1u;
+
+    // ---- 4: the mini-batch chain: mini-batch m on warps m/2 and 2 + m/2 ---------------
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int m = mb0 + i;
+      if (m >= nmb) break;
+      const int tk = MB * m + 8 * hh + fr;  // token of this thread's K row
+      const float e0 = eta_s[tk];
       wait_or_abort(&bars[m == 0 ? BAR_P : BAR_C0 + m - 1], par, abort);
       tc_fence_after_sync();
       __syncwarp();
-      uint32_t yr[32];
-      tmem_ld_16x256b_x8(tmem_addr(tP, 32 * m, 0), yr);
-      tmem_wait_ld();
-      float2 y0[8], y1[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        y0[j] = make_float2(__uint_as_float(yr[4 * j + 0]), __uint_as_float(yr[4 * j + 1]));
-        y1[j] = make_float2(__uint_as_float(yr[4 * j + 2]), __uint_as_float(yr[4 * j + 3]));
-      }
-      // Stores eta * (dl/dy) of one column pair of both rows as bf16 hi + lo; the
-      // lo half overwrites V, which this thread has read for exactly these cells.
-      auto store_grad = [&](int col, float2 g0, float2 g1) {
-        uint32_t h0, l0, h1, l1;
-        split_bf16x2(g0.x, g0.y, h0, l0);
-        split_bf16x2(g1.x, g1.y, h1, l1);
-        *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r0, col)) = h0;
-        *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r0, col)) = l0;
-        *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(r1, col)) = h1;
-        *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(r1, col)) = l1;
+      float2 y[8];
+      tmem_rows_16x256b(tmem_addr(tP, 32 * warp + 16 * i, 0), 0, y);
+      // Stores eta * (dl/dy) of one column pair as bf16 hi + lo; the lo half
+      // overwrites V, which this thread has read for exactly these cells.
+      auto store_grad = [&](int col, float2 g) {
+        uint32_t h, l;
+        split_bf16x2(g.x, g.y, h, l);
+        *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(tk, col)) = h;
+        *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(tk, col)) = l;
       };
       if (!LN) {
         // dl/dy = 2 (y - v)
-        const float2 f0 = make_float2(2.f * e0, 2.f * e0), f1 = make_float2(2.f * e1, 2.f * e1);
+        const float2 f = make_float2(2.f * e0, 2.f * e0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          store_grad(8 * j + 2 * q4, __fmul2_rn(f0, __fsub2(y0[j], u0[j])),
-                     __fmul2_rn(f1, __fsub2(y1[j], u1[j])));
+        for (int j = 0; j < 8; ++j) store_grad(8 * j + 2 * q4, __fmul2_rn(f, __fsub2(y[j], u[i][j])));
       } else {
         // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y.  With
         // dx = dl/dxhat = u + w xhat (w = 2 gamma^2), A = mean(dx), B = mean(dx xhat):
         // dl/dy = rstd (dx - A - xhat B) = rstd (u + xhat (w - B) - A).
-        const float mean0 = quad_sum(sum8(y0)) * (1.f / D);
-        const float mean1 = quad_sum(sum8(y1)) * (1.f / D);
-        const float2 nm0 = make_float2(-mean0, -mean0), nm1 = make_float2(-mean1, -mean1);
-        float2 q0a = make_float2(0.f, 0.f), q0b = q0a, q1a = q0a, q1b = q0a;
+        const float mean = quad_sum(sum8(y)) * (1.f / D);
+        const float2 nm = make_float2(-mean, -mean);
+        float2 qa = make_float2(0.f, 0.f), qb = qa;
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
-          y0[j] = __fadd2_rn(y0[j], nm0);
-          y0[j + 1] = __fadd2_rn(y0[j + 1], nm0);
-          y1[j] = __fadd2_rn(y1[j], nm1);
-          y1[j + 1] = __fadd2_rn(y1[j + 1], nm1);
-          q0a = __ffma2_rn(y0[j], y0[j], q0a);
-          q0b = __ffma2_rn(y0[j + 1], y0[j + 1], q0b);
-          q1a = __ffma2_rn(y1[j], y1[j], q1a);
-          q1b = __ffma2_rn(y1[j + 1], y1[j + 1], q1b);
+          y[j] = __fadd2_rn(y[j], nm);
+          y[j + 1] = __fadd2_rn(y[j + 1], nm);
+          qa = __ffma2_rn(y[j], y[j], qa);
+          qb = __ffma2_rn(y[j + 1], y[j + 1], qb);
         }
-        const float rstd0 = rsqrtf(quad_sum((q0a.x + q0b.x) + (q0a.y + q0b.y)) * (1.f / D) + p.eps);
-        const float rstd1 = rsqrtf(quad_sum((q1a.x + q1b.x) + (q1a.y + q1b.y)) * (1.f / D) + p.eps);
-        const float2 rs0 = make_float2(rstd0, rstd0), rs1 = make_float2(rstd1, rstd1);
-        float2 wx0 = make_float2(0.f, 0.f), wx1 = wx0, ux0 = wx0, ux1 = wx0, wxx0 = wx0, wxx1 = wx0;
+        const float rstd = rsqrtf(quad_sum((qa.x + qb.x) + (qa.y + qb.y)) * (1.f / D) + p.eps);
+        const float2 rs = make_float2(rstd, rstd);
+        float2 wx = make_float2(0.f, 0.f), ux = wx, wxx = wx;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float2 w2 = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
-          y0[j] = __fmul2_rn(y0[j], rs0);  // xhat
-          y1[j] = __fmul2_rn(y1[j], rs1);
-          const float2 wa = __fmul2_rn(w2, y0[j]), wb = __fmul2_rn(w2, y1[j]);
-          wx0 = __fadd2_rn(wx0, wa);
-          wx1 = __fadd2_rn(wx1, wb);
-          wxx0 = __ffma2_rn(wa, y0[j], wxx0);
-          wxx1 = __ffma2_rn(wb, y1[j], wxx1);
-          ux0 = __ffma2_rn(u0[j], y0[j], ux0);
-          ux1 = __ffma2_rn(u1[j], y1[j], ux1);
+          y[j] = __fmul2_rn(y[j], rs);  // xhat
+          const float2 ta = __fmul2_rn(w2, y[j]);
+          wx = __fadd2_rn(wx, ta);
+          wxx = __ffma2_rn(ta, y[j], wxx);
+          ux = __ffma2_rn(u[i][j], y[j], ux);
         }
-        const float A0 = um0 + quad_sum(wx0.x + wx0.y) * (1.f / D);
-        const float A1 = um1 + quad_sum(wx1.x + wx1.y) * (1.f / D);
-        const float B0 = quad_sum((ux0.x + ux0.y) + (wxx0.x + wxx0.y)) * (1.f / D);
-        const float B1 = quad_sum((ux1.x + ux1.y) + (wxx1.x + wxx1.y)) * (1.f / D);
-        const float2 f0 = make_float2(e0 * rstd0, e0 * rstd0), f1 = make_float2(e1 * rstd1, e1 * rstd1);
-        const float2 nA0 = make_float2(-A0, -A0), nA1 = make_float2(-A1, -A1);
-        const float2 nB0 = make_float2(-B0, -B0), nB1 = make_float2(-B1, -B1);
+        const float A = um[i] + quad_sum(wx.x + wx.y) * (1.f / D);
+        const float B = quad_sum((ux.x + ux.y) + (wxx.x + wxx.y)) * (1.f / D);
+        const float2 f = make_float2(e0 * rstd, e0 * rstd);
+        const float2 nA = make_float2(-A, -A), nB = make_float2(-B, -B);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const float2 w2 = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
-          const float2 ga = __fmul2_rn(f0, __fadd2_rn(__ffma2_rn(y0[j], __fadd2_rn(w2, nB0), u0[j]), nA0));
-          const float2 gb = __fmul2_rn(f1, __fadd2_rn(__ffma2_rn(y1[j], __fadd2_rn(w2, nB1), u1[j]), nA1));
-          store_grad(8 * j + 2 * q4, ga, gb);
+          store_grad(8 * j + 2 * q4,
+                     __fmul2_rn(f, __fadd2_rn(__ffma2_rn(y[j], __fadd2_rn(w2, nB), u[i][j]), nA)));
         }
       }
+      // Both halves of eta*G_m written: the pair's first warp issues the update.
       fence_proxy_async_smem();
       tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0 && !*abort) {
+      named_barrier_sync(1 + (warp & 1), 64);
+      if (hh == 0) {
+        __syncwarp();
+        const bool issue = elect_one_sync() && !*abort;
         tc_fence_after_sync();
         const uint64_t bhi = smem_desc_sw128(aGhi + 2048 * m, 8192, 1024);
         const uint64_t blo = smem_desc_sw128(aGlo + 2048 * m, 8192, 1024);
-        umma_ts(tP, tS + 16 * m, bhi, ID_UPD, true);
-        umma_ts(tP, tS + 16 * m, blo, ID_UPD, true);
-        umma_ts(tP, tS + 16 * m + 8, bhi, ID_UPD, true);
-        umma_commit(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
+        if (issue) umma_ts(tP, tS + 8 * m, bhi, ID_UPD, true);       // A hi x G hi
+        if (issue) umma_ts(tP, tS + 8 * m, blo, ID_UPD, true);       // A hi x G lo
+        if (issue) umma_ts(tP, tS + 32 + 8 * m, bhi, ID_UPD, true);  // A lo x G hi
+        if (issue) umma_commit(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
+        __syncwarp();
       }
-      __syncwarp();
+    }
 
-      // ---- 5: output of this mini-batch's Q rows.  After update m their value is
-      // final: later updates add exactly zero to them (A is zero there).
+    // Outputs of this warp's Q rows: after their mini-batch's update they are
+    // final (later updates add exactly zero to them, A being zero there).
+    float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int m = mb0 + i;
+      if (m >= nmb) break;
+      const int tq = MB * m + 8 * hh + fr;  // token of this thread's Q row
       wait_or_abort(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m], par, abort);
       tc_fence_after_sync();
       __syncwarp();
-      uint32_t zr[32];
-      tmem_ld_16x256b_x8(tmem_addr(tP, 32 * m + 16, 0), zr);
-      tmem_wait_ld();
-      float2 z0[8], z1[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        z0[j] = make_float2(__uint_as_float(zr[4 * j + 0]), __uint_as_float(zr[4 * j + 1]));
-        z1[j] = make_float2(__uint_as_float(zr[4 * j + 2]), __uint_as_float(zr[4 * j + 3]));
-      }
-      float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
-      const bool ok0 = r0 < ntok, ok1 = r1 < ntok;
-      const uint32_t qb = sbase + q_block(m);
+      float2 z[8];
+      tmem_rows_16x256b(tmem_addr(tP, 32 * warp + 16 * i, 0), 1, z);
+      float *zrow = Zc + tq * D;
       if (LN) {
-        const float mean0 = quad_sum(sum8(z0)) * (1.f / D);
-        const float mean1 = quad_sum(sum8(z1)) * (1.f / D);
-        const float2 nm0 = make_float2(-mean0, -mean0), nm1 = make_float2(-mean1, -mean1);
-        float2 q0a = make_float2(0.f, 0.f), q0b = q0a, q1a = q0a, q1b = q0a;
+        const float mean = quad_sum(sum8(z)) * (1.f / D);
+        const float2 nm = make_float2(-mean, -mean);
+        float2 qa = make_float2(0.f, 0.f), qb = qa;
 #pragma unroll
         for (int j = 0; j < 8; j += 2) {
-          z0[j] = __fadd2_rn(z0[j], nm0);
-          z0[j + 1] = __fadd2_rn(z0[j + 1], nm0);
-          z1[j] = __fadd2_rn(z1[j], nm1);
-          z1[j + 1] = __fadd2_rn(z1[j + 1], nm1);
-          q0a = __ffma2_rn(z0[j], z0[j], q0a);
-          q0b = __ffma2_rn(z0[j + 1], z0[j + 1], q0b);
-          q1a = __ffma2_rn(z1[j], z1[j], q1a);
-          q1b = __ffma2_rn(z1[j + 1], z1[j + 1], q1b);
+          z[j] = __fadd2_rn(z[j], nm);
+          z[j + 1] = __fadd2_rn(z[j + 1], nm);
+          qa = __ffma2_rn(z[j], z[j], qa);
+          qb = __ffma2_rn(z[j + 1], z[j + 1], qb);
         }
-        const float rstd0 = rsqrtf(quad_sum((q0a.x + q0b.x) + (q0a.y + q0b.y)) * (1.f / D) + p.eps);
-        const float rstd1 = rsqrtf(quad_sum((q1a.x + q1b.x) + (q1a.y + q1b.y)) * (1.f / D) + p.eps);
-        const float2 rs0 = make_float2(rstd0, rstd0), rs1 = make_float2(rstd1, rstd1);
+        const float rstd = rsqrtf(quad_sum((qa.x + qb.x) + (qa.y + qb.y)) * (1.f / D) + p.eps);
+        const float2 rs = make_float2(rstd, rstd);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int col = 8 * j + 2 * q4;
           const float2 gm = *reinterpret_cast<const float2 *>(sm + OFF_GAMMA + 4 * col);
           const float2 bt = *reinterpret_cast<const float2 *>(sm + OFF_BETA + 4 * col);
-          const float2 qa = unpack_bf16x2(lds_u32(qb + sw128_offset(fr, col)));
-          const float2 qc = unpack_bf16x2(lds_u32(qb + sw128_offset(fr + 8, col)));
-          if (ok0)
-            *reinterpret_cast<float2 *>(Zc + r0 * D + col) =
-                __fadd2_rn(qa, __ffma2_rn(gm, __fmul2_rn(z0[j], rs0), bt));
-          if (ok1)
-            *reinterpret_cast<float2 *>(Zc + r1 * D + col) =
-                __fadd2_rn(qc, __ffma2_rn(gm, __fmul2_rn(z1[j], rs1), bt));
+          const float2 q = unpack_bf16x2(lds_u32(sbase + kq_offset(tq, 1, col)));
+          *reinterpret_cast<float2 *>(zrow + col) = __fadd2_rn(q, __ffma2_rn(gm, __fmul2_rn(z[j], rs), bt));
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          if (ok0) *reinterpret_cast<float2 *>(Zc + r0 * D + col) = z0[j];
-          if (ok1) *reinterpret_cast<float2 *>(Zc + r1 * D + col) = z1[j];
-        }
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<float2 *>(zrow + 8 * j + 2 * q4) = z[j];
       }
-      // This warp's Q block is no longer needed: refill it with the next chunk.
-      // The Q barrier completes only when all four warps have arrived, i.e. after
-      // every thread has passed its wait on this chunk's Q phase.
-      __syncwarp();
-      if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q_block(c + 1, m);
     }
+    // This warp's Q rows are no longer needed: refill them with the next chunk.
+    __syncwarp();
+    if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
 
-    // ---- 6: dW on the tensor core after the last update; state update -------------
+    // ---- 5: dW on the tensor core after the last update; state update -------------
     wait_or_abort(&bars[BAR_LAST], par, abort);
     tc_fence_after_sync();
-    if (tid == 0 && !*abort) {
+    if (warp == 0) {
+      __syncwarp();
+      const bool issue = elect_one_sync() && !*abort;
+      // dW = K^T (eta G) into the S columns (their operand is consumed).  Step k
+      // takes the K rows of groups 4k and 4k + 2 (tokens of mini-batches
+      // 2(k % 2), 2(k % 2) + 1, half k / 2), read twice (lbo 0) so that rows
+      // 64..127 repeat rows 0..63 for warps 2-3, against the eta*G rows of the
+      // same tokens (two 8-row groups 2 KB apart).
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        umma_ss(tS, smem_desc_sw128(sbase + k_block(k), 0, 1024), smem_desc_sw128(aGhi + 2048 * k, 8192, 1024),
-                ID_DW, k > 0);
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        umma_ss(tS, smem_desc_sw128(sbase + k_block(k), 0, 1024), smem_desc_sw128(aGlo + 2048 * k, 8192, 1024),
-                ID_DW, true);
-      umma_commit(&bars[BAR_DW]);
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ak = smem_desc_sw128(aA + 4096 * k, 0, 2048);
+        const uint32_t gk = 4096u * (k & 1) + 1024u * (k >> 1);
+        if (issue) umma_ss(tS, ak, smem_desc_sw128(aGhi + gk, 8192, 2048), ID_DW, k > 0);
+        if (issue) umma_ss(tS, ak, smem_desc_sw128(aGlo + gk, 8192, 2048), ID_DW, true);
+      }
+      if (issue) umma_commit(&bars[BAR_DW]);
+      __syncwarp();
     }
     wait_or_abort(&bars[BAR_DW], par, abort);
     tc_fence_after_sync();
     __syncwarp();
     // K, V (lo half of eta*G) and eta are free once dW is done; every thread passed
-    // this chunk's wait on their barrier before the A-operand barrier above.
+    // this chunk's wait on their barrier in the chunk head.
     if (tid == 0 && c + 1 < nchunks && !*abort) issue_loads_kv(c + 1);
     {
-      uint32_t dw[32];
-      tmem_ld_32x32b_x32(tmem_addr(tS, 32 * warp, wc0), dw);
-      tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) wm[e] -= __uint_as_float(dw[e]);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t dw[16];
+        tmem_ld_32x32b_x16(tmem_addr(tS, 32 * warp, wc0 + 16 * h), dw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) wm[16 * h + e] -= __uint_as_float(dw[e]);
+      }
       write_w_operand();
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
-    __syncthreads();
+    __syncthreads();  // P and S of this chunk fully consumed; W operand written
     tc_fence_after_sync();
     if (*abort) break;
+    if (c + 1 < nchunks) chunk_head(c + 1);
   }
 
   // Final state.

@@ -198,13 +198,12 @@ template <bool LN>
 int launch_linear_tc(const Call &c) {
   const long long units = (long long)c.B * c.H;
   CUtensorMap mq, mk, mv;
-  // Q and K arrive as one 16-token box per mini-batch (interleaved operand), V as
+  // Q and K arrive as 8-token boxes (the row groups of the [K;Q] operand), V as
   // one 64-token box per chunk.
-  if (!make_qkv_map(&mq, c.Q, c.T, units, tc::MB) || !make_qkv_map(&mk, c.K, c.T, units, tc::MB) ||
+  if (!make_qkv_map(&mq, c.Q, c.T, units, 8) || !make_qkv_map(&mk, c.K, c.T, units, 8) ||
       !make_qkv_map(&mv, c.V, c.T, units, tc::CHUNK))
     return TTT_ERR_CUDA;
   tc::Params p;
-  p.Q = static_cast<const __nv_bfloat16 *>(c.Q);
   p.eta = c.eta;
   p.W0 = c.W0;
   p.gamma = c.gamma;
