@@ -80,10 +80,12 @@ constexpr uint32_t OFF_ETA = 49152;    // eta of the chunk, 64 floats
 constexpr uint32_t OFF_GAMMA = 49408;  // LN gamma, 64 floats
 constexpr uint32_t OFF_BETA = 49664;   // LN beta, 64 floats
 constexpr uint32_t OFF_W2 = 49920;     // 2 gamma^2, 64 floats
-constexpr uint32_t OFF_BAR = 50176;    // mbarriers (9 x 8 bytes)
-constexpr uint32_t OFF_TSLOT = 50248;  // TMEM base address
-constexpr uint32_t OFF_ABORT = 50252;  // set when a bounded wait expired
-constexpr uint32_t SMEM_USED = 50256;
+constexpr uint32_t OFF_G2 = 50176;     // 2 gamma, 64 floats
+constexpr uint32_t OFF_G2B = 50432;    // 2 gamma beta, 64 floats
+constexpr uint32_t OFF_BAR = 50688;    // mbarriers (9 x 8 bytes)
+constexpr uint32_t OFF_TSLOT = 50760;  // TMEM base address
+constexpr uint32_t OFF_ABORT = 50764;  // set when a bounded wait expired
+constexpr uint32_t SMEM_USED = 50768;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 // 8-row group of token `row` of the chunk in the [K;Q] operand: K (q = 0) or Q
@@ -192,6 +194,8 @@ __global__ void __launch_bounds__(THREADS, 4)
     reinterpret_cast<float *>(sm + OFF_GAMMA)[tid] = g;
     reinterpret_cast<float *>(sm + OFF_BETA)[tid] = p.beta[head * D + tid];
     reinterpret_cast<float *>(sm + OFF_W2)[tid] = 2.f * g * g;
+    reinterpret_cast<float *>(sm + OFF_G2)[tid] = 2.f * g;
+    reinterpret_cast<float *>(sm + OFF_G2B)[tid] = 2.f * g * p.beta[head * D + tid];
   }
 
   // Each thread owns 32 elements of the fp32 state: row wi, columns wc0..wc0+31
@@ -264,14 +268,42 @@ __global__ void __launch_bounds__(THREADS, 4)
   constexpr uint32_t ID_UPD = idesc_bf16_f32(128, 64, false, true, true);  // P -= A x (eta G)
   constexpr uint32_t ID_DW = idesc_bf16_f32(128, 64, true, true, false);   // [K^T;K^T] x (eta G)
 
-  // Steps 1-3 of chunk c: wait for its tiles, issue S then P, precompute the
-  // P-independent part of this thread's LN backward, mask S into the A operand.
-  // This thread's K and Q rows: token MB (mb0 + i) + 8 hh + fr, i = 0, 1.
-  float2 u[2][8];
-  float um[2] = {0.f, 0.f};
+  // The P-independent part of the LN backward of this thread's K row of token
+  // tk: u = 2 gamma (k + beta - v) = g2 (k - v) + g2b (or v for the plain linear
+  // model) and mean(u), from k and v (kr, vr: bf16 pairs).
+  uint32_t kr[8], vr[8];
+  float2 u[8];
+  float um = 0.f;
+  auto load_kv = [&](int tk) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int col = 8 * j + 2 * q4;
+      vr[j] = lds_u32(aGlo + sw128_offset(tk, col));
+      if (LN) kr[j] = lds_u32(sbase + kq_offset(tk, 0, col));
+    }
+  };
+  auto make_u = [&]() {
+    um = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float2 v = unpack_bf16x2(vr[j]);
+      if (LN) {
+        const int col = 8 * j + 2 * q4;
+        const float2 g2 = *reinterpret_cast<const float2 *>(sm + OFF_G2 + 4 * col);
+        const float2 g2b = *reinterpret_cast<const float2 *>(sm + OFF_G2B + 4 * col);
+        u[j] = __ffma2_rn(g2, __fsub2(unpack_bf16x2(kr[j]), v), g2b);
+        um += u[j].x + u[j].y;
+      } else {
+        u[j] = v;
+      }
+    }
+    if (LN) um = quad_sum(um) * (1.f / D);
+  };
+
+  // Steps 1-3 of chunk c: wait for its tiles, issue S then P, mask S into the A
+  // operand.  This thread's K and Q rows: token MB (mb0 + i) + 8 hh + fr, i = 0, 1.
   auto chunk_head = [&](int c) {
     const int ntok = chunk_tokens(c);
-    const int nmb = ntok / MB;
     const uint32_t par = (uint32_t)c & 1u;
     wait_or_abort(&bars[BAR_LOAD], par, abort);
     wait_or_abort(&bars[BAR_LOADQ], par, abort);
@@ -302,30 +334,6 @@ __global__ void __launch_bounds__(THREADS, 4)
         const int row = ntok + x / 32, col = 2 * (x % 32);
         *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(row, col)) = 0u;
         *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(row, col)) = 0u;
-      }
-    }
-    // u = 2 gamma (k + beta - v) (or v for the plain linear model) and mean(u)
-    // for this thread's two K rows, while the tensor core works.
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int tk = MB * (mb0 + i) + 8 * hh + fr;
-      um[i] = 0.f;
-      if (mb0 + i < nmb) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int col = 8 * j + 2 * q4;
-          const float2 v = unpack_bf16x2(lds_u32(aGlo + sw128_offset(tk, col)));
-          if (LN) {
-            const float2 k = unpack_bf16x2(lds_u32(sbase + kq_offset(tk, 0, col)));
-            const float2 gm = *reinterpret_cast<const float2 *>(sm + OFF_GAMMA + 4 * col);
-            const float2 bt = *reinterpret_cast<const float2 *>(sm + OFF_BETA + 4 * col);
-            u[i][j] = __fmul2_rn(__fadd2_rn(gm, gm), __fadd2_rn(k, __fsub2(bt, v)));
-            um[i] += u[i][j].x + u[i][j].y;
-          } else {
-            u[i][j] = v;
-          }
-        }
-        if (LN) um[i] = quad_sum(um[i]) * (1.f / D);
       }
     }
     wait_or_abort(&bars[BAR_S], par, abort);
@@ -389,6 +397,10 @@ __global__ void __launch_bounds__(THREADS, 4)
       if (m >= nmb) break;
       const int tk = MB * m + 8 * hh + fr;  // token of this thread's K row
       const float e0 = eta_s[tk];
+      // The P-independent part of the LN backward, while the previous update is
+      // in flight.
+      load_kv(tk);
+      make_u();
       wait_or_abort(&bars[m == 0 ? BAR_P : BAR_C0 + m - 1], par, abort);
       tc_fence_after_sync();
       __syncwarp();
@@ -406,7 +418,7 @@ __global__ void __launch_bounds__(THREADS, 4)
         // dl/dy = 2 (y - v)
         const float2 f = make_float2(2.f * e0, 2.f * e0);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) store_grad(8 * j + 2 * q4, __fmul2_rn(f, __fsub2(y[j], u[i][j])));
+        for (int j = 0; j < 8; ++j) store_grad(8 * j + 2 * q4, __fmul2_rn(f, __fsub2(y[j], u[j])));
       } else {
         // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y.  With
         // dx = dl/dxhat = u + w xhat (w = 2 gamma^2), A = mean(dx), B = mean(dx xhat):
@@ -431,9 +443,9 @@ __global__ void __launch_bounds__(THREADS, 4)
           const float2 ta = __fmul2_rn(w2, y[j]);
           wx = __fadd2_rn(wx, ta);
           wxx = __ffma2_rn(ta, y[j], wxx);
-          ux = __ffma2_rn(u[i][j], y[j], ux);
+          ux = __ffma2_rn(u[j], y[j], ux);
         }
-        const float A = um[i] + quad_sum(wx.x + wx.y) * (1.f / D);
+        const float A = um + quad_sum(wx.x + wx.y) * (1.f / D);
         const float B = quad_sum((ux.x + ux.y) + (wxx.x + wxx.y)) * (1.f / D);
         const float2 f = make_float2(e0 * rstd, e0 * rstd);
         const float2 nA = make_float2(-A, -A), nB = make_float2(-B, -B);
@@ -441,7 +453,7 @@ __global__ void __launch_bounds__(THREADS, 4)
         for (int j = 0; j < 8; ++j) {
           const float2 w2 = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
           store_grad(8 * j + 2 * q4,
-                     __fmul2_rn(f, __fadd2_rn(__ffma2_rn(y[j], __fadd2_rn(w2, nB), u[i][j]), nA)));
+                     __fmul2_rn(f, __fadd2_rn(__ffma2_rn(y[j], __fadd2_rn(w2, nB), u[j]), nA)));
         }
       }
       // Both halves of eta*G_m written: the pair's first warp issues the update.
