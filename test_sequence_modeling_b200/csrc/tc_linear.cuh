@@ -77,11 +77,9 @@ constexpr uint32_t OFF_WLO = 24576;    // W lo
 constexpr uint32_t OFF_GHI = 32768;    // eta*G hi [token][d_out] bf16
 constexpr uint32_t OFF_GLO = 40960;    // V tile on arrival; eta*G lo once a mini-batch is done
 constexpr uint32_t OFF_ETA = 49152;    // eta of the chunk, 64 floats
-constexpr uint32_t OFF_GAMMA = 49408;  // LN gamma, 64 floats
-constexpr uint32_t OFF_BETA = 49664;   // LN beta, 64 floats
-constexpr uint32_t OFF_W2 = 49920;     // 2 gamma^2, 64 floats
-constexpr uint32_t OFF_G2 = 50176;     // 2 gamma, 64 floats
-constexpr uint32_t OFF_G2B = 50432;    // 2 gamma beta, 64 floats
+constexpr uint32_t OFF_GB = 49408;     // per column pair {gamma x2, beta x2}, 32 x 16 bytes
+constexpr uint32_t OFF_UC = 49920;     // per column pair {2 gamma x2, 2 gamma beta x2}
+constexpr uint32_t OFF_W2 = 50432;     // 2 gamma^2, 64 floats
 constexpr uint32_t OFF_BAR = 50688;    // mbarriers (9 x 8 bytes)
 constexpr uint32_t OFF_TSLOT = 50760;  // TMEM base address
 constexpr uint32_t OFF_ABORT = 50764;  // set when a bounded wait expired
@@ -101,14 +99,14 @@ __device__ __forceinline__ uint32_t kq_offset(int row, int q, int col) {
 // base + i/4, which = 1: lane base + 8 + i/4), all 64 columns, as column pairs
 // 8j + 2(i%4) + {0,1}; two 32-column loads keep the live registers low.
 __device__ __forceinline__ void tmem_rows_16x256b(uint32_t taddr, int which, float2 (&y)[8]) {
+  uint32_t r0[16], r1[16];
+  tmem_ld_16x256b_x4(taddr, r0);
+  tmem_ld_16x256b_x4(taddr + 32, r1);
+  tmem_wait_ld();
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    uint32_t r[16];
-    tmem_ld_16x256b_x4(taddr + 32 * h, r);
-    tmem_wait_ld();
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-      y[4 * h + j] = make_float2(__uint_as_float(r[4 * j + 2 * which]), __uint_as_float(r[4 * j + 2 * which + 1]));
+  for (int j = 0; j < 4; ++j) {
+    y[j] = make_float2(__uint_as_float(r0[4 * j + 2 * which]), __uint_as_float(r0[4 * j + 2 * which + 1]));
+    y[4 + j] = make_float2(__uint_as_float(r1[4 * j + 2 * which]), __uint_as_float(r1[4 * j + 2 * which + 1]));
   }
 }
 
@@ -191,11 +189,14 @@ __global__ void __launch_bounds__(THREADS, 4)
   }
   if (LN && tid < D) {
     const float g = p.gamma[head * D + tid];
-    reinterpret_cast<float *>(sm + OFF_GAMMA)[tid] = g;
-    reinterpret_cast<float *>(sm + OFF_BETA)[tid] = p.beta[head * D + tid];
+    const float b = p.beta[head * D + tid];
+    float *gb = reinterpret_cast<float *>(sm + OFF_GB + 16 * (tid >> 1)) + (tid & 1);
+    float *uc = reinterpret_cast<float *>(sm + OFF_UC + 16 * (tid >> 1)) + (tid & 1);
+    gb[0] = g;
+    gb[2] = b;
+    uc[0] = 2.f * g;
+    uc[2] = 2.f * g * b;
     reinterpret_cast<float *>(sm + OFF_W2)[tid] = 2.f * g * g;
-    reinterpret_cast<float *>(sm + OFF_G2)[tid] = 2.f * g;
-    reinterpret_cast<float *>(sm + OFF_G2B)[tid] = 2.f * g * p.beta[head * D + tid];
   }
 
   // Each thread owns 32 elements of the fp32 state: row wi, columns wc0..wc0+31
@@ -288,10 +289,8 @@ __global__ void __launch_bounds__(THREADS, 4)
     for (int j = 0; j < 8; ++j) {
       const float2 v = unpack_bf16x2(vr[j]);
       if (LN) {
-        const int col = 8 * j + 2 * q4;
-        const float2 g2 = *reinterpret_cast<const float2 *>(sm + OFF_G2 + 4 * col);
-        const float2 g2b = *reinterpret_cast<const float2 *>(sm + OFF_G2B + 4 * col);
-        u[j] = __ffma2_rn(g2, __fsub2(unpack_bf16x2(kr[j]), v), g2b);
+        const float4 c = *reinterpret_cast<const float4 *>(sm + OFF_UC + 16 * (4 * j + q4));
+        u[j] = __ffma2_rn(make_float2(c.x, c.y), __fsub2(unpack_bf16x2(kr[j]), v), make_float2(c.z, c.w));
         um += u[j].x + u[j].y;
       } else {
         u[j] = v;
@@ -422,38 +421,35 @@ __global__ void __launch_bounds__(THREADS, 4)
       } else {
         // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y.  With
         // dx = dl/dxhat = u + w xhat (w = 2 gamma^2), A = mean(dx), B = mean(dx xhat):
-        // dl/dy = rstd (dx - A - xhat B) = rstd (u + xhat (w - B) - A).
+        // dl/dy = r (dx - A - xhat B) = r (u + xhat (w - B) - A), r = 1/std(y).
+        // With d = y - mean(y) and xhat = r d, every sum needed is a sum over d:
+        // A = mean(u) + r sum(w d) / D, B = r sum(u d) / D + r^2 sum(w d^2) / D,
+        // so one reduction round follows the one for the mean.
         const float mean = quad_sum(sum8(y)) * (1.f / D);
         const float2 nm = make_float2(-mean, -mean);
-        float2 qa = make_float2(0.f, 0.f), qb = qa;
-#pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-          y[j] = __fadd2_rn(y[j], nm);
-          y[j + 1] = __fadd2_rn(y[j + 1], nm);
-          qa = __ffma2_rn(y[j], y[j], qa);
-          qb = __ffma2_rn(y[j + 1], y[j + 1], qb);
-        }
-        const float rstd = rsqrtf(quad_sum((qa.x + qb.x) + (qa.y + qb.y)) * (1.f / D) + p.eps);
-        const float2 rs = make_float2(rstd, rstd);
-        float2 wx = make_float2(0.f, 0.f), ux = wx, wxx = wx;
+        float2 w2[8];
+        float2 sdd = make_float2(0.f, 0.f), swd = sdd, swdd = sdd, sud = sdd;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float2 w2 = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
-          y[j] = __fmul2_rn(y[j], rs);  // xhat
-          const float2 ta = __fmul2_rn(w2, y[j]);
-          wx = __fadd2_rn(wx, ta);
-          wxx = __ffma2_rn(ta, y[j], wxx);
-          ux = __ffma2_rn(u[j], y[j], ux);
+          w2[j] = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
+          y[j] = __fadd2_rn(y[j], nm);  // d
+          const float2 t = __fmul2_rn(w2[j], y[j]);
+          swd = __fadd2_rn(swd, t);
+          swdd = __ffma2_rn(t, y[j], swdd);
+          sdd = __ffma2_rn(y[j], y[j], sdd);
+          sud = __ffma2_rn(u[j], y[j], sud);
         }
-        const float A = um + quad_sum(wx.x + wx.y) * (1.f / D);
-        const float B = quad_sum((ux.x + ux.y) + (wxx.x + wxx.y)) * (1.f / D);
-        const float2 f = make_float2(e0 * rstd, e0 * rstd);
+        const float vdd = quad_sum(sdd.x + sdd.y), vwd = quad_sum(swd.x + swd.y);
+        const float vwdd = quad_sum(swdd.x + swdd.y), vud = quad_sum(sud.x + sud.y);
+        const float r = rsqrtf(vdd * (1.f / D) + p.eps);
+        const float A = um + r * vwd * (1.f / D);
+        const float B = (r * vud + r * r * vwdd) * (1.f / D);
+        const float2 f = make_float2(e0 * r, e0 * r), rr = make_float2(r, r);
         const float2 nA = make_float2(-A, -A), nB = make_float2(-B, -B);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const float2 w2 = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
-          store_grad(8 * j + 2 * q4,
-                     __fmul2_rn(f, __fadd2_rn(__ffma2_rn(y[j], __fadd2_rn(w2, nB), u[j]), nA)));
+          const float2 xh = __fmul2_rn(y[j], rr);
+          store_grad(8 * j + 2 * q4, __fmul2_rn(f, __fadd2_rn(__ffma2_rn(xh, __fadd2_rn(w2[j], nB), u[j]), nA)));
         }
       }
       // Both halves of eta*G_m written: the pair's first warp issues the update.
@@ -504,8 +500,8 @@ __global__ void __launch_bounds__(THREADS, 4)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int col = 8 * j + 2 * q4;
-          const float2 gm = *reinterpret_cast<const float2 *>(sm + OFF_GAMMA + 4 * col);
-          const float2 bt = *reinterpret_cast<const float2 *>(sm + OFF_BETA + 4 * col);
+          const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_GB + 16 * (4 * j + q4));
+          const float2 gm = make_float2(gb.x, gb.y), bt = make_float2(gb.z, gb.w);
           const float2 q = unpack_bf16x2(lds_u32(sbase + kq_offset(tq, 1, col)));
           *reinterpret_cast<float2 *>(zrow + col) = __fadd2_rn(q, __ffma2_rn(gm, __fmul2_rn(z[j], rs), bt));
         }
