@@ -140,6 +140,17 @@ TTT_API int ttt_set_path(int path);
 /* Number of CUDA kernels this library enqueued since load (for launch accounting). */
 TTT_API long long ttt_launch_count(void);
 
+/*
+ * Test hook for the timeout path (no counterpart in the method).  While on,
+ * every CTA of the tensor-core kernels launched by later calls first waits on a
+ * barrier that nothing arrives at, bounded at ~2^20 SM cycles: the wait
+ * expires, the CTA records TTT_ERR_TIMEOUT in the device status word, skips its
+ * remaining work (its outputs are then undefined), waits (bounded) for its own
+ * loads and tensor-core products in flight, frees its tensor memory and
+ * returns.  No GPU fault is involved.  Returns the previous setting (0 or 1).
+ */
+TTT_API int ttt_debug_inject_timeout(int on);
+
 #ifdef __cplusplus
 }
 #endif

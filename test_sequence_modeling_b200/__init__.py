@@ -4,15 +4,15 @@ The computation lives in ``libttt.so`` (C ABI in ``include/ttt.h``); the
 functions below are its Python binding over torch CUDA tensors.  ``inputs``
 holds the seeded synthetic workloads.
 """
-from ._lib import (TTT_BF16, TTT_F32, TTT_PATH_AUTO, TTT_PATH_SIMT, TTT_PATH_TC,  # noqa: F401
-                   TTTError)
+from ._lib import (TTT_BF16, TTT_ERR_TIMEOUT, TTT_F32, TTT_OK, TTT_PATH_AUTO,  # noqa: F401
+                   TTT_PATH_SIMT, TTT_PATH_TC, TTTError)
 
 
 def __getattr__(name):
     # The torch-facing binding is imported on first use so that ``inputs`` and the
     # ABI constants stay importable without touching CUDA.
     if name in ("ttt_linear_fwd", "ttt_linear_ln_fwd", "ttt_mlp_fwd", "set_path",
-                "last_device_status", "launch_count"):
+                "last_device_status", "launch_count", "debug_inject_timeout"):
         from . import ttt
         return getattr(ttt, name)
     raise AttributeError(name)

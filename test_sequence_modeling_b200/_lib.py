@@ -24,6 +24,7 @@ SIGNATURES = {
     "ttt_last_device_status": (_i, [_vp]),
     "ttt_set_path": (_i, [_i]),
     "ttt_launch_count": (ctypes.c_longlong, []),
+    "ttt_debug_inject_timeout": (_i, [_i]),
 }
 
 _lib = None

@@ -80,10 +80,10 @@ constexpr uint32_t OFF_ETA = 49152;    // eta of the chunk, 64 floats
 constexpr uint32_t OFF_GB = 49408;     // per column pair {gamma x2, beta x2}, 32 x 16 bytes
 constexpr uint32_t OFF_UC = 49920;     // per column pair {2 gamma x2, 2 gamma beta x2}
 constexpr uint32_t OFF_W2 = 50432;     // 2 gamma^2, 64 floats
-constexpr uint32_t OFF_BAR = 50688;    // mbarriers (9 x 8 bytes)
-constexpr uint32_t OFF_TSLOT = 50760;  // TMEM base address
-constexpr uint32_t OFF_ABORT = 50764;  // set when a bounded wait expired
-constexpr uint32_t SMEM_USED = 50768;
+constexpr uint32_t OFF_BAR = 50688;    // mbarriers (14 x 8 bytes)
+constexpr uint32_t OFF_TSLOT = 50800;  // TMEM base address
+constexpr uint32_t OFF_ABORT = 50804;  // set when a bounded wait expired
+constexpr uint32_t SMEM_USED = 50808;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 
 // 8-row group of token `row` of the chunk in the [K;Q] operand: K (q = 0) or Q
@@ -111,8 +111,15 @@ __device__ __forceinline__ void tmem_rows_16x256b(uint32_t taddr, int which, flo
 }
 
 // mbarriers: K/V/eta loads; MMA S; updates of mini-batches 0,1,2; last update;
-// dW; Q loads (four arrivals: one per warp); MMA P.
-enum { BAR_LOAD = 0, BAR_S = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, BAR_LOADQ = 7, BAR_P = 8, NUM_BARS = 9 };
+// dW; Q loads of warps 0..3; MMA P; the drain of an aborted CTA's products; one
+// that nothing arrives at (the injected-timeout test).
+enum {
+  BAR_LOAD = 0, BAR_S = 1, BAR_C0 = 2, BAR_LAST = 5, BAR_DW = 6, BAR_LOADQ = 7, BAR_P = 11,
+  BAR_DRAIN = 12, BAR_NEVER = 13, NUM_BARS = 14
+};
+// Bound of every wait (SM cycles, ~2 s) and of the injected one.
+constexpr long long WAIT_LIMIT = 1ll << 32;
+constexpr long long INJECTED_WAIT_LIMIT = 1ll << 20;
 
 struct Params {
   const float *eta;
@@ -122,6 +129,7 @@ struct Params {
   int H, T;
   float *Z;
   float *W_out;
+  int inject_timeout;  // test hook: start with a wait that nothing completes
 };
 
 __device__ __forceinline__ float sum8(const float2 (&x)[8]) {
@@ -142,9 +150,10 @@ __device__ __forceinline__ float quad_sum(float x) {
 }
 
 // Waits, or flags the CTA as aborted and records the timeout if the wait expires.
-__device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                              long long limit = WAIT_LIMIT) {
   if (*abort) return;
-  if (!mbar_wait(bar, parity)) {
+  if (!mbar_wait(bar, parity, limit)) {
     *abort = 1;
     record_device_error(-5 /* TTT_ERR_TIMEOUT */);
   }
@@ -176,7 +185,7 @@ __global__ void __launch_bounds__(THREADS, 4)
   const int hh = warp >> 1;        // ... half hh of each
 
   if (tid == 0) {
-    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], i == BAR_LOADQ ? 4 : 1);
+    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], i == BAR_DRAIN ? 64 : 1);
     *abort = 0;
     fence_mbarrier_init();
     prefetch_tensormap(&tmQ);
@@ -236,7 +245,11 @@ __global__ void __launch_bounds__(THREADS, 4)
   // Loads are split so that each tile is fetched as soon as its buffer is free:
   // each warp refills its own Q rows once it has written its outputs, thread 0
   // refills K / V / eta once dW is computed.
+  // The last chunk whose loads this thread issued (thread 0: K, V, eta; lane 0
+  // of each warp: its Q rows), for the drain of an aborted CTA.
+  int kv_last = -1, q_last = -1;
   auto issue_loads_kv = [&](int c) {
+    kv_last = c;
     const int ntok = chunk_tokens(c);
     mbar_arrive_expect_tx(&bars[BAR_LOAD], 8u * 1024u + 8192u + (uint32_t)ntok * 4u);
 #pragma unroll
@@ -245,13 +258,15 @@ __global__ void __launch_bounds__(THREADS, 4)
     tma_load_3d(sm + OFF_GLO, &tmV, 0, c * CHUNK, unit, &bars[BAR_LOAD]);
     bulk_load(eta_s, p.eta + tok_base + (size_t)c * CHUNK, (uint32_t)ntok * 4u, &bars[BAR_LOAD]);
   };
-  // One of the four arrivals of the Q barrier: this warp's 16 Q rows of chunk c.
+  // This warp's 16 Q rows of chunk c, on the warp's own Q barrier.
   auto issue_load_q = [&](int c) {
-    mbar_arrive_expect_tx(&bars[BAR_LOADQ], 2048u);
+    q_last = c;
+    mbar_arrive_expect_tx(&bars[BAR_LOADQ + warp], 2048u);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int t0 = MB * (mb0 + i) + 8 * hh;
-      tma_load_3d(sm + OFF_A + 1024u * kq_group(t0, 1), &tmQ, 0, c * CHUNK + t0, unit, &bars[BAR_LOADQ]);
+      tma_load_3d(sm + OFF_A + 1024u * kq_group(t0, 1), &tmQ, 0, c * CHUNK + t0, unit,
+                  &bars[BAR_LOADQ + warp]);
     }
   };
 
@@ -305,7 +320,8 @@ __global__ void __launch_bounds__(THREADS, 4)
     const int ntok = chunk_tokens(c);
     const uint32_t par = (uint32_t)c & 1u;
     wait_or_abort(&bars[BAR_LOAD], par, abort);
-    wait_or_abort(&bars[BAR_LOADQ], par, abort);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) wait_or_abort(&bars[BAR_LOADQ + w], par, abort);
     // Products are issued by one elected lane of a converged warp (the whole warp
     // computes the operand descriptors).
     if (warp == 0) {
@@ -382,6 +398,7 @@ __global__ void __launch_bounds__(THREADS, 4)
     tc_fence_after_sync();
   };
 
+  if (p.inject_timeout) wait_or_abort(&bars[BAR_NEVER], 0, abort, INJECTED_WAIT_LIMIT);
   if (nchunks > 0) chunk_head(0);
 
   for (int c = 0; c < nchunks; ++c) {
@@ -558,6 +575,17 @@ __global__ void __launch_bounds__(THREADS, 4)
     tc_fence_after_sync();
     if (*abort) break;
     if (c + 1 < nchunks) chunk_head(c + 1);
+  }
+
+  // An aborted CTA (a wait ran past its bound) waits, again with a bound, for
+  // its own loads and products still in flight before it frees TMEM and exits.
+  __syncthreads();
+  if (*abort) {
+    if (tid == 0 && kv_last >= 0) mbar_wait(&bars[BAR_LOAD], (uint32_t)kv_last & 1u, WAIT_LIMIT);
+    if (lane == 0 && q_last >= 0) mbar_wait(&bars[BAR_LOADQ + warp], (uint32_t)q_last & 1u, WAIT_LIMIT);
+    if (warp < 2) umma_commit(&bars[BAR_DRAIN]);  // every thread that may have issued products
+    mbar_wait(&bars[BAR_DRAIN], 0, WAIT_LIMIT);
+    tc_fence_after_sync();
   }
 
   // Final state.

@@ -23,6 +23,7 @@ namespace {
 
 std::atomic<int> g_path{TTT_PATH_AUTO};
 std::atomic<long long> g_launches{0};
+std::atomic<int> g_inject_timeout{0};
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -213,6 +214,7 @@ int launch_linear_tc(const Call &c) {
   p.T = c.T;
   p.Z = c.Z;
   p.W_out = c.W_out;
+  p.inject_timeout = g_inject_timeout.load();
   auto kernel = tc::linear_tc_kernel<LN>;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)tc::SMEM_BYTES) != cudaSuccess ||
@@ -294,5 +296,7 @@ int ttt_set_path(int path) {
 }
 
 long long ttt_launch_count(void) { return g_launches.load(); }
+
+int ttt_debug_inject_timeout(int on) { return g_inject_timeout.exchange(on ? 1 : 0); }
 
 }  // extern "C"

@@ -126,3 +126,9 @@ def last_device_status(stream=None) -> int:
 
 def launch_count() -> int:
     return int(_lib.load().ttt_launch_count())
+
+
+def debug_inject_timeout(on: bool) -> bool:
+    """Test hook: while on, tensor-core launches run their bounded-wait expiry path
+    (see ``ttt_debug_inject_timeout`` in include/ttt.h).  Returns the previous setting."""
+    return bool(_lib.load().ttt_debug_inject_timeout(1 if on else 0))

@@ -145,3 +145,25 @@ def test_tensor_core_matches_cuda_core_path(name):
     for k in a:
         rel = np.linalg.norm(a[k] - b[k]) / np.linalg.norm(b[k])
         assert rel < 2e-4, (k, rel)
+
+
+@pytest.mark.parametrize("variant", ["linear", "linear_ln"])
+def test_bounded_wait_expiry_is_reported_and_recoverable(variant):
+    """The timeout path without a fault: every CTA waits on a barrier that nothing
+    arrives at, the bounded wait expires, the status word reports it, and the
+    context stays usable (the next call is exact again)."""
+    base = {"linear": "linear_bf16_B16H12T2048", "linear_ln": "linear_ln_B16H32T8192"}[variant]
+    cfg = I.CONFIGS[base].replace(B=2, H=3, T=320)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    ttt.set_path(ttt.TTT_PATH_TC)
+    assert ttt.last_device_status() == 0
+    ttt.debug_inject_timeout(True)
+    try:
+        run_gpu(cfg, dev)
+        assert ttt.last_device_status() == ttt.TTT_ERR_TIMEOUT
+        assert ttt.last_device_status() == 0, "reading the status word clears it"
+    finally:
+        ttt.debug_inject_timeout(False)
+    worst = compare(cfg, run_gpu(cfg, dev), all_units(cfg))
+    assert ttt.last_device_status() == 0
+    assert max(worst.values()) <= TOL[cfg.dtype], worst
