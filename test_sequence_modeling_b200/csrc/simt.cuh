@@ -212,38 +212,48 @@ __global__ void __launch_bounds__(THREADS) linear_kernel(const Params p) {
   for (int x = tid; x < D * D; x += THREADS) Wo[x] = W[x];
 }
 
-inline size_t mlp_smem_bytes(int b) {
-  return sizeof(float) * ((size_t)D * HID + (size_t)HID * W2_LD + 3 * (size_t)b * D +
-                          4 * (size_t)b * HID + 2 * (size_t)b * D + 2 * (size_t)b * b + b);
-}
+// TTT-MLP: b <= 16 rows per mini-batch, padded to MBR = 16 (padded rows are
+// zero and carry eta = 0, so they touch neither the state nor any output).
+// Row tiles that are contracted over their columns are kept transposed,
+// [column][16 rows] (`t` suffix), so that one 16-byte shared load serves four
+// rows and every product runs as f32x2 FMAs over row pairs; hidden-width tiles
+// get a padded stride (20 floats) so that a thread's 16-row column is written
+// without bank conflicts.
+constexpr int MBR = 16;
+constexpr int HT_LD = 20;
+
+struct MlpSmem {
+  float W1[D * HID];          // [D][HID] state
+  float W2[HID * W2_LD];      // [HID][W2_LD] state
+  float Qt[D * MBR], Kt[D * MBR];
+  float V[MBR * D];           // [16][D]
+  float X2t[HID * HT_LD];     // GELU(K W1), [HID][16]
+  float Z2t[HID * HT_LD];     // GELU(Z1), [HID][16]
+  float G3[MBR * D];          // X2 W2, then dl/d(X2 W2), [16][D]
+  float G3t[D * MBR];         // eta-free copy of G3 transposed
+  float part[4 * MBR * D];    // partial sums over hidden quarters, [4][16][D]
+  float A[MBR * MBR], A2[MBR * MBR];
+  float eta[MBR];
+};
+
+inline size_t mlp_smem_bytes(int) { return sizeof(MlpSmem) + 16; }
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
 template <typename InT>
 __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
-  extern __shared__ __align__(16) float sm[];
+  extern __shared__ __align__(16) float smem_f[];
+  MlpSmem &S = *reinterpret_cast<MlpSmem *>(smem_f);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const long unit = blockIdx.x;
   const int head = (int)(unit % p.H);
   const int b = p.b;  // <= 16
-  float *W1 = sm;                 // [D][HID]
-  float *W2 = W1 + D * HID;       // [HID][W2_LD]
-  float *Qs = W2 + HID * W2_LD;   // [b][D]
-  float *Ks = Qs + b * D;
-  float *Vs = Ks + b * D;
-  float *X1 = Vs + b * D;         // [b][HID]  K W1
-  float *X2 = X1 + b * HID;       // [b][HID]  GELU(X1)
-  float *G2 = X2 + b * HID;       // [b][HID]  dl/dX1
-  float *ZQ = G2 + b * HID;       // [b][HID]  Q W1 -> Z1 -> GELU(Z1)
-  float *G3 = ZQ + b * HID;       // [b][D]    X2 W2 -> dl/d(X2 W2)
-  float *Z3 = G3 + b * D;         // [b][D]    pre-LN output
-  float *A = Z3 + b * D;          // [b][b]    tril(Q K^T) diag(eta)
-  float *A2 = A + b * b;          // [b][b]    tril(Z2 X2^T) diag(eta)
-  float *es = A2 + b * b;         // [b]
 
   {
     const float *w1 = p.W0 + (long)head * D * HID;
     const float *w2 = p.W2_0 + (long)head * HID * D;
-    for (int x = tid; x < D * HID; x += THREADS) W1[x] = w1[x];
-    for (int x = tid; x < HID * D; x += THREADS) W2[(x / D) * W2_LD + x % D] = w2[x];
+    for (int x = tid; x < D * HID; x += THREADS) S.W1[x] = w1[x];
+    for (int x = tid; x < HID * D; x += THREADS) S.W2[(x / D) * W2_LD + x % D] = w2[x];
   }
   const float gam0 = p.gamma[head * D + lane], gam1 = p.gamma[head * D + lane + 32];
   const float bet0 = p.beta[head * D + lane], bet1 = p.beta[head * D + lane + 32];
@@ -254,151 +264,248 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
   float *Zg = p.Z + tok0 * D;
   const int nmb = p.T / b;
   const int i = tid;                           // hidden unit owned in [.][HID] passes
-  const int j = tid & (D - 1), rg = tid >> 6;  // column / row group in [.][D] passes
+  const int j = tid & (D - 1), rg = tid >> 6;  // column / hidden quarter in [.][D] passes
+
+  // Reads the 16 rows of column c of a transposed tile as 8 row pairs.
+  auto col16 = [&](const float *t, float2 (&v)[8]) {
+    const float4 *q = reinterpret_cast<const float4 *>(t);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 x = q[k];
+      v[2 * k] = make_float2(x.x, x.y);
+      v[2 * k + 1] = make_float2(x.z, x.w);
+    }
+  };
+  auto store16 = [&](float *t, const float2 (&v)[8]) {
+    float4 *q = reinterpret_cast<float4 *>(t);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) q[k] = make_float4(v[2 * k].x, v[2 * k].y, v[2 * k + 1].x, v[2 * k + 1].y);
+  };
 
   for (int n = 0; n < nmb; ++n) {
     __syncthreads();
     const long off = (long)n * b * D;
-    for (int x = tid; x < b * D; x += THREADS) {
-      Qs[x] = load_in(Qg, off + x);
-      Ks[x] = load_in(Kg, off + x);
-      Vs[x] = load_in(Vg, off + x);
+    for (int x = tid; x < MBR * D; x += THREADS) {
+      const int r = x / D, c = x % D;
+      const bool in = r < b;
+      S.Qt[c * MBR + r] = in ? load_in(Qg, off + r * D + c) : 0.f;
+      S.Kt[c * MBR + r] = in ? load_in(Kg, off + r * D + c) : 0.f;
+      S.V[x] = in ? load_in(Vg, off + x) : 0.f;
     }
-    if (tid < b) es[tid] = p.eta[tok0 + (long)n * b + tid];
+    if (tid < MBR) S.eta[tid] = tid < b ? p.eta[tok0 + (long)n * b + tid] : 0.f;
     __syncthreads();
 
-    // X1 = K W1, ZQ = Q W1 (column i of both).
+    // X1 = K W1 and Z1 = Q W1, column i (rows in pairs).
+    float2 x1[8], zq[8];
     {
-      float ak[16], aq[16];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) ak[r] = aq[r] = 0.f;
+      for (int k = 0; k < 8; ++k) x1[k] = zq[k] = make_float2(0.f, 0.f);
+#pragma unroll 4
       for (int pp = 0; pp < D; ++pp) {
-        const float w = W1[pp * HID + i];
+        const float w = S.W1[pp * HID + i];
+        const float2 ww = make_float2(w, w);
+        float2 kv[8], qv[8];
+        col16(&S.Kt[pp * MBR], kv);
+        col16(&S.Qt[pp * MBR], qv);
 #pragma unroll
-        for (int r = 0; r < 16; ++r)
-          if (r < b) {
-            ak[r] = fmaf(Ks[r * D + pp], w, ak[r]);
-            aq[r] = fmaf(Qs[r * D + pp], w, aq[r]);
-          }
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r)
-        if (r < b) {
-          X1[r * HID + i] = ak[r];
-          X2[r * HID + i] = gelu(ak[r]);
-          ZQ[r * HID + i] = aq[r];
+        for (int k = 0; k < 8; ++k) {
+          x1[k] = ffma2(kv[k], ww, x1[k]);
+          zq[k] = ffma2(qv[k], ww, zq[k]);
         }
-    }
-    for (int pr = warp; pr < b * b; pr += THREADS / 32) {
-      const int t = pr / b, s = pr % b;
-      float acc = 0.f;
-      if (s <= t) {
-        acc = fmaf(Qs[t * D + lane + 32], Ks[s * D + lane + 32], Qs[t * D + lane] * Ks[s * D + lane]);
-        acc = warp_sum(acc) * es[s];
       }
-      if (lane == 0) A[pr] = acc;
+      float2 x2[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x2[k] = make_float2(gelu(x1[k].x), gelu(x1[k].y));
+      store16(&S.X2t[i * HT_LD], x2);
+    }
+    // A = tril(Q K^T) diag(eta), one entry per thread.
+    {
+      const int t = tid >> 4, s0 = tid & 15;
+      float acc = 0.f;
+      if (s0 <= t) {
+#pragma unroll 8
+        for (int pp = 0; pp < D; ++pp) acc = fmaf(S.Qt[pp * MBR + t], S.Kt[pp * MBR + s0], acc);
+        acc *= S.eta[s0];
+      }
+      S.A[tid] = acc;
     }
     __syncthreads();
 
-    // X3 = X2 W2 into G3.
-    for (int t = rg; t < b; t += 4) {
-      float acc = 0.f;
-      for (int ii = 0; ii < HID; ++ii) acc = fmaf(X2[t * HID + ii], W2[ii * W2_LD + j], acc);
-      G3[t * D + j] = acc;
-    }
-    __syncthreads();
-    // G3 = dl / d X3 through LN and the residual.
-    for (int r = warp; r < b; r += THREADS / 32) {
-      float dy0, dy1;
-      ln_residual_grad(G3[r * D + lane], G3[r * D + lane + 32], Ks[r * D + lane],
-                       Ks[r * D + lane + 32], Vs[r * D + lane], Vs[r * D + lane + 32], gam0, gam1,
-                       bet0, bet1, p.eps, dy0, dy1);
-      G3[r * D + lane] = dy0;
-      G3[r * D + lane + 32] = dy1;
-    }
-    __syncthreads();
-    // G2 = (G3 W2^T) * GELU'(X1); then Z1 = Q W1 - A G2 and Z2 = GELU(Z1).
+    // X3 = X2 W2: partial sums over hidden quarter rg, for column j.
     {
-      float acc[16];
+      float2 acc[8];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) acc[r] = 0.f;
+      for (int k = 0; k < 8; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll 4
+      for (int ii = HID / 4 * rg; ii < HID / 4 * (rg + 1); ++ii) {
+        const float w = S.W2[ii * W2_LD + j];
+        const float2 ww = make_float2(w, w);
+        float2 xv[8];
+        col16(&S.X2t[ii * HT_LD], xv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = ffma2(xv[k], ww, acc[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        S.part[(rg * MBR + 2 * k) * D + j] = acc[k].x;
+        S.part[(rg * MBR + 2 * k + 1) * D + j] = acc[k].y;
+      }
+    }
+    __syncthreads();
+    for (int x = tid; x < MBR * D; x += THREADS)
+      S.G3[x] = (S.part[x] + S.part[MBR * D + x]) + (S.part[2 * MBR * D + x] + S.part[3 * MBR * D + x]);
+    __syncthreads();
+    // G3 = dl / d X3 through LN and the residual (a warp per row).
+    for (int r = warp; r < MBR; r += THREADS / 32) {
+      float dy0, dy1;
+      ln_residual_grad(S.G3[r * D + lane], S.G3[r * D + lane + 32], S.Kt[lane * MBR + r],
+                       S.Kt[(lane + 32) * MBR + r], S.V[r * D + lane], S.V[r * D + lane + 32], gam0,
+                       gam1, bet0, bet1, p.eps, dy0, dy1);
+      S.G3[r * D + lane] = dy0;
+      S.G3[r * D + lane + 32] = dy1;
+      S.G3t[lane * MBR + r] = dy0;
+      S.G3t[(lane + 32) * MBR + r] = dy1;
+    }
+    __syncthreads();
+
+    // G2 = (G3 W2^T) * GELU'(X1) for column i; then Z1 = Q W1 - A G2 and Z2 = GELU(Z1).
+    float2 g2[8];
+    {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) g2[k] = make_float2(0.f, 0.f);
+#pragma unroll 4
       for (int jj = 0; jj < D; ++jj) {
-        const float w = W2[i * W2_LD + jj];
+        const float w = S.W2[i * W2_LD + jj];
+        const float2 ww = make_float2(w, w);
+        float2 gv[8];
+        col16(&S.G3t[jj * MBR], gv);
 #pragma unroll
-        for (int r = 0; r < 16; ++r)
-          if (r < b) acc[r] = fmaf(G3[r * D + jj], w, acc[r]);
+        for (int k = 0; k < 8; ++k) g2[k] = ffma2(gv[k], ww, g2[k]);
       }
 #pragma unroll
-      for (int r = 0; r < 16; ++r)
-        if (r < b) acc[r] *= gelu_deriv(X1[r * HID + i]);
+      for (int k = 0; k < 8; ++k)
+        g2[k] = make_float2(g2[k].x * gelu_deriv(x1[k].x), g2[k].y * gelu_deriv(x1[k].y));
+      float g2s[MBR];
 #pragma unroll
-      for (int r = 0; r < 16; ++r)
-        if (r < b) G2[r * HID + i] = acc[r];
+      for (int k = 0; k < 8; ++k) {
+        g2s[2 * k] = g2[k].x;
+        g2s[2 * k + 1] = g2[k].y;
+      }
+      float2 z2[8];
 #pragma unroll
-      for (int t = 0; t < 16; ++t)
-        if (t < b) {
-          float z = ZQ[t * HID + i];
-          for (int s = 0; s <= t; ++s) z = fmaf(-A[t * b + s], acc[s], z);
-          ZQ[t * HID + i] = gelu(z);
+      for (int k = 0; k < 8; ++k) {
+        float za = zq[k].x, zb = zq[k].y;
+        const int t0 = 2 * k, t1 = 2 * k + 1;
+#pragma unroll
+        for (int s0 = 0; s0 < MBR; ++s0) {
+          if (s0 <= t0) za = fmaf(-S.A[t0 * MBR + s0], g2s[s0], za);
+          if (s0 <= t1) zb = fmaf(-S.A[t1 * MBR + s0], g2s[s0], zb);
         }
-    }
-    __syncthreads();
-    // A2 = tril(Z2 X2^T) diag(eta).
-    for (int pr = warp; pr < b * b; pr += THREADS / 32) {
-      const int t = pr / b, s = pr % b;
-      float acc = 0.f;
-      if (s <= t) {
-        for (int ii = lane; ii < HID; ii += 32) acc = fmaf(ZQ[t * HID + ii], X2[s * HID + ii], acc);
-        acc = warp_sum(acc) * es[s];
+        z2[k] = make_float2(gelu(za), gelu(zb));
       }
-      if (lane == 0) A2[pr] = acc;
+      store16(&S.Z2t[i * HT_LD], z2);
     }
     __syncthreads();
-    // Z3 = Z2 W2 - A2 G3.
-    for (int t = rg; t < b; t += 4) {
-      float acc = 0.f;
-      for (int ii = 0; ii < HID; ++ii) acc = fmaf(ZQ[t * HID + ii], W2[ii * W2_LD + j], acc);
-      for (int s = 0; s <= t; ++s) acc = fmaf(-A2[t * b + s], G3[s * D + j], acc);
-      Z3[t * D + j] = acc;
+
+    // A2 = tril(Z2 X2^T) diag(eta): entry (t, 4 s4 .. 4 s4 + 3), hidden quarter q.
+    {
+      const int q = tid >> 6, t = (tid >> 2) & 15, s4 = tid & 3;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (4 * s4 <= t) {
+#pragma unroll 4
+        for (int ii = HID / 4 * q; ii < HID / 4 * (q + 1); ++ii) {
+          const float z = S.Z2t[ii * HT_LD + t];
+          const float4 x = *reinterpret_cast<const float4 *>(&S.X2t[ii * HT_LD + 4 * s4]);
+          acc.x = fmaf(z, x.x, acc.x);
+          acc.y = fmaf(z, x.y, acc.y);
+          acc.z = fmaf(z, x.z, acc.z);
+          acc.w = fmaf(z, x.w, acc.w);
+        }
+      }
+      *reinterpret_cast<float4 *>(&S.part[(q * MBR + t) * MBR + 4 * s4]) = acc;
     }
     __syncthreads();
-    // Output Z = Q + LN(Z3); state updates (W1, W2 are no longer read this mini-batch).
+    {
+      const int t = tid >> 4, s0 = tid & 15;
+      const float a = (S.part[tid] + S.part[MBR * MBR + tid]) +
+                      (S.part[2 * MBR * MBR + tid] + S.part[3 * MBR * MBR + tid]);
+      S.A2[tid] = s0 <= t ? a * S.eta[s0] : 0.f;
+    }
+    __syncthreads();
+
+    // Z3 = Z2 W2 - A2 G3: partial sums of Z2 W2 over hidden quarter rg.
+    {
+      float2 acc[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] = make_float2(0.f, 0.f);
+#pragma unroll 4
+      for (int ii = HID / 4 * rg; ii < HID / 4 * (rg + 1); ++ii) {
+        const float w = S.W2[ii * W2_LD + j];
+        const float2 ww = make_float2(w, w);
+        float2 zv[8];
+        col16(&S.Z2t[ii * HT_LD], zv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = ffma2(zv[k], ww, acc[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        S.part[(rg * MBR + 2 * k) * D + j] = acc[k].x;
+        S.part[(rg * MBR + 2 * k + 1) * D + j] = acc[k].y;
+      }
+    }
+    __syncthreads();
+    // Output Z = Q + LN(Z3) (a warp per row); Z3 assembled from the partials.
     for (int r = warp; r < b; r += THREADS / 32) {
+      float y[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int x = r * D + lane + 32 * h;
+        float acc = (S.part[x] + S.part[MBR * D + x]) + (S.part[2 * MBR * D + x] + S.part[3 * MBR * D + x]);
+        for (int s0 = 0; s0 <= r; ++s0) acc = fmaf(-S.A2[r * MBR + s0], S.G3[s0 * D + lane + 32 * h], acc);
+        y[h] = acc;
+      }
       float z0, z1;
-      ln_residual_fwd(Z3[r * D + lane], Z3[r * D + lane + 32], Qs[r * D + lane],
-                      Qs[r * D + lane + 32], gam0, gam1, bet0, bet1, p.eps, z0, z1);
+      ln_residual_fwd(y[0], y[1], S.Qt[lane * MBR + r], S.Qt[(lane + 32) * MBR + r], gam0, gam1, bet0,
+                      bet1, p.eps, z0, z1);
       Zg[off + r * D + lane] = z0;
       Zg[off + r * D + lane + 32] = z1;
     }
+    // State updates (no product of this mini-batch reads W1 or W2 any more).
     {
       // W1[pp][i] -= sum_t K[t][pp] eta_t G2[t][i]
-      float g[16];
+      float2 g[8];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) g[t] = t < b ? es[t] * G2[t * HID + i] : 0.f;
+      for (int k = 0; k < 8; ++k)
+        g[k] = make_float2(S.eta[2 * k] * g2[k].x, S.eta[2 * k + 1] * g2[k].y);
+#pragma unroll 4
       for (int pp = 0; pp < D; ++pp) {
-        float acc = 0.f;
+        float2 kv[8];
+        col16(&S.Kt[pp * MBR], kv);
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
-          if (t < b) acc = fmaf(Ks[t * D + pp], g[t], acc);
-        W1[pp * HID + i] -= acc;
+        for (int k = 0; k < 8; ++k) acc = ffma2(kv[k], g[k], acc);
+        S.W1[pp * HID + i] -= acc.x + acc.y;
       }
-      // W2[ii][j] -= sum_t X2[t][ii] eta_t G3[t][j]
+      // W2[ii][j] -= sum_t X2[t][ii] eta_t G3[t][j], hidden quarter rg
 #pragma unroll
-      for (int t = 0; t < 16; ++t) g[t] = t < b ? es[t] * G3[t * D + j] : 0.f;
-      for (int ii = rg; ii < HID; ii += 4) {
-        float acc = 0.f;
+      for (int k = 0; k < 8; ++k)
+        g[k] = make_float2(S.eta[2 * k] * S.G3[(2 * k) * D + j], S.eta[2 * k + 1] * S.G3[(2 * k + 1) * D + j]);
+#pragma unroll 4
+      for (int ii = HID / 4 * rg; ii < HID / 4 * (rg + 1); ++ii) {
+        float2 xv[8];
+        col16(&S.X2t[ii * HT_LD], xv);
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
-          if (t < b) acc = fmaf(X2[t * HID + ii], g[t], acc);
-        W2[ii * W2_LD + j] -= acc;
+        for (int k = 0; k < 8; ++k) acc = ffma2(xv[k], g[k], acc);
+        S.W2[ii * W2_LD + j] -= acc.x + acc.y;
       }
     }
   }
   __syncthreads();
   float *w1o = p.W_out + unit * D * HID;
   float *w2o = p.W2_out + unit * HID * D;
-  for (int x = tid; x < D * HID; x += THREADS) w1o[x] = W1[x];
-  for (int x = tid; x < HID * D; x += THREADS) w2o[x] = W2[(x / D) * W2_LD + x % D];
+  for (int x = tid; x < D * HID; x += THREADS) w1o[x] = S.W1[x];
+  for (int x = tid; x < HID * D; x += THREADS) w2o[x] = S.W2[(x / D) * W2_LD + x % D];
 }
 
 }  // namespace simt
