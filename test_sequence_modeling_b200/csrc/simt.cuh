@@ -217,10 +217,13 @@ __global__ void __launch_bounds__(THREADS) linear_kernel(const Params p) {
 // Row tiles that are contracted over their columns are kept transposed,
 // [column][16 rows] (`t` suffix), so that one 16-byte shared load serves four
 // rows and every product runs as f32x2 FMAs over row pairs; hidden-width tiles
-// get a padded stride (20 floats) so that a thread's 16-row column is written
-// without bank conflicts.
+// get a padded stride (20 floats) so that a thread's rows of one column are
+// written without bank conflicts.  512 threads: in the [.][HID] passes thread
+// (i, rh) owns hidden unit i and rows 8 rh .. 8 rh + 7; in the [.][D] passes
+// thread (j, e) owns column j and hidden eighth e.
 constexpr int MBR = 16;
 constexpr int HT_LD = 20;
+constexpr int MLP_THREADS = 512;
 
 struct MlpSmem {
   float W1[D * HID];          // [D][HID] state
@@ -230,8 +233,11 @@ struct MlpSmem {
   float X2t[HID * HT_LD];     // GELU(K W1), [HID][16]
   float Z2t[HID * HT_LD];     // GELU(Z1), [HID][16]
   float G3[MBR * D];          // X2 W2, then dl/d(X2 W2), [16][D]
-  float G3t[D * MBR];         // eta-free copy of G3 transposed
-  float part[4 * MBR * D];    // partial sums over hidden quarters, [4][16][D]
+  float G3t[D * MBR];         // G3 transposed
+  union {
+    float part[4 * MBR * D];  // partial sums over hidden parts
+    float G2t[HID * HT_LD];   // dl/dX1, [HID][16] (between the X3 and A2 passes)
+  };
   float A[MBR * MBR], A2[MBR * MBR];
   float eta[MBR];
 };
@@ -240,8 +246,27 @@ inline size_t mlp_smem_bytes(int) { return sizeof(MlpSmem) + 16; }
 
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 
+// Rows 8 h .. 8 h + 7 (h = 0, 1) or all 16 rows of column c of a transposed
+// tile, as row pairs.
+template <int N>
+__device__ __forceinline__ void load_rows(const float *t, float2 (&v)[N]) {
+  const float4 *q = reinterpret_cast<const float4 *>(t);
+#pragma unroll
+  for (int k = 0; k < N / 2; ++k) {
+    const float4 x = q[k];
+    v[2 * k] = make_float2(x.x, x.y);
+    v[2 * k + 1] = make_float2(x.z, x.w);
+  }
+}
+template <int N>
+__device__ __forceinline__ void store_rows(float *t, const float2 (&v)[N]) {
+  float4 *q = reinterpret_cast<float4 *>(t);
+#pragma unroll
+  for (int k = 0; k < N / 2; ++k) q[k] = make_float4(v[2 * k].x, v[2 * k].y, v[2 * k + 1].x, v[2 * k + 1].y);
+}
+
 template <typename InT>
-__global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
+__global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
   extern __shared__ __align__(16) float smem_f[];
   MlpSmem &S = *reinterpret_cast<MlpSmem *>(smem_f);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -252,8 +277,8 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
   {
     const float *w1 = p.W0 + (long)head * D * HID;
     const float *w2 = p.W2_0 + (long)head * HID * D;
-    for (int x = tid; x < D * HID; x += THREADS) S.W1[x] = w1[x];
-    for (int x = tid; x < HID * D; x += THREADS) S.W2[(x / D) * W2_LD + x % D] = w2[x];
+    for (int x = tid; x < D * HID; x += MLP_THREADS) S.W1[x] = w1[x];
+    for (int x = tid; x < HID * D; x += MLP_THREADS) S.W2[(x / D) * W2_LD + x % D] = w2[x];
   }
   const float gam0 = p.gamma[head * D + lane], gam1 = p.gamma[head * D + lane + 32];
   const float bet0 = p.beta[head * D + lane], bet1 = p.beta[head * D + lane + 32];
@@ -263,29 +288,15 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
   const InT *Vg = (const InT *)p.V + tok0 * D;
   float *Zg = p.Z + tok0 * D;
   const int nmb = p.T / b;
-  const int i = tid;                           // hidden unit owned in [.][HID] passes
-  const int j = tid & (D - 1), rg = tid >> 6;  // column / hidden quarter in [.][D] passes
-
-  // Reads the 16 rows of column c of a transposed tile as 8 row pairs.
-  auto col16 = [&](const float *t, float2 (&v)[8]) {
-    const float4 *q = reinterpret_cast<const float4 *>(t);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float4 x = q[k];
-      v[2 * k] = make_float2(x.x, x.y);
-      v[2 * k + 1] = make_float2(x.z, x.w);
-    }
-  };
-  auto store16 = [&](float *t, const float2 (&v)[8]) {
-    float4 *q = reinterpret_cast<float4 *>(t);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) q[k] = make_float4(v[2 * k].x, v[2 * k].y, v[2 * k + 1].x, v[2 * k + 1].y);
-  };
+  const int i = tid & (HID - 1), rh = tid >> 8;  // hidden unit, row half
+  const int r0 = 8 * rh;
+  const int j = tid & (D - 1), e = tid >> 6;     // column, hidden eighth
+  const int ilo = HID / 8 * e, ihi = ilo + HID / 8;
 
   for (int n = 0; n < nmb; ++n) {
     __syncthreads();
     const long off = (long)n * b * D;
-    for (int x = tid; x < MBR * D; x += THREADS) {
+    for (int x = tid; x < MBR * D; x += MLP_THREADS) {
       const int r = x / D, c = x % D;
       const bool in = r < b;
       S.Qt[c * MBR + r] = in ? load_in(Qg, off + r * D + c) : 0.f;
@@ -295,31 +306,31 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
     if (tid < MBR) S.eta[tid] = tid < b ? p.eta[tok0 + (long)n * b + tid] : 0.f;
     __syncthreads();
 
-    // X1 = K W1 and Z1 = Q W1, column i (rows in pairs).
-    float2 x1[8], zq[8];
+    // X1 = K W1 and Z1 = Q W1: column i, this thread's 8 rows.
+    float2 x1[4], zq[4];
     {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) x1[k] = zq[k] = make_float2(0.f, 0.f);
-#pragma unroll 4
+      for (int k = 0; k < 4; ++k) x1[k] = zq[k] = make_float2(0.f, 0.f);
+#pragma unroll 8
       for (int pp = 0; pp < D; ++pp) {
         const float w = S.W1[pp * HID + i];
         const float2 ww = make_float2(w, w);
-        float2 kv[8], qv[8];
-        col16(&S.Kt[pp * MBR], kv);
-        col16(&S.Qt[pp * MBR], qv);
+        float2 kv[4], qv[4];
+        load_rows(&S.Kt[pp * MBR + r0], kv);
+        load_rows(&S.Qt[pp * MBR + r0], qv);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < 4; ++k) {
           x1[k] = ffma2(kv[k], ww, x1[k]);
           zq[k] = ffma2(qv[k], ww, zq[k]);
         }
       }
-      float2 x2[8];
+      float2 x2[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) x2[k] = make_float2(gelu(x1[k].x), gelu(x1[k].y));
-      store16(&S.X2t[i * HT_LD], x2);
+      for (int k = 0; k < 4; ++k) x2[k] = make_float2(gelu(x1[k].x), gelu(x1[k].y));
+      store_rows(&S.X2t[i * HT_LD + r0], x2);
     }
-    // A = tril(Q K^T) diag(eta), one entry per thread.
-    {
+    // A = tril(Q K^T) diag(eta), one entry per thread of the first 256.
+    if (tid < MBR * MBR) {
       const int t = tid >> 4, s0 = tid & 15;
       float acc = 0.f;
       if (s0 <= t) {
@@ -331,32 +342,47 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
     }
     __syncthreads();
 
-    // X3 = X2 W2: partial sums over hidden quarter rg, for column j.
-    {
+    // X3 = X2 W2: partial sums over hidden eighth e for column j, all 16 rows;
+    // eighths 2q and 2q+1 meet in part[q].
+    auto hidden_product = [&](const float *Xt) {
       float2 acc[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) acc[k] = make_float2(0.f, 0.f);
 #pragma unroll 4
-      for (int ii = HID / 4 * rg; ii < HID / 4 * (rg + 1); ++ii) {
+      for (int ii = ilo; ii < ihi; ++ii) {
         const float w = S.W2[ii * W2_LD + j];
         const float2 ww = make_float2(w, w);
         float2 xv[8];
-        col16(&S.X2t[ii * HT_LD], xv);
+        load_rows(&Xt[ii * HT_LD], xv);
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc[k] = ffma2(xv[k], ww, acc[k]);
       }
+      // Two passes through part[]: odd eighths add onto what even eighths wrote.
+      float *dst = &S.part[(e >> 1) * MBR * D + j];
+      if ((e & 1) == 0) {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        S.part[(rg * MBR + 2 * k) * D + j] = acc[k].x;
-        S.part[(rg * MBR + 2 * k + 1) * D + j] = acc[k].y;
+        for (int k = 0; k < 8; ++k) {
+          dst[(2 * k) * D] = acc[k].x;
+          dst[(2 * k + 1) * D] = acc[k].y;
+        }
       }
-    }
-    __syncthreads();
-    for (int x = tid; x < MBR * D; x += THREADS)
+      __syncthreads();
+      if (e & 1) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          dst[(2 * k) * D] += acc[k].x;
+          dst[(2 * k + 1) * D] += acc[k].y;
+        }
+      }
+      __syncthreads();
+    };
+    hidden_product(S.X2t);
+    for (int x = tid; x < MBR * D; x += MLP_THREADS)
       S.G3[x] = (S.part[x] + S.part[MBR * D + x]) + (S.part[2 * MBR * D + x] + S.part[3 * MBR * D + x]);
     __syncthreads();
     // G3 = dl / d X3 through LN and the residual (a warp per row).
-    for (int r = warp; r < MBR; r += THREADS / 32) {
+    {
+      const int r = warp;
       float dy0, dy1;
       ln_residual_grad(S.G3[r * D + lane], S.G3[r * D + lane + 32], S.Kt[lane * MBR + r],
                        S.Kt[(lane + 32) * MBR + r], S.V[r * D + lane], S.V[r * D + lane + 32], gam0,
@@ -368,34 +394,43 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
     }
     __syncthreads();
 
-    // G2 = (G3 W2^T) * GELU'(X1) for column i; then Z1 = Q W1 - A G2 and Z2 = GELU(Z1).
-    float2 g2[8];
+    // G2 = (G3 W2^T) * GELU'(X1): column i, this thread's 8 rows.
     {
+      float2 g2[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) g2[k] = make_float2(0.f, 0.f);
-#pragma unroll 4
+      for (int k = 0; k < 4; ++k) g2[k] = make_float2(0.f, 0.f);
+#pragma unroll 8
       for (int jj = 0; jj < D; ++jj) {
         const float w = S.W2[i * W2_LD + jj];
         const float2 ww = make_float2(w, w);
-        float2 gv[8];
-        col16(&S.G3t[jj * MBR], gv);
+        float2 gv[4];
+        load_rows(&S.G3t[jj * MBR + r0], gv);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) g2[k] = ffma2(gv[k], ww, g2[k]);
+        for (int k = 0; k < 4; ++k) g2[k] = ffma2(gv[k], ww, g2[k]);
       }
 #pragma unroll
-      for (int k = 0; k < 8; ++k)
+      for (int k = 0; k < 4; ++k)
         g2[k] = make_float2(g2[k].x * gelu_deriv(x1[k].x), g2[k].y * gelu_deriv(x1[k].y));
+      store_rows(&S.G2t[i * HT_LD + r0], g2);
+    }
+    __syncthreads();
+    // Z1 = Q W1 - A G2 and Z2 = GELU(Z1): column i, this thread's 8 rows.
+    {
       float g2s[MBR];
+      {
+        float2 gv[8];
+        load_rows(&S.G2t[i * HT_LD], gv);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        g2s[2 * k] = g2[k].x;
-        g2s[2 * k + 1] = g2[k].y;
+        for (int k = 0; k < 8; ++k) {
+          g2s[2 * k] = gv[k].x;
+          g2s[2 * k + 1] = gv[k].y;
+        }
       }
-      float2 z2[8];
+      float2 z2[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
+      for (int k = 0; k < 4; ++k) {
         float za = zq[k].x, zb = zq[k].y;
-        const int t0 = 2 * k, t1 = 2 * k + 1;
+        const int t0 = r0 + 2 * k, t1 = t0 + 1;
 #pragma unroll
         for (int s0 = 0; s0 < MBR; ++s0) {
           if (s0 <= t0) za = fmaf(-S.A[t0 * MBR + s0], g2s[s0], za);
@@ -403,17 +438,36 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
         }
         z2[k] = make_float2(gelu(za), gelu(zb));
       }
-      store16(&S.Z2t[i * HT_LD], z2);
+      store_rows(&S.Z2t[i * HT_LD + r0], z2);
+    }
+    {
+      // W1[pp][i] -= sum_t K[t][pp] eta_t G2[t][i], pp in this thread's half.
+      float2 g[8];
+      {
+        float2 gv[8];
+        load_rows(&S.G2t[i * HT_LD], gv);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) g[k] = make_float2(S.eta[2 * k] * gv[k].x, S.eta[2 * k + 1] * gv[k].y);
+      }
+#pragma unroll 4
+      for (int pp = D / 2 * rh; pp < D / 2 * (rh + 1); ++pp) {
+        float2 kv[8];
+        load_rows(&S.Kt[pp * MBR], kv);
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc = ffma2(kv[k], g[k], acc);
+        S.W1[pp * HID + i] -= acc.x + acc.y;
+      }
     }
     __syncthreads();
 
-    // A2 = tril(Z2 X2^T) diag(eta): entry (t, 4 s4 .. 4 s4 + 3), hidden quarter q.
+    // A2 = tril(Z2 X2^T) diag(eta): entry (t, 4 s4 .. 4 s4 + 3), hidden eighth q.
     {
       const int q = tid >> 6, t = (tid >> 2) & 15, s4 = tid & 3;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       if (4 * s4 <= t) {
 #pragma unroll 4
-        for (int ii = HID / 4 * q; ii < HID / 4 * (q + 1); ++ii) {
+        for (int ii = HID / 8 * q; ii < HID / 8 * (q + 1); ++ii) {
           const float z = S.Z2t[ii * HT_LD + t];
           const float4 x = *reinterpret_cast<const float4 *>(&S.X2t[ii * HT_LD + 4 * s4]);
           acc.x = fmaf(z, x.x, acc.x);
@@ -425,75 +479,47 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
       *reinterpret_cast<float4 *>(&S.part[(q * MBR + t) * MBR + 4 * s4]) = acc;
     }
     __syncthreads();
-    {
+    if (tid < MBR * MBR) {
       const int t = tid >> 4, s0 = tid & 15;
-      const float a = (S.part[tid] + S.part[MBR * MBR + tid]) +
-                      (S.part[2 * MBR * MBR + tid] + S.part[3 * MBR * MBR + tid]);
+      float a = 0.f;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) a += S.part[q * MBR * MBR + tid];
       S.A2[tid] = s0 <= t ? a * S.eta[s0] : 0.f;
     }
     __syncthreads();
 
-    // Z3 = Z2 W2 - A2 G3: partial sums of Z2 W2 over hidden quarter rg.
+    // Z3 = Z2 W2 - A2 G3.
+    hidden_product(S.Z2t);
+    // Output Z = Q + LN(Z3) (a warp per row).
     {
-      float2 acc[8];
+      const int r = warp;
+      if (r < b) {
+        float y[2];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) acc[k] = make_float2(0.f, 0.f);
-#pragma unroll 4
-      for (int ii = HID / 4 * rg; ii < HID / 4 * (rg + 1); ++ii) {
-        const float w = S.W2[ii * W2_LD + j];
-        const float2 ww = make_float2(w, w);
-        float2 zv[8];
-        col16(&S.Z2t[ii * HT_LD], zv);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = ffma2(zv[k], ww, acc[k]);
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        S.part[(rg * MBR + 2 * k) * D + j] = acc[k].x;
-        S.part[(rg * MBR + 2 * k + 1) * D + j] = acc[k].y;
+        for (int h = 0; h < 2; ++h) {
+          const int x = r * D + lane + 32 * h;
+          float acc = (S.part[x] + S.part[MBR * D + x]) + (S.part[2 * MBR * D + x] + S.part[3 * MBR * D + x]);
+          for (int s0 = 0; s0 <= r; ++s0) acc = fmaf(-S.A2[r * MBR + s0], S.G3[s0 * D + lane + 32 * h], acc);
+          y[h] = acc;
+        }
+        float z0, z1;
+        ln_residual_fwd(y[0], y[1], S.Qt[lane * MBR + r], S.Qt[(lane + 32) * MBR + r], gam0, gam1, bet0,
+                        bet1, p.eps, z0, z1);
+        Zg[off + r * D + lane] = z0;
+        Zg[off + r * D + lane + 32] = z1;
       }
     }
-    __syncthreads();
-    // Output Z = Q + LN(Z3) (a warp per row); Z3 assembled from the partials.
-    for (int r = warp; r < b; r += THREADS / 32) {
-      float y[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int x = r * D + lane + 32 * h;
-        float acc = (S.part[x] + S.part[MBR * D + x]) + (S.part[2 * MBR * D + x] + S.part[3 * MBR * D + x]);
-        for (int s0 = 0; s0 <= r; ++s0) acc = fmaf(-S.A2[r * MBR + s0], S.G3[s0 * D + lane + 32 * h], acc);
-        y[h] = acc;
-      }
-      float z0, z1;
-      ln_residual_fwd(y[0], y[1], S.Qt[lane * MBR + r], S.Qt[(lane + 32) * MBR + r], gam0, gam1, bet0,
-                      bet1, p.eps, z0, z1);
-      Zg[off + r * D + lane] = z0;
-      Zg[off + r * D + lane + 32] = z1;
-    }
-    // State updates (no product of this mini-batch reads W1 or W2 any more).
+    // W2 update (no product of this mini-batch reads W2 any more).
     {
-      // W1[pp][i] -= sum_t K[t][pp] eta_t G2[t][i]
       float2 g[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        g[k] = make_float2(S.eta[2 * k] * g2[k].x, S.eta[2 * k + 1] * g2[k].y);
-#pragma unroll 4
-      for (int pp = 0; pp < D; ++pp) {
-        float2 kv[8];
-        col16(&S.Kt[pp * MBR], kv);
-        float2 acc = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc = ffma2(kv[k], g[k], acc);
-        S.W1[pp * HID + i] -= acc.x + acc.y;
-      }
-      // W2[ii][j] -= sum_t X2[t][ii] eta_t G3[t][j], hidden quarter rg
+      // W2[ii][j] -= sum_t X2[t][ii] eta_t G3[t][j], ii in hidden eighth e.
 #pragma unroll
       for (int k = 0; k < 8; ++k)
         g[k] = make_float2(S.eta[2 * k] * S.G3[(2 * k) * D + j], S.eta[2 * k + 1] * S.G3[(2 * k + 1) * D + j]);
 #pragma unroll 4
-      for (int ii = HID / 4 * rg; ii < HID / 4 * (rg + 1); ++ii) {
+      for (int ii = ilo; ii < ihi; ++ii) {
         float2 xv[8];
-        col16(&S.X2t[ii * HT_LD], xv);
+        load_rows(&S.X2t[ii * HT_LD], xv);
         float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc = ffma2(xv[k], g[k], acc);
@@ -504,8 +530,8 @@ __global__ void __launch_bounds__(THREADS) mlp_kernel(const Params p) {
   __syncthreads();
   float *w1o = p.W_out + unit * D * HID;
   float *w2o = p.W2_out + unit * HID * D;
-  for (int x = tid; x < D * HID; x += THREADS) w1o[x] = S.W1[x];
-  for (int x = tid; x < HID * D; x += THREADS) w2o[x] = S.W2[(x / D) * W2_LD + x % D];
+  for (int x = tid; x < D * HID; x += MLP_THREADS) w1o[x] = S.W1[x];
+  for (int x = tid; x < HID * D; x += MLP_THREADS) w2o[x] = S.W2[(x / D) * W2_LD + x % D];
 }
 
 }  // namespace simt

@@ -116,13 +116,13 @@ int validate(const Call &c) {
 
 template <typename KernelT>
 int launch(KernelT kernel, int grid, size_t smem, cudaStream_t stream,
-           const simt::Params &p) {
+           const simt::Params &p, int threads = simt::THREADS) {
   if (smem > 48 * 1024) {
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return TTT_ERR_CUDA;
   }
-  kernel<<<grid, simt::THREADS, smem, stream>>>(p);
+  kernel<<<grid, threads, smem, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return TTT_OK;
@@ -150,8 +150,8 @@ int run_simt(const Call &c) {
   const bool bf16 = c.qkv_dtype == TTT_BF16;
   if (c.kind == MLP_LN) {
     const size_t smem = simt::mlp_smem_bytes(c.b);
-    return bf16 ? launch(simt::mlp_kernel<__nv_bfloat16>, grid, smem, s, p)
-                : launch(simt::mlp_kernel<float>, grid, smem, s, p);
+    return bf16 ? launch(simt::mlp_kernel<__nv_bfloat16>, grid, smem, s, p, simt::MLP_THREADS)
+                : launch(simt::mlp_kernel<float>, grid, smem, s, p, simt::MLP_THREADS);
   }
   const size_t smem = simt::linear_smem_bytes(c.b);
   if (c.kind == LINEAR_LN)
