@@ -269,7 +269,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling cases)")
     ap.add_argument("--seq", type=int, default=None, help="override T (smaller profiling cases)")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the primal-form decode step (TTT-Linear + LN, B=512 H=32, bf16 q/k/v) "
+                         "instead of the forward")
     args = ap.parse_args()
+    if args.decode:
+        return run_decode(args)
     cfg = I.CONFIGS[args.workload]
     if args.batch is not None or args.seq is not None:
         cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T,
@@ -377,6 +382,76 @@ def main():
     nflops = flops_per_head_token(cfg) * cfg.head_tokens
     return finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info, launches,
                   e2e, peaks, peak_kind, nbytes, nflops, dist)
+
+
+def run_decode(args):
+    """The decode step's own line: one timed step = one mini-batch of 16 decode calls
+    (positions 0..15) over B=512 x H=32 (batch, head) units, the state in HBM."""
+    import torch
+    import test_sequence_modeling_b200 as ttt
+    from test_sequence_modeling_b200 import _lib
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=512, T=16, name="decode_linear_ln_B512H32")
+    data = I.make_inputs(cfg)
+    B, H, T, d = cfg.B, cfg.H, cfg.T, cfg.d
+    qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
+    tok = [{k: qkv[k][:, :, t].contiguous() for k in "QKV"} for t in range(T)]
+    eta = torch.from_numpy(np.ascontiguousarray(data["eta"])).to(dev)
+    etas = [eta[:, :, t].contiguous() for t in range(T)]
+    gamma = torch.from_numpy(data["gamma"]).to(dev)
+    beta = torch.from_numpy(data["beta"]).to(dev)
+    W = torch.from_numpy(data["W0"]).to(dev).unsqueeze(0).expand(B, H, d, d).contiguous()
+    W_base = W.clone()
+    z = torch.empty(B, H, d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lib = _lib.load()
+
+    def step():
+        for t in range(T):
+            ttt.ttt_linear_ln_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], W, W_base, gamma,
+                                     beta, cfg.b, t, cfg.ln_eps, z=z, stream=stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_id_for(torch, 0))
+    clocks.start()
+    n0 = lib.ttt_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = lib.ttt_launch_count() - n0
+    clock_info = clocks.stop()
+    if ttt.last_device_status() != 0:
+        raise RuntimeError("device status error")
+    ms = e0.elapsed_time(e1)
+    units = B * H
+    value = units * T * args.steps / (ms / 1e3)
+    # Algorithmic bytes per mini-batch (16 calls) and unit: W_base and W read and W
+    # written each call, W_base written once, q/k/v (bf16), eta and z per call.
+    per_unit = T * (3 * d * d * 4 + 3 * d * 2 + 4 + d * 4) + d * d * 4
+    nbytes = units * per_unit
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / (ms / args.steps / 1e3) / 1e9
+    line = {
+        "metric": "TTT-Linear+LN decode step tokens/s (B x H units, one token each per call)",
+        "value": value, "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "B": B, "H": H, "d": d, "b": cfg.b,
+                   "step": "one mini-batch: 16 decode calls, positions 0..15", "qkv_dtype": "bf16",
+                   "l2": "state (2 x 268 MB) larger than L2 (no flush needed)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)",
+                     "algorithmic_bytes_per_step": nbytes},
+        "clocks": clock_info, "gpu_launches": int(launches),
+    }
+    print(json.dumps(line), flush=True)
 
 
 def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, torch, dist):

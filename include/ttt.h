@@ -117,6 +117,32 @@ TTT_API int ttt_mlp_fwd(const void *Q, const void *K, const void *V, int qkv_dty
                 float ln_eps, int B, int H, int T, int d, int hidden, int b, float *Z,
                 float *W1_out, float *W2_out, void *stream);
 
+/*
+ * Primal-form decode step (generation, §04.3 of the TTT write-up: decoding is
+ * sequential and takes the primal form): one token per (batch, head) and call,
+ * with the state carried in device memory across calls.
+ *   q, k, v  [B][H][d] (qkv_dtype), eta [B][H] fp32: this token's views and rate.
+ *   W        [B][H][d][d] fp32, in/out: the state W_t after the previous token.
+ *   W_base   [B][H][d][d] fp32, in/out: the state the current mini-batch started
+ *            from (every gradient of a mini-batch is taken there, §03.6).
+ *   pos      this token's position in its mini-batch of b tokens, 0 <= pos < b.
+ *   z        [B][H][d] fp32 out.
+ * Per (batch, head):
+ *   G = d l / d(k W_base)        2 (k W_base - v), or through LN and the residual
+ *   W <- W - eta k^T G,  z = q W  (or q + LN(q W)),  and W_base <- W if pos == b-1.
+ * Run over a sequence with pos = t mod b, starting from W = W_base = W0, the calls
+ * produce exactly the forward's Z and final state.  The caller owns all buffers;
+ * W and W_base must not overlap each other or the inputs.  Errors as for the
+ * forward entry points (host checks before any launch).
+ */
+TTT_API int ttt_linear_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                              const float *eta, float *W, float *W_base, int B, int H, int d,
+                              int b, int pos, float *z, void *stream);
+TTT_API int ttt_linear_ln_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                                 const float *eta, float *W, float *W_base, const float *ln_gamma,
+                                 const float *ln_beta, float ln_eps, int B, int H, int d, int b,
+                                 int pos, float *z, void *stream);
+
 /* Static English text for a ttt_status value (never NULL). */
 TTT_API const char *ttt_status_string(int status);
 

@@ -13,11 +13,13 @@
 
 #include "ttt.h"
 #include "device_status.cuh"
+#include "decode.cuh"
 #include "simt.cuh"
 #include "tc_linear.cuh"
 
 namespace simt = ttt::simt;
 namespace tc = ttt::tc;
+namespace decode = ttt::decode;
 
 namespace {
 
@@ -228,6 +230,53 @@ int launch_linear_tc(const Call &c) {
   return TTT_OK;
 }
 
+// One primal-form decode step (decode.cuh).  Checks on the host first, as the
+// forward entry points do.
+int run_decode(bool ln, const void *q, const void *k, const void *v, int qkv_dtype, const float *eta,
+               float *W, float *W_base, const float *gamma, const float *beta, float eps, int B,
+               int H, int d, int b, int pos, float *z, void *stream) {
+  if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (B < 0 || H < 0 || d <= 0 || b <= 0 || pos < 0 || pos >= b) return TTT_ERR_ARG;
+  if (ln && !(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
+  if (d != decode::D) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)B * H;
+  if (units == 0) return TTT_OK;
+  if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  const void *req[] = {q, k, v, eta, W, W_base, z, ln ? (const void *)gamma : q,
+                       ln ? (const void *)beta : q};
+  for (const void *x : req)
+    if (!x) return TTT_ERR_ARG;
+  for (const void *x : req)
+    if (!aligned16(x)) return TTT_ERR_ALIGN;
+  const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
+  Range ins[6] = {range_of(q, units * d * in_elt), range_of(k, units * d * in_elt),
+                  range_of(v, units * d * in_elt), range_of(eta, units * 4),
+                  range_of(ln ? (const void *)gamma : q, ln ? (size_t)H * d * 4 : 0),
+                  range_of(ln ? (const void *)beta : q, ln ? (size_t)H * d * 4 : 0)};
+  Range outs[3] = {range_of(W, units * d * d * 4), range_of(W_base, units * d * d * 4),
+                   range_of(z, units * d * 4)};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 6; ++i)
+      if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
+    for (int o2 = o + 1; o2 < 3; ++o2)
+      if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
+  }
+  decode::Params p{q, k, v, eta, W, W_base, gamma, beta, eps, H, pos, b, z};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bf16 = qkv_dtype == TTT_BF16;
+  const unsigned grid = (unsigned)units;
+  if (ln) {
+    if (bf16) decode::decode_kernel<true, __nv_bfloat16><<<grid, decode::THREADS, 0, s>>>(p);
+    else decode::decode_kernel<true, float><<<grid, decode::THREADS, 0, s>>>(p);
+  } else {
+    if (bf16) decode::decode_kernel<false, __nv_bfloat16><<<grid, decode::THREADS, 0, s>>>(p);
+    else decode::decode_kernel<false, float><<<grid, decode::THREADS, 0, s>>>(p);
+  }
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 int run(const Call &c) {
   const int st = validate(c);
   if (st != TTT_OK) return st;
@@ -298,5 +347,20 @@ int ttt_set_path(int path) {
 long long ttt_launch_count(void) { return g_launches.load(); }
 
 int ttt_debug_inject_timeout(int on) { return g_inject_timeout.exchange(on ? 1 : 0); }
+
+int ttt_linear_decode(const void *q, const void *k, const void *v, int qkv_dtype, const float *eta,
+                      float *W, float *W_base, int B, int H, int d, int b, int pos, float *z,
+                      void *stream) {
+  return run_decode(false, q, k, v, qkv_dtype, eta, W, W_base, nullptr, nullptr, 1.f, B, H, d, b,
+                    pos, z, stream);
+}
+
+int ttt_linear_ln_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                         const float *eta, float *W, float *W_base, const float *ln_gamma,
+                         const float *ln_beta, float ln_eps, int B, int H, int d, int b, int pos,
+                         float *z, void *stream) {
+  return run_decode(true, q, k, v, qkv_dtype, eta, W, W_base, ln_gamma, ln_beta, ln_eps, B, H, d,
+                    b, pos, z, stream);
+}
 
 }  // extern "C"

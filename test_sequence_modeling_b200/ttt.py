@@ -111,6 +111,50 @@ def ttt_mlp_fwd(Q, K, V, eta, W1, W2, gamma, beta, b, eps=1e-6, Z=None, W1_out=N
     return Z, W1_out, W2_out
 
 
+def _decode_args(q, k, v, eta, W, W_base, z):
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _cuda(t, n)
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _QKV_DTYPES:
+        raise TypeError("q, k, v must share one dtype, float32 or bfloat16")
+    if not (q.shape == k.shape == v.shape) or q.dim() != 3:
+        raise ValueError("q, k, v must have the same shape [B, H, d]")
+    B, H, d = q.shape
+    _cuda(eta, "eta", torch.float32)
+    if tuple(eta.shape) != (B, H):
+        raise ValueError(f"eta must have shape {(B, H)}")
+    for n, t in (("W", W), ("W_base", W_base)):
+        _cuda(t, n, torch.float32)
+        if tuple(t.shape) != (B, H, d, d):
+            raise ValueError(f"{n} must have shape {(B, H, d, d)}")
+    z = _out(z, (B, H, d), q.device, "z")
+    return _QKV_DTYPES[q.dtype], B, H, d, z
+
+
+def ttt_linear_decode(q, k, v, eta, W, W_base, b, pos, z=None, stream=None):
+    """One primal-form decode step of TTT-Linear (see include/ttt.h).  q, k, v [B,H,d],
+    eta [B,H]; W and W_base [B,H,d,d] f32 are updated in place.  Returns z [B,H,d] f32."""
+    dt, B, H, d, z = _decode_args(q, k, v, eta, W, W_base, z)
+    with torch.cuda.device(q.device):
+        st = _lib.load().ttt_linear_decode(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta), _ptr(W),
+                                           _ptr(W_base), B, H, d, int(b), int(pos), _ptr(z),
+                                           _stream(stream, q.device))
+    check(st, "ttt_linear_decode")
+    return z
+
+
+def ttt_linear_ln_decode(q, k, v, eta, W, W_base, gamma, beta, b, pos, eps=1e-6, z=None, stream=None):
+    """One primal-form decode step of TTT-Linear with LN + residual; gamma, beta [H,d] f32."""
+    dt, B, H, d, z = _decode_args(q, k, v, eta, W, W_base, z)
+    for n, t in (("gamma", gamma), ("beta", beta)):
+        _cuda(t, n, torch.float32)
+    with torch.cuda.device(q.device):
+        st = _lib.load().ttt_linear_ln_decode(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta), _ptr(W),
+                                              _ptr(W_base), _ptr(gamma), _ptr(beta), float(eps), B, H,
+                                              d, int(b), int(pos), _ptr(z), _stream(stream, q.device))
+    check(st, "ttt_linear_ln_decode")
+    return z
+
+
 def set_path(path: int) -> int:
     """Select the kernel path (TTT_PATH_AUTO / _SIMT / _TC); returns the previous one."""
     prev = _lib.load().ttt_set_path(int(path))

@@ -119,3 +119,36 @@ def test_python_binding_rejects_cpu_tensors():
     x = torch.zeros(1, 1, 16, 64)
     with pytest.raises(ValueError, match="CUDA"):
         ttt.ttt_linear_fwd(x, x, x, torch.zeros(1, 1, 16), torch.zeros(1, 64, 64), 16)
+
+
+def decode(lib, ln=False, **kw):
+    q, k, v, eta, w, wb, z, g, bt = _ptrs(9)
+    a = dict(q=q, k=k, v=v, dt=L.TTT_BF16, eta=eta, W=w, Wb=wb, g=g, bt=bt, eps=1e-6, B=2, H=3,
+             d=64, b=16, pos=0, z=z)
+    a.update(kw)
+    if ln:
+        return lib.ttt_linear_ln_decode(a["q"], a["k"], a["v"], a["dt"], a["eta"], a["W"], a["Wb"],
+                                        a["g"], a["bt"], a["eps"], a["B"], a["H"], a["d"], a["b"],
+                                        a["pos"], a["z"], None)
+    return lib.ttt_linear_decode(a["q"], a["k"], a["v"], a["dt"], a["eta"], a["W"], a["Wb"], a["B"],
+                                 a["H"], a["d"], a["b"], a["pos"], a["z"], None)
+
+
+@pytest.mark.parametrize("ln", [False, True])
+def test_decode_argument_errors(lib, ln):
+    n0 = lib.ttt_launch_count()
+    assert decode(lib, ln, pos=16) == L.TTT_ERR_ARG       # pos outside the mini-batch
+    assert decode(lib, ln, pos=-1) == L.TTT_ERR_ARG
+    assert decode(lib, ln, b=0) == L.TTT_ERR_ARG
+    assert decode(lib, ln, dt=3) == L.TTT_ERR_ARG
+    assert decode(lib, ln, d=32) == L.TTT_ERR_UNSUPPORTED
+    assert decode(lib, ln, q=None) == L.TTT_ERR_ARG
+    assert decode(lib, ln, Wb=None) == L.TTT_ERR_ARG
+    assert decode(lib, ln, W=A + 8) == L.TTT_ERR_ALIGN
+    assert decode(lib, ln, Wb=A + (6 << 30)) == L.TTT_ERR_ARG  # W_base overlaps z
+    assert decode(lib, ln, W=A + (4 << 30) + 1024, Wb=A + (4 << 30) + 4096) == L.TTT_ERR_ARG
+    assert decode(lib, ln, B=0) == L.TTT_OK
+    if ln:
+        assert decode(lib, ln, eps=0.0) == L.TTT_ERR_ARG
+        assert decode(lib, ln, g=None) == L.TTT_ERR_ARG
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
