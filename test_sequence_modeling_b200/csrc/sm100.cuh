@@ -31,16 +31,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
-// Tests the phase of the given parity; the thread may sleep up to ~1 ms (the
-// suspend-time hint) waiting for it, and wakes as soon as the phase completes.
+// Tests the phase of the given parity; the thread may wait for it up to a
+// system-dependent time limit (no suspend-time hint: a hinted wait was measured
+// slower to resume on the chain of the tensor-core kernel).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }

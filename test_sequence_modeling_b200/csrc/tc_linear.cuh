@@ -152,6 +152,7 @@ __device__ __forceinline__ float quad_sum(float x) {
 // Waits, or flags the CTA as aborted and records the timeout if the wait expires.
 __device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort,
                                               long long limit = WAIT_LIMIT) {
+  if (mbar_try_wait(bar, parity)) return;  // the common case: no shared-flag read
   if (*abort) return;
   if (!mbar_wait(bar, parity, limit)) {
     *abort = 1;
@@ -323,10 +324,12 @@ __global__ void __launch_bounds__(THREADS, 4)
 #pragma unroll
     for (int w = 0; w < 4; ++w) wait_or_abort(&bars[BAR_LOADQ + w], par, abort);
     // Products are issued by one elected lane of a converged warp (the whole warp
-    // computes the operand descriptors).
+    // computes the operand descriptors).  No product waits on the abort flag:
+    // products issued after an expired wait are harmless (they complete, and the
+    // drain at the end waits for them).
     if (warp == 0) {
       __syncwarp();
-      const bool issue = elect_one_sync() && !*abort;
+      const bool issue = elect_one_sync();
       tc_fence_after_sync();
       // S = [K;Q] K^T: B = the K rows alone (every other 8-row group, 2 KB apart).
 #pragma unroll
@@ -475,7 +478,7 @@ __global__ void __launch_bounds__(THREADS, 4)
       named_barrier_sync(1 + (warp & 1), 64);
       if (hh == 0) {
         __syncwarp();
-        const bool issue = elect_one_sync() && !*abort;
+        const bool issue = elect_one_sync();
         tc_fence_after_sync();
         const uint64_t bhi = smem_desc_sw128(aGhi + 2048 * m, 8192, 1024);
         const uint64_t blo = smem_desc_sw128(aGlo + 2048 * m, 8192, 1024);
@@ -490,6 +493,19 @@ __global__ void __launch_bounds__(THREADS, 4)
     // Outputs of this warp's Q rows: after their mini-batch's update they are
     // final (later updates add exactly zero to them, A being zero there).
     float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
+    // Q residuals of both rows first, so that the Q rows can be refilled with the
+    // next chunk before the outputs are computed.
+    uint32_t qres[2][8];
+    if (LN) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          qres[i][j] = lds_u32(sbase + kq_offset(MB * (mb0 + i) + 8 * hh + fr, 1, 8 * j + 2 * q4));
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int m = mb0 + i;
@@ -519,7 +535,7 @@ __global__ void __launch_bounds__(THREADS, 4)
           const int col = 8 * j + 2 * q4;
           const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_GB + 16 * (4 * j + q4));
           const float2 gm = make_float2(gb.x, gb.y), bt = make_float2(gb.z, gb.w);
-          const float2 q = unpack_bf16x2(lds_u32(sbase + kq_offset(tq, 1, col)));
+          const float2 q = unpack_bf16x2(qres[i][j]);
           *reinterpret_cast<float2 *>(zrow + col) = __fadd2_rn(q, __ffma2_rn(gm, __fmul2_rn(z[j], rs), bt));
         }
       } else {
@@ -527,16 +543,13 @@ __global__ void __launch_bounds__(THREADS, 4)
         for (int j = 0; j < 8; ++j) *reinterpret_cast<float2 *>(zrow + 8 * j + 2 * q4) = z[j];
       }
     }
-    // This warp's Q rows are no longer needed: refill them with the next chunk.
-    __syncwarp();
-    if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
 
     // ---- 5: dW on the tensor core after the last update; state update -------------
     wait_or_abort(&bars[BAR_LAST], par, abort);
     tc_fence_after_sync();
     if (warp == 0) {
       __syncwarp();
-      const bool issue = elect_one_sync() && !*abort;
+      const bool issue = elect_one_sync();
       // dW = K^T (eta G) into the S columns (their operand is consumed).  Step k
       // takes the K rows of groups 4k and 4k + 2 (tokens of mini-batches
       // 2(k % 2), 2(k % 2) + 1, half k / 2), read twice (lbo 0) so that rows
