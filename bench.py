@@ -33,7 +33,10 @@ METRIC = "TTT layer fwd tokens/s (B×H×T/s) on 1 B200; % of roofline (HBM vs te
 UNIT = "head-tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ("test_sequence_modeling_b200/csrc",)
+# The sources the tensor-core kernel is compiled from (its launch included): a
+# committed DRAM-traffic record is only reported while these are unchanged.
+KERNEL_SOURCES = tuple("test_sequence_modeling_b200/csrc/" + f
+                       for f in ("tc_linear.cuh", "sm100.cuh", "device_status.cuh", "ttt_api.cu"))
 
 
 # --- workload accounting --------------------------------------------------------
@@ -70,11 +73,9 @@ def load_peaks():
 
 def kernel_source_sha() -> str:
     h = hashlib.sha256()
-    for d in KERNEL_SOURCES:
-        full = os.path.join(ROOT, d)
-        for name in sorted(os.listdir(full)):
-            with open(os.path.join(full, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(os.path.basename(rel).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
 
 

@@ -223,17 +223,18 @@ __global__ void __launch_bounds__(THREADS) linear_kernel(const Params p) {
 // thread (j, e) owns column j and hidden eighth e.
 constexpr int MBR = 16;
 constexpr int HT_LD = 20;
+constexpr int DT_LD = 20;  // padded stride of the [D][16] transposed tiles
 constexpr int MLP_THREADS = 512;
 
 struct MlpSmem {
   float W1[D * HID];          // [D][HID] state
   float W2[HID * W2_LD];      // [HID][W2_LD] state
-  float Qt[D * MBR], Kt[D * MBR];
+  float Qt[D * DT_LD], Kt[D * DT_LD];
   float V[MBR * D];           // [16][D]
   float X2t[HID * HT_LD];     // GELU(K W1), [HID][16]
   float Z2t[HID * HT_LD];     // GELU(Z1), [HID][16]
   float G3[MBR * D];          // X2 W2, then dl/d(X2 W2), [16][D]
-  float G3t[D * MBR];         // G3 transposed
+  float G3t[D * DT_LD];       // G3 transposed
   union {
     float part[4 * MBR * D];  // partial sums over hidden parts
     float G2t[HID * HT_LD];   // dl/dX1, [HID][16] (between the X3 and A2 passes)
@@ -299,8 +300,8 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
     for (int x = tid; x < MBR * D; x += MLP_THREADS) {
       const int r = x / D, c = x % D;
       const bool in = r < b;
-      S.Qt[c * MBR + r] = in ? load_in(Qg, off + r * D + c) : 0.f;
-      S.Kt[c * MBR + r] = in ? load_in(Kg, off + r * D + c) : 0.f;
+      S.Qt[c * DT_LD + r] = in ? load_in(Qg, off + r * D + c) : 0.f;
+      S.Kt[c * DT_LD + r] = in ? load_in(Kg, off + r * D + c) : 0.f;
       S.V[x] = in ? load_in(Vg, off + x) : 0.f;
     }
     if (tid < MBR) S.eta[tid] = tid < b ? p.eta[tok0 + (long)n * b + tid] : 0.f;
@@ -316,8 +317,8 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
         const float w = S.W1[pp * HID + i];
         const float2 ww = make_float2(w, w);
         float2 kv[4], qv[4];
-        load_rows(&S.Kt[pp * MBR + r0], kv);
-        load_rows(&S.Qt[pp * MBR + r0], qv);
+        load_rows(&S.Kt[pp * DT_LD + r0], kv);
+        load_rows(&S.Qt[pp * DT_LD + r0], qv);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           x1[k] = ffma2(kv[k], ww, x1[k]);
@@ -335,7 +336,7 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
       float acc = 0.f;
       if (s0 <= t) {
 #pragma unroll 8
-        for (int pp = 0; pp < D; ++pp) acc = fmaf(S.Qt[pp * MBR + t], S.Kt[pp * MBR + s0], acc);
+        for (int pp = 0; pp < D; ++pp) acc = fmaf(S.Qt[pp * DT_LD + t], S.Kt[pp * DT_LD + s0], acc);
         acc *= S.eta[s0];
       }
       S.A[tid] = acc;
@@ -384,13 +385,13 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
     {
       const int r = warp;
       float dy0, dy1;
-      ln_residual_grad(S.G3[r * D + lane], S.G3[r * D + lane + 32], S.Kt[lane * MBR + r],
-                       S.Kt[(lane + 32) * MBR + r], S.V[r * D + lane], S.V[r * D + lane + 32], gam0,
+      ln_residual_grad(S.G3[r * D + lane], S.G3[r * D + lane + 32], S.Kt[lane * DT_LD + r],
+                       S.Kt[(lane + 32) * DT_LD + r], S.V[r * D + lane], S.V[r * D + lane + 32], gam0,
                        gam1, bet0, bet1, p.eps, dy0, dy1);
       S.G3[r * D + lane] = dy0;
       S.G3[r * D + lane + 32] = dy1;
-      S.G3t[lane * MBR + r] = dy0;
-      S.G3t[(lane + 32) * MBR + r] = dy1;
+      S.G3t[lane * DT_LD + r] = dy0;
+      S.G3t[(lane + 32) * DT_LD + r] = dy1;
     }
     __syncthreads();
 
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
         const float w = S.W2[i * W2_LD + jj];
         const float2 ww = make_float2(w, w);
         float2 gv[4];
-        load_rows(&S.G3t[jj * MBR + r0], gv);
+        load_rows(&S.G3t[jj * DT_LD + r0], gv);
 #pragma unroll
         for (int k = 0; k < 4; ++k) g2[k] = ffma2(gv[k], ww, g2[k]);
       }
@@ -452,7 +453,7 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
 #pragma unroll 4
       for (int pp = D / 2 * rh; pp < D / 2 * (rh + 1); ++pp) {
         float2 kv[8];
-        load_rows(&S.Kt[pp * MBR], kv);
+        load_rows(&S.Kt[pp * DT_LD], kv);
         float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < 8; ++k) acc = ffma2(kv[k], g[k], acc);
@@ -503,7 +504,7 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_kernel(const Params p) {
           y[h] = acc;
         }
         float z0, z1;
-        ln_residual_fwd(y[0], y[1], S.Qt[lane * MBR + r], S.Qt[(lane + 32) * MBR + r], gam0, gam1, bet0,
+        ln_residual_fwd(y[0], y[1], S.Qt[lane * DT_LD + r], S.Qt[(lane + 32) * DT_LD + r], gam0, gam1, bet0,
                         bet1, p.eps, z0, z1);
         Zg[off + r * D + lane] = z0;
         Zg[off + r * D + lane + 32] = z1;
