@@ -1,0 +1,37 @@
+"""GPU: the host-memory forward (copies of batch chunks overlapped with the
+forwards on three streams) gives exactly the device-resident forward's outputs."""
+import numpy as np
+import pytest
+import torch
+
+from test_sequence_modeling_b200 import inputs as I
+from test_sequence_modeling_b200.host import HostForward
+from gpu_helpers import run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["linear_bf16_B16H12T2048", "linear_ln_B16H32T8192", "mlp_B8H32T8192"])
+@pytest.mark.parametrize("chunks", [1, 3])
+def test_host_forward_equals_device_forward(name, chunks):
+    cfg = I.CONFIGS[name].replace(B=5, H=3, T=128)
+    data = I.make_inputs(cfg)
+    dev = to_device(cfg, data)
+    ref = run_gpu(cfg, dev)
+    host = {k: v.cpu().pin_memory() for k, v in dev.items()}
+    Z = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d, pin_memory=True)
+    if cfg.variant == "mlp":
+        params = [host[k] for k in ("W1", "W2", "gamma", "beta")]
+        w_shapes = [(cfg.H, cfg.d, cfg.hidden), (cfg.H, cfg.hidden, cfg.d)]
+        outs, keys = [torch.empty((cfg.B,) + s[1:], pin_memory=True) for s in
+                      [(0, cfg.H, cfg.d, cfg.hidden), (0, cfg.H, cfg.hidden, cfg.d)]], ["W1", "W2"]
+    else:
+        params = [host["W0"]] + ([host["gamma"], host["beta"]] if cfg.variant == "linear_ln" else [])
+        w_shapes = [(cfg.H, cfg.d, cfg.d)]
+        outs, keys = [torch.empty(cfg.B, cfg.H, cfg.d, cfg.d, pin_memory=True)], ["W"]
+    fwd = HostForward(cfg.variant, host["Q"], w_shapes, [p.shape for p in params], chunks=chunks)
+    done = fwd.run(host["Q"], host["K"], host["V"], host["eta"], params, cfg.b, cfg.ln_eps, Z, outs)
+    done.synchronize()
+    assert np.array_equal(Z.numpy(), ref["Z"])
+    for k, o in zip(keys, outs):
+        assert np.array_equal(o.numpy(), ref[k]), k
