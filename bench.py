@@ -33,10 +33,10 @@ METRIC = "TTT layer fwd tokens/s (B×H×T/s) on 1 B200; % of roofline (HBM vs te
 UNIT = "head-tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# The sources the tensor-core kernel is compiled from (its launch included): a
-# committed DRAM-traffic record is only reported while these are unchanged.
+# The sources the tensor-core kernel is compiled from: a committed DRAM-traffic
+# record is only reported while these are unchanged.
 KERNEL_SOURCES = tuple("test_sequence_modeling_b200/csrc/" + f
-                       for f in ("tc_linear.cuh", "sm100.cuh", "device_status.cuh", "ttt_api.cu"))
+                       for f in ("tc_linear.cuh", "sm100.cuh", "device_status.cuh"))
 
 
 # --- workload accounting --------------------------------------------------------
@@ -273,9 +273,11 @@ def main():
     ap.add_argument("--decode", action="store_true",
                     help="time the primal-form decode step (TTT-Linear + LN, B=512 H=32, bf16 q/k/v) "
                          "instead of the forward")
+    ap.add_argument("--decode-mlp", action="store_true",
+                    help="the same for the TTT-MLP decode step")
     args = ap.parse_args()
-    if args.decode:
-        return run_decode(args)
+    if args.decode or args.decode_mlp:
+        return run_decode(args, mlp=args.decode_mlp)
     cfg = I.CONFIGS[args.workload]
     if args.batch is not None or args.seq is not None:
         cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T,
@@ -385,7 +387,7 @@ def main():
                   e2e, peaks, peak_kind, nbytes, nflops, dist)
 
 
-def run_decode(args):
+def run_decode(args, mlp=False):
     """The decode step's own line: one timed step = one mini-batch of 16 decode calls
     (positions 0..15) over B=512 x H=32 (batch, head) units, the state in HBM."""
     import torch
@@ -393,7 +395,10 @@ def run_decode(args):
     from test_sequence_modeling_b200 import _lib
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
-    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=512, T=16, name="decode_linear_ln_B512H32")
+    if mlp:
+        cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=512, T=16, name="decode_mlp_B512H32")
+    else:
+        cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=512, T=16, name="decode_linear_ln_B512H32")
     data = I.make_inputs(cfg)
     B, H, T, d = cfg.B, cfg.H, cfg.T, cfg.d
     qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
@@ -402,16 +407,26 @@ def run_decode(args):
     etas = [eta[:, :, t].contiguous() for t in range(T)]
     gamma = torch.from_numpy(data["gamma"]).to(dev)
     beta = torch.from_numpy(data["beta"]).to(dev)
-    W = torch.from_numpy(data["W0"]).to(dev).unsqueeze(0).expand(B, H, d, d).contiguous()
-    W_base = W.clone()
+    if mlp:
+        h = cfg.hidden
+        W1 = torch.from_numpy(data["W1"]).to(dev).unsqueeze(0).expand(B, H, d, h).contiguous()
+        W2 = torch.from_numpy(data["W2"]).to(dev).unsqueeze(0).expand(B, H, h, d).contiguous()
+        W1b, W2b = W1.clone(), W2.clone()
+    else:
+        W = torch.from_numpy(data["W0"]).to(dev).unsqueeze(0).expand(B, H, d, d).contiguous()
+        W_base = W.clone()
     z = torch.empty(B, H, d, device=dev)
     stream = torch.cuda.current_stream(dev)
     lib = _lib.load()
 
     def step():
         for t in range(T):
-            ttt.ttt_linear_ln_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], W, W_base, gamma,
-                                     beta, cfg.b, t, cfg.ln_eps, z=z, stream=stream)
+            if mlp:
+                ttt.ttt_mlp_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], W1, W2, W1b, W2b, gamma,
+                                   beta, cfg.b, t, cfg.ln_eps, z=z, stream=stream)
+            else:
+                ttt.ttt_linear_ln_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], W, W_base, gamma,
+                                         beta, cfg.b, t, cfg.ln_eps, z=z, stream=stream)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -434,18 +449,21 @@ def run_decode(args):
     value = units * T * args.steps / (ms / 1e3)
     # Algorithmic bytes per mini-batch (16 calls) and unit: W_base and W read and W
     # written each call, W_base written once, q/k/v (bf16), eta and z per call.
-    per_unit = T * (3 * d * d * 4 + 3 * d * 2 + 4 + d * 4) + d * d * 4
+    if mlp:  # W1b, W2b, W1, W2 read and W1, W2 written per call; the bases written once
+        per_unit = T * (6 * d * cfg.hidden * 4 + 3 * d * 2 + 4 + d * 4) + 2 * d * cfg.hidden * 4
+    else:
+        per_unit = T * (3 * d * d * 4 + 3 * d * 2 + 4 + d * 4) + d * d * 4
     nbytes = units * per_unit
     peaks, peak_kind = load_peaks()
     achieved = nbytes / (ms / args.steps / 1e3) / 1e9
     line = {
-        "metric": "TTT-Linear+LN decode step tokens/s (B x H units, one token each per call)",
+        "metric": ("TTT-MLP" if mlp else "TTT-Linear+LN") + " decode step tokens/s (B x H units, one token each per call)",
         "value": value, "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "B": B, "H": H, "d": d, "b": cfg.b,
                    "step": "one mini-batch: 16 decode calls, positions 0..15", "qkv_dtype": "bf16",
-                   "l2": "state (2 x 268 MB) larger than L2 (no flush needed)"},
+                   "l2": "state larger than L2 (no flush needed)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)",

@@ -143,6 +143,19 @@ TTT_API int ttt_linear_ln_decode(const void *q, const void *k, const void *v, in
                                  const float *ln_beta, float ln_eps, int B, int H, int d, int b,
                                  int pos, float *z, void *stream);
 
+/*
+ * The same step for TTT-MLP, f(x) = x + LN(GELU(x W1) W2): the state is W1
+ * [B][H][d][hidden] and W2 [B][H][hidden][d] (fp32, in/out) with their
+ * mini-batch bases W1_base, W2_base (in/out); hidden = 4 d.  Per (batch, head),
+ * with X1 = k W1_base, X2 = GELU(X1) and G3, G2 the loss gradients w.r.t.
+ * X2 W2_base and X1:  W1 <- W1 - eta k^T G2,  W2 <- W2 - eta X2^T G3,
+ * z = q + LN(GELU(q W1) W2), and both bases follow at pos == b - 1.
+ */
+TTT_API int ttt_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                           const float *eta, float *W1, float *W2, float *W1_base, float *W2_base,
+                           const float *ln_gamma, const float *ln_beta, float ln_eps, int B, int H,
+                           int d, int hidden, int b, int pos, float *z, void *stream);
+
 /* Static English text for a ttt_status value (never NULL). */
 TTT_API const char *ttt_status_string(int status);
 

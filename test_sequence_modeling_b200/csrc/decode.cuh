@@ -1,5 +1,5 @@
-// decode.cuh - primal-form decode step of TTT-Linear and TTT-Linear + LN: one
-// token per (batch, head) and call, the state carried in HBM.  Decoding is
+// decode.cuh - primal-form decode step of TTT-Linear, TTT-Linear + LN and
+// TTT-MLP: one token per (batch, head) and call, the state carried in HBM.  Decoding is
 // sequential, so it takes the primal form rather than the dual one (TTT
 // write-up §04.3, generation).
 //
@@ -106,6 +106,143 @@ __global__ void __launch_bounds__(THREADS) decode_kernel(const Params p) {
       simt::ln_residual_fwd(z0, z1, qs[lane], qs[lane + 32], p.gamma[head * D + lane],
                             p.gamma[head * D + lane + 32], p.beta[head * D + lane],
                             p.beta[head * D + lane + 32], p.eps, o0, o1);
+    p.z[unit * D + lane] = o0;
+    p.z[unit * D + lane + 32] = o1;
+  }
+}
+
+// TTT-MLP, f(x) = x + LN(GELU(x W1) W2) (§03.9): the same step with two state
+// matrices, W1 [D][HID] and W2 [HID][D], each with its mini-batch base.  With
+// X1 = k W1b, X2 = GELU(X1), X3 = X2 W2b and G3 = dl/dX3 (LN backward), the
+// gradient w.r.t. X1 is G2 = (G3 W2b^T) * GELU'(X1), and
+//   W1 <- W1 - eta k^T G2,  W2 <- W2 - eta X2^T G3,
+//   z   = q + LN(GELU(q W1) W2)   with the updated W1, W2.
+// Per (batch, head) a call reads the four matrices (256 KB) and writes W1, W2
+// (128 KB, and the bases once per mini-batch).  Thread i of the CTA owns hidden
+// unit i: column i of W1 (and W1b) and row i of W2 (and W2b).
+struct MlpParams {
+  const void *q, *k, *v;
+  const float *eta;
+  float *W1, *W2, *W1_base, *W2_base;  // [units][D][HID], [units][HID][D]
+  const float *gamma, *beta;
+  float eps;
+  int H, pos, b;
+  float *z;
+};
+constexpr int HID = simt::HID;
+constexpr int MLP_THREADS = HID;
+
+template <typename InT>
+__global__ void __launch_bounds__(MLP_THREADS) mlp_decode_kernel(const MlpParams p) {
+  __shared__ float qs[D], ks[D], vs[D], x2s[HID], z2s[HID], g3[D], part[8][D];
+  const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+  const long unit = blockIdx.x;
+  const int head = (int)(unit % p.H);
+  if (i < D) {
+    qs[i] = simt::load_in(static_cast<const InT *>(p.q), unit * D + i);
+    ks[i] = simt::load_in(static_cast<const InT *>(p.k), unit * D + i);
+    vs[i] = simt::load_in(static_cast<const InT *>(p.v), unit * D + i);
+  }
+  float *W1 = p.W1 + unit * D * HID, *W1b = p.W1_base + unit * D * HID;
+  float *W2 = p.W2 + unit * HID * D, *W2b = p.W2_base + unit * HID * D;
+  __syncthreads();
+
+  // X1 = k W1b (column i), X2 = GELU(X1).
+  float x1 = 0.f;
+#pragma unroll 8
+  for (int pp = 0; pp < D; ++pp) x1 = fmaf(ks[pp], W1b[pp * HID + i], x1);
+  const float x2 = simt::gelu(x1);
+  x2s[i] = x2;
+  __syncthreads();
+  // X3 = X2 W2b: warp w sums hidden rows 32w .. 32w + 31 for columns lane, lane + 32.
+  {
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) {
+      const int ii = 32 * warp + r;
+      a0 = fmaf(x2s[ii], W2b[ii * D + lane], a0);
+      a1 = fmaf(x2s[ii], W2b[ii * D + lane + 32], a1);
+    }
+    part[warp][lane] = a0;
+    part[warp][lane + 32] = a1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      y0 += part[w][lane];
+      y1 += part[w][lane + 32];
+    }
+    float d0, d1;
+    simt::ln_residual_grad(y0, y1, ks[lane], ks[lane + 32], vs[lane], vs[lane + 32],
+                           p.gamma[head * D + lane], p.gamma[head * D + lane + 32], p.beta[head * D + lane],
+                           p.beta[head * D + lane + 32], p.eps, d0, d1);
+    g3[lane] = d0;
+    g3[lane + 32] = d1;
+  }
+  __syncthreads();
+  // G2 = (G3 W2b^T) * GELU'(X1) for hidden unit i (row i of W2b).
+  float g2 = 0.f;
+  {
+    const float4 *row = reinterpret_cast<const float4 *>(W2b + i * D);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c) {
+      const float4 w = row[c];
+      g2 = fmaf(g3[4 * c], w.x, g2);
+      g2 = fmaf(g3[4 * c + 1], w.y, g2);
+      g2 = fmaf(g3[4 * c + 2], w.z, g2);
+      g2 = fmaf(g3[4 * c + 3], w.w, g2);
+    }
+  }
+  const float e = p.eta[unit];
+  g2 *= simt::gelu_deriv(x1) * e;
+  const bool last = p.pos == p.b - 1;
+  // W1 -= eta k^T G2 (column i) and Z1 = q W1 with the updated W1.
+  float z1 = 0.f;
+#pragma unroll 8
+  for (int pp = 0; pp < D; ++pp) {
+    const float w = fmaf(-ks[pp], g2, W1[pp * HID + i]);
+    W1[pp * HID + i] = w;
+    if (last) W1b[pp * HID + i] = w;
+    z1 = fmaf(qs[pp], w, z1);
+  }
+  z2s[i] = simt::gelu(z1);
+  __syncthreads();
+  // W2 -= eta X2^T G3 (rows 32w .. 32w + 31) and Z3 = Z2 W2 with the updated W2.
+  {
+    const float eg0 = e * g3[lane], eg1 = e * g3[lane + 32];
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll 8
+    for (int r = 0; r < 32; ++r) {
+      const int ii = 32 * warp + r;
+      const float w0 = fmaf(-x2s[ii], eg0, W2[ii * D + lane]);
+      const float w1 = fmaf(-x2s[ii], eg1, W2[ii * D + lane + 32]);
+      W2[ii * D + lane] = w0;
+      W2[ii * D + lane + 32] = w1;
+      if (last) {
+        W2b[ii * D + lane] = w0;
+        W2b[ii * D + lane + 32] = w1;
+      }
+      a0 = fmaf(z2s[ii], w0, a0);
+      a1 = fmaf(z2s[ii], w1, a1);
+    }
+    __syncthreads();  // every warp has read part[] of the X3 pass long before; reuse it
+    part[warp][lane] = a0;
+    part[warp][lane + 32] = a1;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      y0 += part[w][lane];
+      y1 += part[w][lane + 32];
+    }
+    float o0, o1;
+    simt::ln_residual_fwd(y0, y1, qs[lane], qs[lane + 32], p.gamma[head * D + lane],
+                          p.gamma[head * D + lane + 32], p.beta[head * D + lane],
+                          p.beta[head * D + lane + 32], p.eps, o0, o1);
     p.z[unit * D + lane] = o0;
     p.z[unit * D + lane + 32] = o1;
   }

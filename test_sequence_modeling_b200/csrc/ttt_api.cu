@@ -277,6 +277,46 @@ int run_decode(bool ln, const void *q, const void *k, const void *v, int qkv_dty
   return TTT_OK;
 }
 
+// One primal-form decode step of TTT-MLP (decode.cuh), host checks first.
+int run_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype, const float *eta,
+                   float *W1, float *W2, float *W1_base, float *W2_base, const float *gamma,
+                   const float *beta, float eps, int B, int H, int d, int hidden, int b, int pos,
+                   float *z, void *stream) {
+  if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (B < 0 || H < 0 || d <= 0 || hidden <= 0 || b <= 0 || pos < 0 || pos >= b) return TTT_ERR_ARG;
+  if (!(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
+  if (d != decode::D || hidden != decode::HID) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)B * H;
+  if (units == 0) return TTT_OK;
+  if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  const void *req[] = {q, k, v, eta, W1, W2, W1_base, W2_base, z, gamma, beta};
+  for (const void *x : req)
+    if (!x) return TTT_ERR_ARG;
+  for (const void *x : req)
+    if (!aligned16(x)) return TTT_ERR_ALIGN;
+  const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t wbytes = (size_t)units * d * hidden * 4;
+  Range ins[6] = {range_of(q, units * d * in_elt), range_of(k, units * d * in_elt),
+                  range_of(v, units * d * in_elt), range_of(eta, units * 4),
+                  range_of(gamma, (size_t)H * d * 4), range_of(beta, (size_t)H * d * 4)};
+  Range outs[5] = {range_of(W1, wbytes), range_of(W2, wbytes), range_of(W1_base, wbytes),
+                   range_of(W2_base, wbytes), range_of(z, units * d * 4)};
+  for (int o = 0; o < 5; ++o) {
+    for (int i = 0; i < 6; ++i)
+      if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
+    for (int o2 = o + 1; o2 < 5; ++o2)
+      if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
+  }
+  decode::MlpParams p{q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, eps, H, pos, b, z};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)units;
+  if (qkv_dtype == TTT_BF16) decode::mlp_decode_kernel<__nv_bfloat16><<<grid, decode::MLP_THREADS, 0, s>>>(p);
+  else decode::mlp_decode_kernel<float><<<grid, decode::MLP_THREADS, 0, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 int run(const Call &c) {
   const int st = validate(c);
   if (st != TTT_OK) return st;
@@ -353,6 +393,14 @@ int ttt_linear_decode(const void *q, const void *k, const void *v, int qkv_dtype
                       void *stream) {
   return run_decode(false, q, k, v, qkv_dtype, eta, W, W_base, nullptr, nullptr, 1.f, B, H, d, b,
                     pos, z, stream);
+}
+
+int ttt_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype, const float *eta,
+                   float *W1, float *W2, float *W1_base, float *W2_base, const float *ln_gamma,
+                   const float *ln_beta, float ln_eps, int B, int H, int d, int hidden, int b, int pos,
+                   float *z, void *stream) {
+  return run_mlp_decode(q, k, v, qkv_dtype, eta, W1, W2, W1_base, W2_base, ln_gamma, ln_beta, ln_eps,
+                        B, H, d, hidden, b, pos, z, stream);
 }
 
 int ttt_linear_ln_decode(const void *q, const void *k, const void *v, int qkv_dtype,

@@ -155,6 +155,36 @@ def ttt_linear_ln_decode(q, k, v, eta, W, W_base, gamma, beta, b, pos, eps=1e-6,
     return z
 
 
+def ttt_mlp_decode(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, b, pos, eps=1e-6, z=None,
+                   stream=None):
+    """One primal-form decode step of TTT-MLP.  W1, W1_base [B,H,d,hidden] and W2, W2_base
+    [B,H,hidden,d] f32 are updated in place; gamma, beta [H,d].  Returns z [B,H,d] f32."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _cuda(t, n)
+    if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _QKV_DTYPES:
+        raise TypeError("q, k, v must share one dtype, float32 or bfloat16")
+    if not (q.shape == k.shape == v.shape) or q.dim() != 3:
+        raise ValueError("q, k, v must have the same shape [B, H, d]")
+    B, H, d = q.shape
+    hidden = W1.shape[-1]
+    _cuda(eta, "eta", torch.float32)
+    for n, t, shp in (("W1", W1, (B, H, d, hidden)), ("W1_base", W1_base, (B, H, d, hidden)),
+                      ("W2", W2, (B, H, hidden, d)), ("W2_base", W2_base, (B, H, hidden, d))):
+        _cuda(t, n, torch.float32)
+        if tuple(t.shape) != shp:
+            raise ValueError(f"{n} must have shape {shp}")
+    for n, t in (("gamma", gamma), ("beta", beta)):
+        _cuda(t, n, torch.float32)
+    z = _out(z, (B, H, d), q.device, "z")
+    with torch.cuda.device(q.device):
+        st = _lib.load().ttt_mlp_decode(_ptr(q), _ptr(k), _ptr(v), _QKV_DTYPES[q.dtype], _ptr(eta),
+                                        _ptr(W1), _ptr(W2), _ptr(W1_base), _ptr(W2_base), _ptr(gamma),
+                                        _ptr(beta), float(eps), B, H, d, hidden, int(b), int(pos), _ptr(z),
+                                        _stream(stream, q.device))
+    check(st, "ttt_mlp_decode")
+    return z
+
+
 def set_path(path: int) -> int:
     """Select the kernel path (TTT_PATH_AUTO / _SIMT / _TC); returns the previous one."""
     prev = _lib.load().ttt_set_path(int(path))

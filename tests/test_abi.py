@@ -152,3 +152,27 @@ def test_decode_argument_errors(lib, ln):
         assert decode(lib, ln, eps=0.0) == L.TTT_ERR_ARG
         assert decode(lib, ln, g=None) == L.TTT_ERR_ARG
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
+
+
+def test_mlp_decode_argument_errors(lib):
+    n0 = lib.ttt_launch_count()
+    q, k, v, eta, w1, w2, w1b, w2b, z, g, bt = _ptrs(11)
+
+    def call(**kw):
+        a = dict(q=q, k=k, v=v, dt=L.TTT_BF16, eta=eta, w1=w1, w2=w2, w1b=w1b, w2b=w2b, g=g, bt=bt,
+                 eps=1e-6, B=2, H=3, d=64, h=256, b=16, pos=0, z=z)
+        a.update(kw)
+        return lib.ttt_mlp_decode(a["q"], a["k"], a["v"], a["dt"], a["eta"], a["w1"], a["w2"], a["w1b"],
+                                  a["w2b"], a["g"], a["bt"], a["eps"], a["B"], a["H"], a["d"], a["h"],
+                                  a["b"], a["pos"], a["z"], None)
+
+    assert call(pos=16) == L.TTT_ERR_ARG
+    assert call(h=0) == L.TTT_ERR_ARG
+    assert call(h=128) == L.TTT_ERR_UNSUPPORTED
+    assert call(d=32) == L.TTT_ERR_UNSUPPORTED
+    assert call(eps=-1.0) == L.TTT_ERR_ARG
+    assert call(w2b=None) == L.TTT_ERR_ARG
+    assert call(w1=A + 4) == L.TTT_ERR_ALIGN
+    assert call(w2b=w1b + 4096) == L.TTT_ERR_ARG      # the two bases overlap
+    assert call(B=0) == L.TTT_OK
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"

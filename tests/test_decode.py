@@ -60,3 +60,28 @@ def test_decode_mid_mini_batch_keeps_base():
     assert torch.equal(W_base, W0)
     assert not torch.equal(W, W0)
     assert ttt.last_device_status() == 0
+
+
+def decode_sequence_mlp(cfg, dev):
+    B, H, T, d, h = cfg.B, cfg.H, cfg.T, cfg.d, cfg.hidden
+    W1 = dev["W1"].unsqueeze(0).expand(B, H, d, h).contiguous()
+    W2 = dev["W2"].unsqueeze(0).expand(B, H, h, d).contiguous()
+    W1b, W2b = W1.clone(), W2.clone()
+    Z = torch.empty(B, H, T, d, dtype=torch.float32, device="cuda")
+    for t in range(T):
+        q, k, v = (dev[n][:, :, t].contiguous() for n in ("Q", "K", "V"))
+        Z[:, :, t] = ttt.ttt_mlp_decode(q, k, v, dev["eta"][:, :, t].contiguous(), W1, W2, W1b, W2b,
+                                        dev["gamma"], dev["beta"], cfg.b, t % cfg.b, cfg.ln_eps)
+    torch.cuda.synchronize()
+    return {"Z": Z.cpu().numpy(), "W1": W1.cpu().numpy(), "W2": W2.cpu().numpy()}, (W1b, W2b)
+
+
+@pytest.mark.parametrize("b", [1, 16])
+def test_mlp_decode_matches_oracle(b):
+    cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=2, H=3, T=32, b=b)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    out, (W1b, W2b) = decode_sequence_mlp(cfg, dev)
+    worst = compare(cfg, out, all_units(cfg))
+    assert max(worst.values()) <= DECODE_TOL, worst
+    assert torch.equal(W1b.cpu(), torch.from_numpy(out["W1"]))
+    assert torch.equal(W2b.cpu(), torch.from_numpy(out["W2"]))
