@@ -60,6 +60,10 @@ def load(path: str | None = None):
     lib.oracle_apply_f64.argtypes = [ctypes.c_int, _dp, _dp, ctypes.c_int, ctypes.c_int, _dp, _dp,
                                      ctypes.c_double, _dp]
     lib.oracle_default_threads.restype = ctypes.c_int
+    lib.oracle_ttt_momentum_forward_f64.restype = ctypes.c_int
+    lib.oracle_ttt_momentum_forward_f64.argtypes = [
+        ctypes.c_int, _dp, _dp, _dp, _dp, _dp, _dp, _dp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, _dp, _dp, ctypes.c_double, _dp, _dp, _dp]
     if path is None:
         _lib_handle = lib
     return lib
@@ -124,6 +128,26 @@ class Oracle:
                             nthreads=nthreads)
         Bn = W.shape[0]
         return Z, W[:, :, : d * h].reshape(Bn, H, d, h), W[:, :, d * h:].reshape(Bn, H, h, d)
+
+    def momentum_forward(self, kind, Q, K, V, eta, alpha, lam, params, b, gamma=None, beta=None,
+                         eps=1e-6, hidden=0):
+        """The momentum and decay variant (Titans-style): S_t = alpha_t S_{t-1} - eta_t grad,
+        W_t = (1 - lambda_t) W_{t-1} + S_t, gradients at the mini-batch base.
+        Returns (Z [B,H,T,d], W_out [B,H,P], S_out [B,H,P])."""
+        Q, K, V, eta, alpha, lam, params = map(_f64, (Q, K, V, eta, alpha, lam, params))
+        gamma, beta = _f64(gamma), _f64(beta)
+        B, H, T, d = Q.shape
+        P = params.shape[-1]
+        Z = np.zeros((B, H, T, d))
+        W_out = np.zeros((B, H, P))
+        S_out = np.zeros((B, H, P))
+        rc = self.lib.oracle_ttt_momentum_forward_f64(
+            int(kind), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(params),
+            B, H, T, d, int(hidden), int(b), _ptr(gamma), _ptr(beta), float(eps), _ptr(Z),
+            _ptr(W_out), _ptr(S_out))
+        if rc != 0:
+            raise ValueError(f"oracle_ttt_momentum_forward_f64 failed with status {rc}")
+        return Z, W_out, S_out
 
     def loss_grad(self, kind, params, k, v, gamma=None, beta=None, eps=1e-6, hidden=0):
         """Loss ||f(k; W) - v||^2 of one head and its gradient (flat, like params)."""

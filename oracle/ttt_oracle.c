@@ -263,6 +263,87 @@ static int run_sequence(const model_t *m, const double *Q, const double *K, cons
   return 0;
 }
 
+/* --- momentum and decay variant (Titans-style memory update) ------------- */
+
+/* The Titans article (page 4 of the sources, §二.1(2)) adds to the gradient
+ * ("surprise") step a momentum on past surprise and a weight decay that forgets.
+ * Plainest reading, kept to TTT's mini-batch rule (§03.6; the article calls the
+ * update equivalent to mini-batch gradient descent with momentum and weight
+ * decay): with S_0 = 0 and t' the base of token t's mini-batch,
+ *   S_t = alpha_t S_{t-1} - eta_t grad l(W_{t'}; x_t)
+ *   W_t = (1 - lambda_t) W_{t-1} + S_t,     z_t = f(q_t; W_t).
+ * alpha = lambda = 0 is TTT itself. */
+static int run_sequence_momentum(const model_t *m, const double *Q, const double *K,
+                                 const double *V, const double *eta, const double *alpha,
+                                 const double *lam, const double *W0, int T, int b, double *Z,
+                                 double *Wout, double *Sout) {
+  const int d = m->d;
+  const long P = param_count(m);
+  double *W = (double *)malloc(sizeof(double) * P);
+  double *Wbase = (double *)malloc(sizeof(double) * P);
+  double *S = (double *)calloc((size_t)P, sizeof(double));
+  double *grad = (double *)malloc(sizeof(double) * P);
+  scratch_t sc;
+  if (!W || !Wbase || !S || !grad || scratch_init(&sc, m) != 0) {
+    free(W);
+    free(Wbase);
+    free(S);
+    free(grad);
+    return -2;
+  }
+  memcpy(W, W0, sizeof(double) * P);
+  for (int t = 0; t < T; ++t) {
+    if (t % b == 0) memcpy(Wbase, W, sizeof(double) * P);
+    const double *k = K + (long)t * d, *v = V + (long)t * d, *q = Q + (long)t * d;
+    model_loss_grad(m, Wbase, k, v, grad, &sc);
+    for (long p = 0; p < P; ++p) {
+      S[p] = alpha[t] * S[p] - eta[t] * grad[p];
+      W[p] = (1.0 - lam[t]) * W[p] + S[p];
+    }
+    model_apply(m, W, q, Z + (long)t * d, &sc);
+  }
+  memcpy(Wout, W, sizeof(double) * P);
+  memcpy(Sout, S, sizeof(double) * P);
+  scratch_free(&sc);
+  free(W);
+  free(Wbase);
+  free(S);
+  free(grad);
+  return 0;
+}
+
+/* One thread over every unit (the variant is checked at small sizes only).
+ * alpha, lam: [B][H][T] like eta; S_out: [B][H][P], the final momentum.
+ * Returns 0, -1 on a bad argument, -2 on allocation failure. */
+int oracle_ttt_momentum_forward_f64(int kind, const double *Q, const double *K, const double *V,
+                                    const double *eta, const double *alpha, const double *lam,
+                                    const double *W0, int B, int H, int T, int d, int hidden,
+                                    int b, const double *gamma, const double *beta, double eps,
+                                    double *Z, double *Wout, double *Sout) {
+  if (kind < ORACLE_LINEAR || kind > ORACLE_MLP_LN) return -1;
+  if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0 || T % b != 0) return -1;
+  if (kind == ORACLE_MLP_LN && hidden <= 0) return -1;
+  if (kind != ORACLE_LINEAR && (!gamma || !beta || !(eps > 0.0))) return -1;
+  if ((long)B * H == 0) return 0;
+  if (!W0 || !Wout || !Sout || (T > 0 && (!Q || !K || !V || !eta || !alpha || !lam || !Z)))
+    return -1;
+  model_t m = {kind, d, hidden, NULL, NULL, eps};
+  const long P = param_count(&m);
+  for (long u = 0; u < (long)B * H; ++u) {
+    const int hh = (int)(u % H);
+    const long tok = u * (long)T;
+    if (kind != ORACLE_LINEAR) {
+      m.gamma = gamma + (long)hh * d;
+      m.beta = beta + (long)hh * d;
+    }
+    const int rc = run_sequence_momentum(&m, Q + tok * d, K + tok * d, V + tok * d, eta + tok,
+                                         alpha + tok, lam + tok, W0 + (long)hh * P, T, b,
+                                         Z + tok * d, Wout + u * P, Sout + u * P);
+    if (rc != 0) return rc;
+  }
+  return 0;
+}
+
 /* --- multithreaded driver over (batch, head) units ------------------------- */
 
 typedef struct {
