@@ -275,9 +275,11 @@ def main():
                          "instead of the forward")
     ap.add_argument("--decode-mlp", action="store_true",
                     help="the same for the TTT-MLP decode step")
+    ap.add_argument("--decode-momentum", action="store_true",
+                    help="the same for the TTT-Linear + LN decode step with the momentum and decay update")
     args = ap.parse_args()
-    if args.decode or args.decode_mlp:
-        return run_decode(args, mlp=args.decode_mlp)
+    if args.decode or args.decode_mlp or args.decode_momentum:
+        return run_decode(args, mlp=args.decode_mlp, momentum=args.decode_momentum)
     cfg = I.CONFIGS[args.workload]
     if args.batch is not None or args.seq is not None:
         cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T,
@@ -387,9 +389,10 @@ def main():
                   e2e, peaks, peak_kind, nbytes, nflops, dist)
 
 
-def run_decode(args, mlp=False):
+def run_decode(args, mlp=False, momentum=False):
     """The decode step's own line: one timed step = one mini-batch of 16 decode calls
-    (positions 0..15) over B=512 x H=32 (batch, head) units, the state in HBM."""
+    (positions 0..15) over B=512 x H=32 (batch, head) units, the state in HBM.
+    ``momentum``: the TTT-Linear + LN step with the momentum and decay update."""
     import torch
     import test_sequence_modeling_b200 as ttt
     from test_sequence_modeling_b200 import _lib
@@ -398,7 +401,8 @@ def run_decode(args, mlp=False):
     if mlp:
         cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=512, T=16, name="decode_mlp_B512H32")
     else:
-        cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=512, T=16, name="decode_linear_ln_B512H32")
+        name = "decode_momentum_linear_ln_B512H32" if momentum else "decode_linear_ln_B512H32"
+        cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=512, T=16, name=name)
     data = I.make_inputs(cfg)
     B, H, T, d = cfg.B, cfg.H, cfg.T, cfg.d
     qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
@@ -415,6 +419,11 @@ def run_decode(args, mlp=False):
     else:
         W = torch.from_numpy(data["W0"]).to(dev).unsqueeze(0).expand(B, H, d, d).contiguous()
         W_base = W.clone()
+        if momentum:
+            S = torch.zeros_like(W)
+            alpha, lam = (torch.from_numpy(x).to(dev) for x in I.momentum_rates(cfg))
+            als = [alpha[:, :, t].contiguous() for t in range(T)]
+            lms = [lam[:, :, t].contiguous() for t in range(T)]
     z = torch.empty(B, H, d, device=dev)
     stream = torch.cuda.current_stream(dev)
     lib = _lib.load()
@@ -424,6 +433,10 @@ def run_decode(args, mlp=False):
             if mlp:
                 ttt.ttt_mlp_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], W1, W2, W1b, W2b, gamma,
                                    beta, cfg.b, t, cfg.ln_eps, z=z, stream=stream)
+            elif momentum:
+                ttt.ttt_linear_ln_momentum_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], als[t],
+                                                  lms[t], W, W_base, S, gamma, beta, cfg.b, t, cfg.ln_eps,
+                                                  z=z, stream=stream)
             else:
                 ttt.ttt_linear_ln_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], W, W_base, gamma,
                                          beta, cfg.b, t, cfg.ln_eps, z=z, stream=stream)
@@ -451,13 +464,16 @@ def run_decode(args, mlp=False):
     # written each call, W_base written once, q/k/v (bf16), eta and z per call.
     if mlp:  # W1b, W2b, W1, W2 read and W1, W2 written per call; the bases written once
         per_unit = T * (6 * d * cfg.hidden * 4 + 3 * d * 2 + 4 + d * 4) + 2 * d * cfg.hidden * 4
+    elif momentum:  # W_base, W, S read and W, S written per call, plus alpha and lambda
+        per_unit = T * (5 * d * d * 4 + 3 * d * 2 + 3 * 4 + d * 4) + d * d * 4
     else:
         per_unit = T * (3 * d * d * 4 + 3 * d * 2 + 4 + d * 4) + d * d * 4
     nbytes = units * per_unit
     peaks, peak_kind = load_peaks()
     achieved = nbytes / (ms / args.steps / 1e3) / 1e9
     line = {
-        "metric": ("TTT-MLP" if mlp else "TTT-Linear+LN") + " decode step tokens/s (B x H units, one token each per call)",
+        "metric": ("TTT-MLP" if mlp else "TTT-Linear+LN" + (" momentum/decay" if momentum else ""))
+        + " decode step tokens/s (B x H units, one token each per call)",
         "value": value, "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",

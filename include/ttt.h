@@ -144,6 +144,30 @@ TTT_API int ttt_linear_ln_decode(const void *q, const void *k, const void *v, in
                                  int pos, float *z, void *stream);
 
 /*
+ * The decode step with the momentum and decay update of the Titans article
+ * (§二.1(2): momentum on past surprise, weight decay that forgets), kept to the
+ * TTT mini-batch base above.  Besides the arguments of the plain step:
+ *   alpha   [B][H] fp32: this token's momentum factor (0 <= alpha < 1 in use).
+ *   lambda  [B][H] fp32: this token's weight decay (0 <= lambda <= 1 in use).
+ *   S       [B][H][d][d] fp32, in/out: the momentum, all zero before the first token.
+ * Per (batch, head), with G at W_base as above:
+ *   S <- alpha S - eta k^T G,   W <- (1 - lambda) W + S,   z = q W (or q + LN(q W)),
+ *   and W_base <- W if pos == b-1.
+ * alpha = lambda = 0 is the plain step.  The caller owns all buffers; W, W_base,
+ * S and z must not overlap each other or the inputs.  Errors as for the plain step.
+ */
+TTT_API int ttt_linear_momentum_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                                       const float *eta, const float *alpha, const float *lambda,
+                                       float *W, float *W_base, float *S, int B, int H, int d,
+                                       int b, int pos, float *z, void *stream);
+TTT_API int ttt_linear_ln_momentum_decode(const void *q, const void *k, const void *v,
+                                          int qkv_dtype, const float *eta, const float *alpha,
+                                          const float *lambda, float *W, float *W_base, float *S,
+                                          const float *ln_gamma, const float *ln_beta,
+                                          float ln_eps, int B, int H, int d, int b, int pos,
+                                          float *z, void *stream);
+
+/*
  * The same step for TTT-MLP, f(x) = x + LN(GELU(x W1) W2): the state is W1
  * [B][H][d][hidden] and W2 [B][H][hidden][d] (fp32, in/out) with their
  * mini-batch bases W1_base, W2_base (in/out); hidden = 4 d.  Per (batch, head),

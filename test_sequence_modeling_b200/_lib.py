@@ -28,6 +28,10 @@ SIGNATURES = {
     "ttt_linear_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _i, _i, _i, _i, _i, _fp, _vp]),
     "ttt_linear_ln_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i, _i, _i,
                                   _fp, _vp]),
+    "ttt_linear_momentum_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _i, _i, _i,
+                                        _i, _i, _fp, _vp]),
+    "ttt_linear_ln_momentum_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp,
+                                           _f, _i, _i, _i, _i, _i, _fp, _vp]),
     "ttt_mlp_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i, _i,
                             _i, _i, _fp, _vp]),
 }

@@ -13,6 +13,12 @@
 //                              starts from the state this one ends in)
 // Per (batch, head) a call reads W_base and W (32 KB) and writes W (16 KB, and
 // W_base once per mini-batch): HBM-bound, 48 KB against ~16 kFLOP.
+//
+// The momentum and decay variant of the linear kernels (the Titans article's
+// memory update, §二.1(2), kept to the mini-batch base above) carries a third
+// state S, zero at the start:
+//   S <- alpha S - eta k^T G,   W <- (1 - lambda) W + S
+// and otherwise runs the same call: 80 KB per (batch, head) and call.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -34,9 +40,13 @@ struct Params {
   float eps;
   int H, pos, b;
   float *z;               // [units][D]
+  // Momentum and decay variant (Titans-style memory update) when S != nullptr:
+  //   S <- alpha S - eta k^T G,  W <- (1 - lambda) W + S   (S [units][D][D], in place)
+  const float *alpha, *lambda;  // [units]
+  float *S;
 };
 
-template <bool LN, typename InT>
+template <bool LN, typename InT, bool MOMENTUM = false>
 __global__ void __launch_bounds__(THREADS) decode_kernel(const Params p) {
   __shared__ float qs[D], ks[D], vs[D], part[4][D], g[D];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -52,11 +62,13 @@ __global__ void __launch_bounds__(THREADS) decode_kernel(const Params p) {
   float *Wb = p.W_base + unit * D * D;
   // Both state rows of this thread are read up front (one coalesced 128-byte
   // line per warp and row).
-  float wb[16], w[16];
+  float wb[16], w[16], sm_[MOMENTUM ? 16 : 1];
+  float *Su = MOMENTUM ? p.S + unit * D * D : nullptr;
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     wb[r] = Wb[(16 * rq + r) * D + j];
     w[r] = Wu[(16 * rq + r) * D + j];
+    if (MOMENTUM) sm_[r] = Su[(16 * rq + r) * D + j];
   }
   __syncthreads();
 
@@ -84,14 +96,23 @@ __global__ void __launch_bounds__(THREADS) decode_kernel(const Params p) {
   }
   __syncthreads();
 
-  // W -= k^T (eta G); z = q W with the updated state.
+  // W -= k^T (eta G) (or the momentum and decay update); z = q W with the
+  // updated state.
   const float gj = g[j];
   const bool last = p.pos == p.b - 1;
+  const float al = MOMENTUM ? p.alpha[unit] : 0.f;
+  const float keep = MOMENTUM ? 1.f - p.lambda[unit] : 1.f;
   float zacc = 0.f;
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     const int i = 16 * rq + r;
-    w[r] = fmaf(-ks[i], gj, w[r]);
+    if (MOMENTUM) {
+      sm_[r] = fmaf(al, sm_[r], -ks[i] * gj);
+      w[r] = fmaf(keep, w[r], sm_[r]);
+      Su[i * D + j] = sm_[r];
+    } else {
+      w[r] = fmaf(-ks[i], gj, w[r]);
+    }
     zacc = fmaf(qs[i], w[r], zacc);
     Wu[i * D + j] = w[r];
     if (last) Wb[i * D + j] = w[r];

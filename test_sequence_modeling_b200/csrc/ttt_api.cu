@@ -234,7 +234,8 @@ int launch_linear_tc(const Call &c) {
 // forward entry points do.
 int run_decode(bool ln, const void *q, const void *k, const void *v, int qkv_dtype, const float *eta,
                float *W, float *W_base, const float *gamma, const float *beta, float eps, int B,
-               int H, int d, int b, int pos, float *z, void *stream) {
+               int H, int d, int b, int pos, float *z, void *stream, bool momentum = false,
+               const float *alpha = nullptr, const float *lambda = nullptr, float *S = nullptr) {
   if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
   if (B < 0 || H < 0 || d <= 0 || b <= 0 || pos < 0 || pos >= b) return TTT_ERR_ARG;
   if (ln && !(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
@@ -243,29 +244,41 @@ int run_decode(bool ln, const void *q, const void *k, const void *v, int qkv_dty
   if (units == 0) return TTT_OK;
   if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
   const void *req[] = {q, k, v, eta, W, W_base, z, ln ? (const void *)gamma : q,
-                       ln ? (const void *)beta : q};
+                       ln ? (const void *)beta : q, momentum ? (const void *)alpha : q,
+                       momentum ? (const void *)lambda : q, momentum ? (const void *)S : q};
   for (const void *x : req)
     if (!x) return TTT_ERR_ARG;
   for (const void *x : req)
     if (!aligned16(x)) return TTT_ERR_ALIGN;
   const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
-  Range ins[6] = {range_of(q, units * d * in_elt), range_of(k, units * d * in_elt),
+  Range ins[8] = {range_of(q, units * d * in_elt), range_of(k, units * d * in_elt),
                   range_of(v, units * d * in_elt), range_of(eta, units * 4),
                   range_of(ln ? (const void *)gamma : q, ln ? (size_t)H * d * 4 : 0),
-                  range_of(ln ? (const void *)beta : q, ln ? (size_t)H * d * 4 : 0)};
-  Range outs[3] = {range_of(W, units * d * d * 4), range_of(W_base, units * d * d * 4),
-                   range_of(z, units * d * 4)};
-  for (int o = 0; o < 3; ++o) {
-    for (int i = 0; i < 6; ++i)
+                  range_of(ln ? (const void *)beta : q, ln ? (size_t)H * d * 4 : 0),
+                  range_of(momentum ? (const void *)alpha : q, momentum ? units * 4 : 0),
+                  range_of(momentum ? (const void *)lambda : q, momentum ? units * 4 : 0)};
+  Range outs[4] = {range_of(W, units * d * d * 4), range_of(W_base, units * d * d * 4),
+                   range_of(z, units * d * 4),
+                   range_of(momentum ? (const void *)S : z, momentum ? units * d * d * 4 : 0)};
+  for (int o = 0; o < 4; ++o) {
+    for (int i = 0; i < 8; ++i)
       if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
-    for (int o2 = o + 1; o2 < 3; ++o2)
+    for (int o2 = o + 1; o2 < 4; ++o2)
       if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
   }
-  decode::Params p{q, k, v, eta, W, W_base, gamma, beta, eps, H, pos, b, z};
+  decode::Params p{q, k, v, eta, W, W_base, gamma, beta, eps, H, pos, b, z, alpha, lambda, S};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bf16 = qkv_dtype == TTT_BF16;
   const unsigned grid = (unsigned)units;
-  if (ln) {
+  if (momentum) {
+    if (ln) {
+      if (bf16) decode::decode_kernel<true, __nv_bfloat16, true><<<grid, decode::THREADS, 0, s>>>(p);
+      else decode::decode_kernel<true, float, true><<<grid, decode::THREADS, 0, s>>>(p);
+    } else {
+      if (bf16) decode::decode_kernel<false, __nv_bfloat16, true><<<grid, decode::THREADS, 0, s>>>(p);
+      else decode::decode_kernel<false, float, true><<<grid, decode::THREADS, 0, s>>>(p);
+    }
+  } else if (ln) {
     if (bf16) decode::decode_kernel<true, __nv_bfloat16><<<grid, decode::THREADS, 0, s>>>(p);
     else decode::decode_kernel<true, float><<<grid, decode::THREADS, 0, s>>>(p);
   } else {
@@ -393,6 +406,23 @@ int ttt_linear_decode(const void *q, const void *k, const void *v, int qkv_dtype
                       void *stream) {
   return run_decode(false, q, k, v, qkv_dtype, eta, W, W_base, nullptr, nullptr, 1.f, B, H, d, b,
                     pos, z, stream);
+}
+
+int ttt_linear_momentum_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                               const float *eta, const float *alpha, const float *lambda, float *W,
+                               float *W_base, float *S, int B, int H, int d, int b, int pos, float *z,
+                               void *stream) {
+  return run_decode(false, q, k, v, qkv_dtype, eta, W, W_base, nullptr, nullptr, 1.f, B, H, d, b,
+                    pos, z, stream, true, alpha, lambda, S);
+}
+
+int ttt_linear_ln_momentum_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                                  const float *eta, const float *alpha, const float *lambda,
+                                  float *W, float *W_base, float *S, const float *ln_gamma,
+                                  const float *ln_beta, float ln_eps, int B, int H, int d, int b,
+                                  int pos, float *z, void *stream) {
+  return run_decode(true, q, k, v, qkv_dtype, eta, W, W_base, ln_gamma, ln_beta, ln_eps, B, H, d, b,
+                    pos, z, stream, true, alpha, lambda, S);
 }
 
 int ttt_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype, const float *eta,

@@ -164,6 +164,15 @@ def make_inputs(cfg: TTTConfig, threads: int = 8, bf16_as_bits: bool = True,
     return out
 
 
+def momentum_rates(cfg: TTTConfig, seed: int = 0):
+    """Per-token momentum factors alpha in [0, 0.9) and weight decays lambda in
+    [0, 0.05), [B, H, T] float32 each, for the momentum and decay update."""
+    rng = np.random.default_rng([cfg.seed, 3, seed])
+    alpha = (0.9 * rng.random((cfg.B, cfg.H, cfg.T))).astype(np.float32)
+    lam = (0.05 * rng.random((cfg.B, cfg.H, cfg.T))).astype(np.float32)
+    return alpha, lam
+
+
 def unit_as_f64(cfg: TTTConfig, bi: int, hi: int, T: int | None = None) -> dict:
     """One unit's inputs and its head's parameters in float64, shaped [1,1,T,d] and
     [1,...] for feeding a per-unit reference computation."""

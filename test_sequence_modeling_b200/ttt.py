@@ -155,6 +155,46 @@ def ttt_linear_ln_decode(q, k, v, eta, W, W_base, gamma, beta, b, pos, eps=1e-6,
     return z
 
 
+def _momentum_args(B, H, d, alpha, lam, S):
+    for n, t in (("alpha", alpha), ("lam", lam)):
+        _cuda(t, n, torch.float32)
+        if tuple(t.shape) != (B, H):
+            raise ValueError(f"{n} must have shape {(B, H)}")
+    _cuda(S, "S", torch.float32)
+    if tuple(S.shape) != (B, H, d, d):
+        raise ValueError(f"S must have shape {(B, H, d, d)}")
+
+
+def ttt_linear_momentum_decode(q, k, v, eta, alpha, lam, W, W_base, S, b, pos, z=None, stream=None):
+    """One decode step of TTT-Linear with the momentum and decay update (see
+    include/ttt.h): alpha, lam [B,H] f32; W, W_base and the momentum S [B,H,d,d] f32
+    are updated in place (S starts at zero).  Returns z [B,H,d] f32."""
+    dt, B, H, d, z = _decode_args(q, k, v, eta, W, W_base, z)
+    _momentum_args(B, H, d, alpha, lam, S)
+    with torch.cuda.device(q.device):
+        st = _lib.load().ttt_linear_momentum_decode(
+            _ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(W), _ptr(W_base),
+            _ptr(S), B, H, d, int(b), int(pos), _ptr(z), _stream(stream, q.device))
+    check(st, "ttt_linear_momentum_decode")
+    return z
+
+
+def ttt_linear_ln_momentum_decode(q, k, v, eta, alpha, lam, W, W_base, S, gamma, beta, b, pos, eps=1e-6,
+                                  z=None, stream=None):
+    """The momentum and decay decode step of TTT-Linear with LN + residual."""
+    dt, B, H, d, z = _decode_args(q, k, v, eta, W, W_base, z)
+    _momentum_args(B, H, d, alpha, lam, S)
+    for n, t in (("gamma", gamma), ("beta", beta)):
+        _cuda(t, n, torch.float32)
+    with torch.cuda.device(q.device):
+        st = _lib.load().ttt_linear_ln_momentum_decode(
+            _ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(W), _ptr(W_base),
+            _ptr(S), _ptr(gamma), _ptr(beta), float(eps), B, H, d, int(b), int(pos), _ptr(z),
+            _stream(stream, q.device))
+    check(st, "ttt_linear_ln_momentum_decode")
+    return z
+
+
 def ttt_mlp_decode(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, b, pos, eps=1e-6, z=None,
                    stream=None):
     """One primal-form decode step of TTT-MLP.  W1, W1_base [B,H,d,hidden] and W2, W2_base

@@ -154,6 +154,38 @@ def test_decode_argument_errors(lib, ln):
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
 
 
+def momentum(lib, ln=False, **kw):
+    q, k, v, eta, al, lm, w, wb, s, z, g, bt = _ptrs(12)
+    a = dict(q=q, k=k, v=v, dt=L.TTT_BF16, eta=eta, al=al, lm=lm, W=w, Wb=wb, S=s, g=g, bt=bt,
+             eps=1e-6, B=2, H=3, d=64, b=16, pos=0, z=z)
+    a.update(kw)
+    head = (a["q"], a["k"], a["v"], a["dt"], a["eta"], a["al"], a["lm"], a["W"], a["Wb"], a["S"])
+    tail = (a["B"], a["H"], a["d"], a["b"], a["pos"], a["z"], None)
+    if ln:
+        return lib.ttt_linear_ln_momentum_decode(*head, a["g"], a["bt"], a["eps"], *tail)
+    return lib.ttt_linear_momentum_decode(*head, *tail)
+
+
+@pytest.mark.parametrize("ln", [False, True])
+def test_momentum_decode_argument_errors(lib, ln):
+    n0 = lib.ttt_launch_count()
+    assert momentum(lib, ln, pos=16) == L.TTT_ERR_ARG
+    assert momentum(lib, ln, d=32) == L.TTT_ERR_UNSUPPORTED
+    assert momentum(lib, ln, al=None) == L.TTT_ERR_ARG
+    assert momentum(lib, ln, lm=None) == L.TTT_ERR_ARG
+    assert momentum(lib, ln, S=None) == L.TTT_ERR_ARG
+    assert momentum(lib, ln, S=A + 8) == L.TTT_ERR_ALIGN
+    assert momentum(lib, ln, al=A + 4) == L.TTT_ERR_ALIGN
+    w, s = _ptrs(12)[6], _ptrs(12)[8]
+    assert momentum(lib, ln, S=w + 1024) == L.TTT_ERR_ARG    # S overlaps W
+    assert momentum(lib, ln, W=s + 4096) == L.TTT_ERR_ARG    # W overlaps S
+    assert momentum(lib, ln, lm=s + 64) == L.TTT_ERR_ARG     # lambda inside S
+    assert momentum(lib, ln, B=0) == L.TTT_OK
+    if ln:
+        assert momentum(lib, ln, g=None) == L.TTT_ERR_ARG
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
+
+
 def test_mlp_decode_argument_errors(lib):
     n0 = lib.ttt_launch_count()
     q, k, v, eta, w1, w2, w1b, w2b, z, g, bt = _ptrs(11)
