@@ -276,7 +276,8 @@ def main():
     ap.add_argument("--decode-mlp", action="store_true",
                     help="the same for the TTT-MLP decode step")
     ap.add_argument("--decode-momentum", action="store_true",
-                    help="the same for the TTT-Linear + LN decode step with the momentum and decay update")
+                    help="the decode step with the momentum and decay update (TTT-Linear + LN, or with "
+                         "--decode-mlp TTT-MLP)")
     args = ap.parse_args()
     if args.decode or args.decode_mlp or args.decode_momentum:
         return run_decode(args, mlp=args.decode_mlp, momentum=args.decode_momentum)
@@ -392,14 +393,15 @@ def main():
 def run_decode(args, mlp=False, momentum=False):
     """The decode step's own line: one timed step = one mini-batch of 16 decode calls
     (positions 0..15) over B=512 x H=32 (batch, head) units, the state in HBM.
-    ``momentum``: the TTT-Linear + LN step with the momentum and decay update."""
+    ``momentum``: the step with the momentum and decay update."""
     import torch
     import test_sequence_modeling_b200 as ttt
     from test_sequence_modeling_b200 import _lib
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     if mlp:
-        cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=512, T=16, name="decode_mlp_B512H32")
+        name = "decode_momentum_mlp_B512H32" if momentum else "decode_mlp_B512H32"
+        cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=512, T=16, name=name)
     else:
         name = "decode_momentum_linear_ln_B512H32" if momentum else "decode_linear_ln_B512H32"
         cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=512, T=16, name=name)
@@ -416,21 +418,28 @@ def run_decode(args, mlp=False, momentum=False):
         W1 = torch.from_numpy(data["W1"]).to(dev).unsqueeze(0).expand(B, H, d, h).contiguous()
         W2 = torch.from_numpy(data["W2"]).to(dev).unsqueeze(0).expand(B, H, h, d).contiguous()
         W1b, W2b = W1.clone(), W2.clone()
+        if momentum:
+            S1, S2 = torch.zeros_like(W1), torch.zeros_like(W2)
     else:
         W = torch.from_numpy(data["W0"]).to(dev).unsqueeze(0).expand(B, H, d, d).contiguous()
         W_base = W.clone()
         if momentum:
             S = torch.zeros_like(W)
-            alpha, lam = (torch.from_numpy(x).to(dev) for x in I.momentum_rates(cfg))
-            als = [alpha[:, :, t].contiguous() for t in range(T)]
-            lms = [lam[:, :, t].contiguous() for t in range(T)]
+    if momentum:
+        alpha, lam = (torch.from_numpy(x).to(dev) for x in I.momentum_rates(cfg))
+        als = [alpha[:, :, t].contiguous() for t in range(T)]
+        lms = [lam[:, :, t].contiguous() for t in range(T)]
     z = torch.empty(B, H, d, device=dev)
     stream = torch.cuda.current_stream(dev)
     lib = _lib.load()
 
     def step():
         for t in range(T):
-            if mlp:
+            if mlp and momentum:
+                ttt.ttt_mlp_momentum_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], als[t], lms[t],
+                                            W1, W2, W1b, W2b, S1, S2, gamma, beta, cfg.b, t, cfg.ln_eps,
+                                            z=z, stream=stream)
+            elif mlp:
                 ttt.ttt_mlp_decode(tok[t]["Q"], tok[t]["K"], tok[t]["V"], etas[t], W1, W2, W1b, W2b, gamma,
                                    beta, cfg.b, t, cfg.ln_eps, z=z, stream=stream)
             elif momentum:
@@ -462,7 +471,9 @@ def run_decode(args, mlp=False, momentum=False):
     value = units * T * args.steps / (ms / 1e3)
     # Algorithmic bytes per mini-batch (16 calls) and unit: W_base and W read and W
     # written each call, W_base written once, q/k/v (bf16), eta and z per call.
-    if mlp:  # W1b, W2b, W1, W2 read and W1, W2 written per call; the bases written once
+    if mlp and momentum:  # W1b, W2b, W1, W2, S1, S2 read, W1, W2, S1, S2 written per call
+        per_unit = T * (10 * d * cfg.hidden * 4 + 3 * d * 2 + 3 * 4 + d * 4) + 2 * d * cfg.hidden * 4
+    elif mlp:  # W1b, W2b, W1, W2 read and W1, W2 written per call; the bases written once
         per_unit = T * (6 * d * cfg.hidden * 4 + 3 * d * 2 + 4 + d * 4) + 2 * d * cfg.hidden * 4
     elif momentum:  # W_base, W, S read and W, S written per call, plus alpha and lambda
         per_unit = T * (5 * d * d * 4 + 3 * d * 2 + 3 * 4 + d * 4) + d * d * 4
@@ -472,7 +483,7 @@ def run_decode(args, mlp=False, momentum=False):
     peaks, peak_kind = load_peaks()
     achieved = nbytes / (ms / args.steps / 1e3) / 1e9
     line = {
-        "metric": ("TTT-MLP" if mlp else "TTT-Linear+LN" + (" momentum/decay" if momentum else ""))
+        "metric": ("TTT-MLP" if mlp else "TTT-Linear+LN") + (" momentum/decay" if momentum else "")
         + " decode step tokens/s (B x H units, one token each per call)",
         "value": value, "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,

@@ -180,6 +180,25 @@ TTT_API int ttt_mlp_decode(const void *q, const void *k, const void *v, int qkv_
                            const float *ln_gamma, const float *ln_beta, float ln_eps, int B, int H,
                            int d, int hidden, int b, int pos, float *z, void *stream);
 
+/*
+ * The TTT-MLP decode step with the momentum and decay update (the Titans
+ * article's MLP memory, §二.1(2); the same reading as the linear momentum step):
+ * S1 [B][H][d][hidden] and S2 [B][H][hidden][d] fp32 (in/out, zero before the
+ * first token) are the momenta of W1 and W2; alpha, lambda [B][H] fp32.  Per
+ * (batch, head), with G2, G3 at the bases as in ttt_mlp_decode:
+ *   S1 <- alpha S1 - eta k^T G2,   W1 <- (1 - lambda) W1 + S1,
+ *   S2 <- alpha S2 - eta X2^T G3,  W2 <- (1 - lambda) W2 + S2,
+ *   z = q + LN(GELU(q W1) W2), and both bases follow at pos == b - 1.
+ * The caller owns all buffers; the seven state and output buffers must not
+ * overlap each other or the inputs.  Errors as for ttt_mlp_decode.
+ */
+TTT_API int ttt_mlp_momentum_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                                    const float *eta, const float *alpha, const float *lambda,
+                                    float *W1, float *W2, float *W1_base, float *W2_base, float *S1,
+                                    float *S2, const float *ln_gamma, const float *ln_beta,
+                                    float ln_eps, int B, int H, int d, int hidden, int b, int pos,
+                                    float *z, void *stream);
+
 /* Static English text for a ttt_status value (never NULL). */
 TTT_API const char *ttt_status_string(int status);
 

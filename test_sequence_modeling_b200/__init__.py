@@ -14,7 +14,8 @@ def __getattr__(name):
     if name in ("ttt_linear_fwd", "ttt_linear_ln_fwd", "ttt_mlp_fwd", "set_path",
                 "last_device_status", "launch_count", "debug_inject_timeout",
                 "ttt_linear_decode", "ttt_linear_ln_decode", "ttt_mlp_decode",
-                "ttt_linear_momentum_decode", "ttt_linear_ln_momentum_decode"):
+                "ttt_linear_momentum_decode", "ttt_linear_ln_momentum_decode",
+                "ttt_mlp_momentum_decode"):
         from . import ttt
         return getattr(ttt, name)
     raise AttributeError(name)

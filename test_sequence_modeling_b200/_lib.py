@@ -32,6 +32,8 @@ SIGNATURES = {
                                         _i, _i, _fp, _vp]),
     "ttt_linear_ln_momentum_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp,
                                            _f, _i, _i, _i, _i, _i, _fp, _vp]),
+    "ttt_mlp_momentum_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp,
+                                     _fp, _fp, _f, _i, _i, _i, _i, _i, _i, _fp, _vp]),
     "ttt_mlp_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i, _i,
                             _i, _i, _fp, _vp]),
 }

@@ -141,6 +141,11 @@ __global__ void __launch_bounds__(THREADS) decode_kernel(const Params p) {
 // Per (batch, head) a call reads the four matrices (256 KB) and writes W1, W2
 // (128 KB, and the bases once per mini-batch).  Thread i of the CTA owns hidden
 // unit i: column i of W1 (and W1b) and row i of W2 (and W2b).
+//
+// The momentum and decay variant (the Titans article's MLP memory, §二.1) adds
+// the momenta S1, S2 (the shapes of W1, W2, zero at the start):
+//   S1 <- alpha S1 - eta k^T G2,   W1 <- (1 - lambda) W1 + S1   (and so for W2)
+// 640 KB of state traffic per (batch, head) and call.
 struct MlpParams {
   const void *q, *k, *v;
   const float *eta;
@@ -149,11 +154,13 @@ struct MlpParams {
   float eps;
   int H, pos, b;
   float *z;
+  const float *alpha, *lambda;  // [units], momentum variant only
+  float *S1, *S2;               // like W1, W2, momentum variant only
 };
 constexpr int HID = simt::HID;
 constexpr int MLP_THREADS = HID;
 
-template <typename InT>
+template <typename InT, bool MOMENTUM = false>
 __global__ void __launch_bounds__(MLP_THREADS) mlp_decode_kernel(const MlpParams p) {
   __shared__ float qs[D], ks[D], vs[D], x2s[HID], z2s[HID], g3[D], part[8][D];
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
@@ -219,11 +226,23 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_decode_kernel(const MlpParams
   const float e = p.eta[unit];
   g2 *= simt::gelu_deriv(x1) * e;
   const bool last = p.pos == p.b - 1;
-  // W1 -= eta k^T G2 (column i) and Z1 = q W1 with the updated W1.
+  const float al = MOMENTUM ? p.alpha[unit] : 0.f;
+  const float keep = MOMENTUM ? 1.f - p.lambda[unit] : 1.f;
+  float *S1 = MOMENTUM ? p.S1 + unit * D * HID : nullptr;
+  float *S2 = MOMENTUM ? p.S2 + unit * HID * D : nullptr;
+  // W1 -= eta k^T G2 (column i; or the momentum and decay update) and Z1 = q W1
+  // with the updated W1.
   float z1 = 0.f;
 #pragma unroll 8
   for (int pp = 0; pp < D; ++pp) {
-    const float w = fmaf(-ks[pp], g2, W1[pp * HID + i]);
+    float w;
+    if (MOMENTUM) {
+      const float sm = fmaf(al, S1[pp * HID + i], -ks[pp] * g2);
+      S1[pp * HID + i] = sm;
+      w = fmaf(keep, W1[pp * HID + i], sm);
+    } else {
+      w = fmaf(-ks[pp], g2, W1[pp * HID + i]);
+    }
     W1[pp * HID + i] = w;
     if (last) W1b[pp * HID + i] = w;
     z1 = fmaf(qs[pp], w, z1);
@@ -237,8 +256,18 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_decode_kernel(const MlpParams
 #pragma unroll 8
     for (int r = 0; r < 32; ++r) {
       const int ii = 32 * warp + r;
-      const float w0 = fmaf(-x2s[ii], eg0, W2[ii * D + lane]);
-      const float w1 = fmaf(-x2s[ii], eg1, W2[ii * D + lane + 32]);
+      float w0, w1;
+      if (MOMENTUM) {
+        const float s0 = fmaf(al, S2[ii * D + lane], -x2s[ii] * eg0);
+        const float s1 = fmaf(al, S2[ii * D + lane + 32], -x2s[ii] * eg1);
+        S2[ii * D + lane] = s0;
+        S2[ii * D + lane + 32] = s1;
+        w0 = fmaf(keep, W2[ii * D + lane], s0);
+        w1 = fmaf(keep, W2[ii * D + lane + 32], s1);
+      } else {
+        w0 = fmaf(-x2s[ii], eg0, W2[ii * D + lane]);
+        w1 = fmaf(-x2s[ii], eg1, W2[ii * D + lane + 32]);
+      }
       W2[ii * D + lane] = w0;
       W2[ii * D + lane + 32] = w1;
       if (last) {

@@ -294,7 +294,8 @@ int run_decode(bool ln, const void *q, const void *k, const void *v, int qkv_dty
 int run_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype, const float *eta,
                    float *W1, float *W2, float *W1_base, float *W2_base, const float *gamma,
                    const float *beta, float eps, int B, int H, int d, int hidden, int b, int pos,
-                   float *z, void *stream) {
+                   float *z, void *stream, bool momentum = false, const float *alpha = nullptr,
+                   const float *lambda = nullptr, float *S1 = nullptr, float *S2 = nullptr) {
   if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
   if (B < 0 || H < 0 || d <= 0 || hidden <= 0 || b <= 0 || pos < 0 || pos >= b) return TTT_ERR_ARG;
   if (!(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
@@ -302,29 +303,43 @@ int run_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype, c
   const long long units = (long long)B * H;
   if (units == 0) return TTT_OK;
   if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
-  const void *req[] = {q, k, v, eta, W1, W2, W1_base, W2_base, z, gamma, beta};
+  const void *req[] = {q, k, v, eta, W1, W2, W1_base, W2_base, z, gamma, beta,
+                       momentum ? (const void *)alpha : q, momentum ? (const void *)lambda : q,
+                       momentum ? (const void *)S1 : q, momentum ? (const void *)S2 : q};
   for (const void *x : req)
     if (!x) return TTT_ERR_ARG;
   for (const void *x : req)
     if (!aligned16(x)) return TTT_ERR_ALIGN;
   const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
   const size_t wbytes = (size_t)units * d * hidden * 4;
-  Range ins[6] = {range_of(q, units * d * in_elt), range_of(k, units * d * in_elt),
+  const size_t sbytes = momentum ? wbytes : 0, rbytes = momentum ? units * 4 : 0;
+  Range ins[8] = {range_of(q, units * d * in_elt), range_of(k, units * d * in_elt),
                   range_of(v, units * d * in_elt), range_of(eta, units * 4),
-                  range_of(gamma, (size_t)H * d * 4), range_of(beta, (size_t)H * d * 4)};
-  Range outs[5] = {range_of(W1, wbytes), range_of(W2, wbytes), range_of(W1_base, wbytes),
-                   range_of(W2_base, wbytes), range_of(z, units * d * 4)};
-  for (int o = 0; o < 5; ++o) {
-    for (int i = 0; i < 6; ++i)
+                  range_of(gamma, (size_t)H * d * 4), range_of(beta, (size_t)H * d * 4),
+                  range_of(momentum ? (const void *)alpha : q, rbytes),
+                  range_of(momentum ? (const void *)lambda : q, rbytes)};
+  Range outs[7] = {range_of(W1, wbytes), range_of(W2, wbytes), range_of(W1_base, wbytes),
+                   range_of(W2_base, wbytes), range_of(z, units * d * 4),
+                   range_of(momentum ? (const void *)S1 : z, sbytes),
+                   range_of(momentum ? (const void *)S2 : z, sbytes)};
+  for (int o = 0; o < 7; ++o) {
+    for (int i = 0; i < 8; ++i)
       if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
-    for (int o2 = o + 1; o2 < 5; ++o2)
+    for (int o2 = o + 1; o2 < 7; ++o2)
       if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
   }
-  decode::MlpParams p{q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, eps, H, pos, b, z};
+  decode::MlpParams p{q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, eps, H, pos, b, z,
+                      alpha, lambda, S1, S2};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)units;
-  if (qkv_dtype == TTT_BF16) decode::mlp_decode_kernel<__nv_bfloat16><<<grid, decode::MLP_THREADS, 0, s>>>(p);
-  else decode::mlp_decode_kernel<float><<<grid, decode::MLP_THREADS, 0, s>>>(p);
+  const bool bf16 = qkv_dtype == TTT_BF16;
+  if (momentum) {
+    if (bf16) decode::mlp_decode_kernel<__nv_bfloat16, true><<<grid, decode::MLP_THREADS, 0, s>>>(p);
+    else decode::mlp_decode_kernel<float, true><<<grid, decode::MLP_THREADS, 0, s>>>(p);
+  } else {
+    if (bf16) decode::mlp_decode_kernel<__nv_bfloat16><<<grid, decode::MLP_THREADS, 0, s>>>(p);
+    else decode::mlp_decode_kernel<float><<<grid, decode::MLP_THREADS, 0, s>>>(p);
+  }
   if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return TTT_OK;
@@ -431,6 +446,15 @@ int ttt_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype, c
                    float *z, void *stream) {
   return run_mlp_decode(q, k, v, qkv_dtype, eta, W1, W2, W1_base, W2_base, ln_gamma, ln_beta, ln_eps,
                         B, H, d, hidden, b, pos, z, stream);
+}
+
+int ttt_mlp_momentum_decode(const void *q, const void *k, const void *v, int qkv_dtype,
+                            const float *eta, const float *alpha, const float *lambda, float *W1,
+                            float *W2, float *W1_base, float *W2_base, float *S1, float *S2,
+                            const float *ln_gamma, const float *ln_beta, float ln_eps, int B, int H,
+                            int d, int hidden, int b, int pos, float *z, void *stream) {
+  return run_mlp_decode(q, k, v, qkv_dtype, eta, W1, W2, W1_base, W2_base, ln_gamma, ln_beta, ln_eps,
+                        B, H, d, hidden, b, pos, z, stream, true, alpha, lambda, S1, S2);
 }
 
 int ttt_linear_ln_decode(const void *q, const void *k, const void *v, int qkv_dtype,

@@ -199,6 +199,39 @@ def ttt_mlp_decode(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, b, pos, 
                    stream=None):
     """One primal-form decode step of TTT-MLP.  W1, W1_base [B,H,d,hidden] and W2, W2_base
     [B,H,hidden,d] f32 are updated in place; gamma, beta [H,d].  Returns z [B,H,d] f32."""
+    dt, B, H, d, hidden, z = _mlp_decode_args(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, z)
+    with torch.cuda.device(q.device):
+        st = _lib.load().ttt_mlp_decode(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta),
+                                        _ptr(W1), _ptr(W2), _ptr(W1_base), _ptr(W2_base), _ptr(gamma),
+                                        _ptr(beta), float(eps), B, H, d, hidden, int(b), int(pos), _ptr(z),
+                                        _stream(stream, q.device))
+    check(st, "ttt_mlp_decode")
+    return z
+
+
+def ttt_mlp_momentum_decode(q, k, v, eta, alpha, lam, W1, W2, W1_base, W2_base, S1, S2, gamma, beta, b,
+                            pos, eps=1e-6, z=None, stream=None):
+    """The TTT-MLP decode step with the momentum and decay update: alpha, lam [B,H] f32;
+    the momenta S1 (like W1) and S2 (like W2) start at zero and are updated in place."""
+    dt, B, H, d, hidden, z = _mlp_decode_args(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, z)
+    for n, t in (("alpha", alpha), ("lam", lam)):
+        _cuda(t, n, torch.float32)
+        if tuple(t.shape) != (B, H):
+            raise ValueError(f"{n} must have shape {(B, H)}")
+    for n, t, ref in (("S1", S1, W1), ("S2", S2, W2)):
+        _cuda(t, n, torch.float32)
+        if t.shape != ref.shape:
+            raise ValueError(f"{n} must have shape {tuple(ref.shape)}")
+    with torch.cuda.device(q.device):
+        st = _lib.load().ttt_mlp_momentum_decode(
+            _ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(W1), _ptr(W2),
+            _ptr(W1_base), _ptr(W2_base), _ptr(S1), _ptr(S2), _ptr(gamma), _ptr(beta), float(eps), B, H,
+            d, hidden, int(b), int(pos), _ptr(z), _stream(stream, q.device))
+    check(st, "ttt_mlp_momentum_decode")
+    return z
+
+
+def _mlp_decode_args(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, z):
     for n, t in (("q", q), ("k", k), ("v", v)):
         _cuda(t, n)
     if not (q.dtype == k.dtype == v.dtype) or q.dtype not in _QKV_DTYPES:
@@ -216,13 +249,7 @@ def ttt_mlp_decode(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, b, pos, 
     for n, t in (("gamma", gamma), ("beta", beta)):
         _cuda(t, n, torch.float32)
     z = _out(z, (B, H, d), q.device, "z")
-    with torch.cuda.device(q.device):
-        st = _lib.load().ttt_mlp_decode(_ptr(q), _ptr(k), _ptr(v), _QKV_DTYPES[q.dtype], _ptr(eta),
-                                        _ptr(W1), _ptr(W2), _ptr(W1_base), _ptr(W2_base), _ptr(gamma),
-                                        _ptr(beta), float(eps), B, H, d, hidden, int(b), int(pos), _ptr(z),
-                                        _stream(stream, q.device))
-    check(st, "ttt_mlp_decode")
-    return z
+    return _QKV_DTYPES[q.dtype], B, H, d, hidden, z
 
 
 def set_path(path: int) -> int:

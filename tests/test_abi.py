@@ -186,6 +186,31 @@ def test_momentum_decode_argument_errors(lib, ln):
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
 
 
+def test_mlp_momentum_decode_argument_errors(lib):
+    n0 = lib.ttt_launch_count()
+    q, k, v, eta, al, lm, w1, w2, w1b, w2b, s1, s2, z, g, bt = _ptrs(15)
+
+    def call(**kw):
+        a = dict(q=q, k=k, v=v, dt=L.TTT_BF16, eta=eta, al=al, lm=lm, w1=w1, w2=w2, w1b=w1b, w2b=w2b,
+                 s1=s1, s2=s2, g=g, bt=bt, eps=1e-6, B=2, H=3, d=64, h=256, b=16, pos=0, z=z)
+        a.update(kw)
+        return lib.ttt_mlp_momentum_decode(a["q"], a["k"], a["v"], a["dt"], a["eta"], a["al"], a["lm"],
+                                           a["w1"], a["w2"], a["w1b"], a["w2b"], a["s1"], a["s2"],
+                                           a["g"], a["bt"], a["eps"], a["B"], a["H"], a["d"], a["h"],
+                                           a["b"], a["pos"], a["z"], None)
+
+    assert call(pos=16) == L.TTT_ERR_ARG
+    assert call(h=128) == L.TTT_ERR_UNSUPPORTED
+    assert call(s1=None) == L.TTT_ERR_ARG
+    assert call(lm=None) == L.TTT_ERR_ARG
+    assert call(s2=A + 8) == L.TTT_ERR_ALIGN
+    assert call(s2=s1 + 4096) == L.TTT_ERR_ARG        # the two momenta overlap
+    assert call(s1=w2 + 1024) == L.TTT_ERR_ARG        # S1 overlaps W2
+    assert call(al=s2 + 64) == L.TTT_ERR_ARG          # alpha inside S2
+    assert call(B=0) == L.TTT_OK
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
+
+
 def test_mlp_decode_argument_errors(lib):
     n0 = lib.ttt_launch_count()
     q, k, v, eta, w1, w2, w1b, w2b, z, g, bt = _ptrs(11)

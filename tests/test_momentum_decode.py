@@ -9,6 +9,7 @@ import oracle
 import test_sequence_modeling_b200 as ttt
 from test_sequence_modeling_b200 import inputs as I
 from gpu_helpers import rel_fro, to_device
+from test_momentum_tolerance import MLP_MOMENTUM_TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -81,3 +82,46 @@ def test_zero_momentum_and_decay_is_the_plain_step():
     torch.cuda.synchronize()
     np.testing.assert_allclose(Zm, Z.cpu().numpy(), rtol=0, atol=1e-6)
     np.testing.assert_allclose(Wm, W.cpu().numpy(), rtol=0, atol=1e-7)
+
+
+@pytest.mark.parametrize("b", [1, 16])
+def test_mlp_momentum_decode_matches_oracle(b):
+    cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=2, H=3, T=32, b=b)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    alpha, lam = I.momentum_rates(cfg)
+    al_d, lm_d = torch.from_numpy(alpha).cuda(), torch.from_numpy(lam).cuda()
+    B, H, T, d, h = cfg.B, cfg.H, cfg.T, cfg.d, cfg.hidden
+    W1 = dev["W1"].unsqueeze(0).expand(B, H, d, h).contiguous()
+    W2 = dev["W2"].unsqueeze(0).expand(B, H, h, d).contiguous()
+    W1b, W2b = W1.clone(), W2.clone()
+    S1, S2 = torch.zeros_like(W1), torch.zeros_like(W2)
+    Z = torch.empty(B, H, T, d, dtype=torch.float32, device="cuda")
+    for t in range(T):
+        q, k, v = (dev[n][:, :, t].contiguous() for n in ("Q", "K", "V"))
+        eta, al, lm = (x[:, :, t].contiguous() for x in (dev["eta"], al_d, lm_d))
+        Z[:, :, t] = ttt.ttt_mlp_momentum_decode(q, k, v, eta, al, lm, W1, W2, W1b, W2b, S1, S2,
+                                                 dev["gamma"], dev["beta"], cfg.b, t % cfg.b, cfg.ln_eps)
+    torch.cuda.synchronize()
+    assert ttt.last_device_status() == 0
+    Z, W1, W2, S1, S2 = (x.cpu().numpy() for x in (Z, W1, W2, S1, S2))
+    worst = {}
+    for bi in range(B):
+        for hi in range(H):
+            u = I.unit_as_f64(cfg, bi, hi)
+            params = np.concatenate([u["W1"].reshape(1, -1), u["W2"].reshape(1, -1)], axis=1)
+            Zr, Wr, Sr = oracle.default().momentum_forward(
+                oracle.MLP_LN, u["Q"], u["K"], u["V"], u["eta"],
+                alpha[bi, hi][None, None].astype(np.float64), lam[bi, hi][None, None].astype(np.float64),
+                params, cfg.b, u["gamma"], u["beta"], cfg.ln_eps, hidden=h)
+            n1 = d * h
+            for key, g, r in (("Z", Z[bi, hi], Zr[0, 0]), ("W1", W1[bi, hi].ravel(), Wr[0, 0, :n1]),
+                              ("W2", W2[bi, hi].ravel(), Wr[0, 0, n1:]),
+                              ("S1", S1[bi, hi].ravel(), Sr[0, 0, :n1]),
+                              ("S2", S2[bi, hi].ravel(), Sr[0, 0, n1:])):
+                assert np.all(np.isfinite(g))
+                worst[key] = max(worst.get(key, 0.0), rel_fro(g, r))
+    # fp32 rounding grows along the sequence under momentum with b = 1: the tolerance
+    # is derived from an independent fp32 evaluation in test_momentum_tolerance.py.
+    assert max(worst.values()) <= MLP_MOMENTUM_TOL, worst
+    assert torch.equal(W1b.cpu(), torch.from_numpy(W1))
+    assert torch.equal(W2b.cpu(), torch.from_numpy(W2))

@@ -1,0 +1,73 @@
+"""Where the momentum and decay tolerance comes from (no GPU): an fp32 evaluation
+of the TTT-MLP momentum recursion, written here with torch CPU float32 ops in an
+operation order unrelated to the CUDA kernel's, lands this far from the fp64
+oracle.  With b = 1 the momentum (alpha up to 0.9, an effective rate up to ten
+times eta) makes the token-to-token map far less contractive than plain TTT, so
+per-step fp32 rounding grows along the sequence: the spread exceeds the 1e-5 of
+the TTT forward, and the GPU parity test for this case uses MLP_MOMENTUM_TOL."""
+import numpy as np
+import torch
+
+import oracle
+from test_sequence_modeling_b200 import inputs as I
+
+MLP_MOMENTUM_TOL = 1e-4
+
+
+def _ln(y, g, bt, eps):
+    mu = y.mean()
+    var = ((y - mu) ** 2).mean()
+    return g * (y - mu) / torch.sqrt(var + eps) + bt
+
+
+def fp32_spread(b, B=2, H=3, T=32):
+    """Max relative Frobenius error of the fp32 evaluation against the oracle, per output."""
+    cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=B, H=H, T=T, b=b)
+    alpha, lam = I.momentum_rates(cfg)
+    gelu = torch.nn.functional.gelu
+    worst = {}
+    for bi in range(B):
+        for hi in range(H):
+            q, k, v, e = (torch.from_numpy(x) for x in I.unit_inputs(cfg, bi, hi))
+            p = I.head_params(cfg, hi)
+            g, bt = torch.from_numpy(p["gamma"]), torch.from_numpy(p["beta"])
+            W1, W2 = torch.from_numpy(p["W1"]).clone(), torch.from_numpy(p["W2"]).clone()
+            W1b, W2b = W1.clone(), W2.clone()
+            S1, S2 = torch.zeros_like(W1), torch.zeros_like(W2)
+            Z = []
+            for t in range(T):
+                X1 = (k[t] @ W1b).requires_grad_(True)
+                X2 = gelu(X1)
+                loss = ((k[t] + _ln(X2 @ W2b, g, bt, cfg.ln_eps) - v[t]) ** 2).sum()
+                G1, = torch.autograd.grad(loss, X1, retain_graph=True)
+                X3 = (X2.detach() @ W2b).requires_grad_(True)
+                G3, = torch.autograd.grad(((k[t] + _ln(X3, g, bt, cfg.ln_eps) - v[t]) ** 2).sum(), X3)
+                a, keep = float(alpha[bi, hi, t]), float(np.float32(1) - lam[bi, hi, t])
+                S1 = a * S1 - torch.outer(k[t], e[t] * G1)
+                S2 = a * S2 - torch.outer(X2.detach(), e[t] * G3)
+                W1, W2 = keep * W1 + S1, keep * W2 + S2
+                Z.append(q[t] + _ln(gelu(q[t] @ W1) @ W2, g, bt, cfg.ln_eps))
+                if t % b == b - 1:
+                    W1b, W2b = W1.clone(), W2.clone()
+            u = I.unit_as_f64(cfg, bi, hi)
+            params = np.concatenate([u["W1"].reshape(1, -1), u["W2"].reshape(1, -1)], axis=1)
+            Zr, Wr, Sr = oracle.default().momentum_forward(
+                oracle.MLP_LN, u["Q"], u["K"], u["V"], u["eta"],
+                alpha[bi, hi][None, None].astype(np.float64), lam[bi, hi][None, None].astype(np.float64),
+                params, b, u["gamma"], u["beta"], cfg.ln_eps, hidden=cfg.hidden)
+            n1 = cfg.d * cfg.hidden
+            for key, x, r in (("Z", torch.stack(Z), Zr[0, 0]), ("W1", W1, Wr[0, 0, :n1]),
+                              ("W2", W2, Wr[0, 0, n1:]), ("S1", S1, Sr[0, 0, :n1]),
+                              ("S2", S2, Sr[0, 0, n1:])):
+                x = x.detach().numpy().astype(np.float64).ravel()
+                r = r.ravel()
+                worst[key] = max(worst.get(key, 0.0), float(np.linalg.norm(x - r) / np.linalg.norm(r)))
+    return worst
+
+
+def test_fp32_spread_of_the_mlp_momentum_recursion():
+    spread = fp32_spread(b=1)
+    # fp32 arithmetic itself does not reach the forward's 1e-5 here ...
+    assert max(spread.values()) > 1e-5, spread
+    # ... and the tolerance leaves no more than a small factor above it.
+    assert max(spread.values()) * 1.5 <= MLP_MOMENTUM_TOL, spread
