@@ -275,10 +275,14 @@ def main():
                          "instead of the forward")
     ap.add_argument("--decode-mlp", action="store_true",
                     help="the same for the TTT-MLP decode step")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass of TTT-Linear + LN on the bench workload (B=16 H=32 T=8192)")
     ap.add_argument("--decode-momentum", action="store_true",
                     help="the decode step with the momentum and decay update (TTT-Linear + LN, or with "
                          "--decode-mlp TTT-MLP)")
     args = ap.parse_args()
+    if args.backward:
+        return run_backward(args)
     if args.decode or args.decode_mlp or args.decode_momentum:
         return run_decode(args, mlp=args.decode_mlp, momentum=args.decode_momentum)
     cfg = I.CONFIGS[args.workload]
@@ -388,6 +392,73 @@ def main():
     nflops = flops_per_head_token(cfg) * cfg.head_tokens
     return finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info, launches,
                   e2e, peaks, peak_kind, nbytes, nflops, dist)
+
+
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz.
+ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_backward(args):
+    """The backward pass's own line: one step = one launch of ttt_linear_ln_bwd over
+    the linear + LN workload (B=16 H=32 T=8192, b=16) with its incoming gradients."""
+    import torch
+    import test_sequence_modeling_b200 as ttt
+    from test_sequence_modeling_b200 import _lib
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"]
+    data = I.make_inputs(cfg)
+    B, H, T, d, b = cfg.B, cfg.H, cfg.T, cfg.d, cfg.b
+    qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
+    eta = torch.from_numpy(np.ascontiguousarray(data["eta"])).to(dev)
+    W0, gamma, beta = (torch.from_numpy(data[k]).to(dev) for k in ("W0", "gamma", "beta"))
+    dZ, dWT = (torch.from_numpy(x).to(dev) for x in I.cotangents(cfg))
+    stream = torch.cuda.current_stream(dev)
+    lib = _lib.load()
+
+    def step():
+        return ttt.ttt_linear_bwd(qkv["Q"], qkv["K"], qkv["V"], eta, W0, dZ, b, dW_T=dWT, gamma=gamma,
+                                  beta=beta, eps=cfg.ln_eps, stream=stream)
+
+    outs = step()  # allocates the outputs once; the timed steps reuse the allocator's blocks
+    del outs
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_id_for(torch, 0))
+    clocks.start()
+    n0 = lib.ttt_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = lib.ttt_launch_count() - n0
+    clock_info = clocks.stop()
+    if ttt.last_device_status() != 0:
+        raise RuntimeError("device status error")
+    ms = e0.elapsed_time(e1) / args.steps
+    units, N = B * H, T // b
+    # Multiply-adds of the dual-form backward per mini-batch (LN): the forward pass's
+    # K W and K^T E (2 b d^2); the reverse pass's K W, Q W, P W^T, K dW, E dW^T,
+    # dY W^T, Q^T P, K^T dY (8 b d^2) and the six masked b x b products (3 b^2 d).
+    flops = 2.0 * units * N * (10 * b * d * d + 3 * b * b * d)
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {
+        "metric": "TTT-Linear+LN backward tokens/s (B x H x T / s)",
+        "value": units * T / (ms / 1e3), "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "backward_" + cfg.name, "B": B, "H": H, "T": T, "d": d, "b": b,
+                   "qkv_dtype": "bf16", "l2": "inputs larger than L2 (no flush needed)"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_F32_TFLOPS, "unit": "TFLOP/s",
+                     "frac": achieved / ALU_F32_TFLOPS, "traffic": None,
+                     "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz (CUDA-core fp32 FMA)",
+                     "flops_per_launch": flops},
+        "clocks": clock_info, "gpu_launches": int(launches),
+    }
+    print(json.dumps(line), flush=True)
 
 
 def run_decode(args, mlp=False, momentum=False):

@@ -118,6 +118,34 @@ TTT_API int ttt_mlp_fwd(const void *Q, const void *K, const void *V, int qkv_dty
                 float *W1_out, float *W2_out, void *stream);
 
 /*
+ * Backward pass of TTT-Linear (and, _ln_, TTT-Linear with LN and residual): the
+ * gradients of L = <dZ, Z> + <dW_T, W_T> through the forward of ttt_linear_fwd /
+ * ttt_linear_ln_fwd (the write-up trains the layer end to end and computes the
+ * backward in the dual form too, §04.3).  Inputs as for the forward, plus
+ *   dZ     [B][H][T][d] fp32: the cotangent of Z.
+ *   dW_T   [B][H][d][d] fp32 or NULL (zero): the cotangent of the final state.
+ * Outputs (fp32, caller-owned, fully written):
+ *   dQ, dK, dV [B][H][T][d];  deta [B][H][T];
+ *   dW0    [B][H][d][d]: per (batch, head) unit; the gradient of a W0 shared by
+ *          the batch is the sum over the batch;
+ *   dgamma, dbeta [B][H][d] (LN only): per unit likewise;
+ *   W_ckpt [B][H][T/b][d][d]: the state at the start of every mini-batch
+ *          (W_ckpt[.][.][0] = W0), which the reverse pass reads.
+ * Mini-batch size 1 <= b <= 16 and d = 64 (else TTT_ERR_UNSUPPORTED); T % b == 0.
+ * No output may overlap an input or another output.  Errors as for the forward.
+ */
+TTT_API int ttt_linear_bwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                           const float *eta, const float *W0, const float *dZ, const float *dW_T,
+                           int B, int H, int T, int d, int b, float *dQ, float *dK, float *dV,
+                           float *deta, float *dW0, float *W_ckpt, void *stream);
+TTT_API int ttt_linear_ln_bwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                              const float *eta, const float *W0, const float *ln_gamma,
+                              const float *ln_beta, float ln_eps, const float *dZ,
+                              const float *dW_T, int B, int H, int T, int d, int b, float *dQ,
+                              float *dK, float *dV, float *deta, float *dW0, float *dgamma,
+                              float *dbeta, float *W_ckpt, void *stream);
+
+/*
  * Primal-form decode step (generation, §04.3 of the TTT write-up: decoding is
  * sequential and takes the primal form): one token per (batch, head) and call,
  * with the state carried in device memory across calls.

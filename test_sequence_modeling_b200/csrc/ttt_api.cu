@@ -13,6 +13,7 @@
 
 #include "ttt.h"
 #include "device_status.cuh"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "simt.cuh"
 #include "tc_linear.cuh"
@@ -20,6 +21,7 @@
 namespace simt = ttt::simt;
 namespace tc = ttt::tc;
 namespace decode = ttt::decode;
+namespace bwd = ttt::bwd;
 
 namespace {
 
@@ -345,6 +347,67 @@ int run_mlp_decode(const void *q, const void *k, const void *v, int qkv_dtype, c
   return TTT_OK;
 }
 
+int run_bwd(bool ln, const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+            const float *W0, const float *gamma, const float *beta, float eps, const float *dZ,
+            const float *dW_T, int B, int H, int T, int d, int b, float *dQ, float *dK, float *dV,
+            float *deta, float *dW0, float *dgamma, float *dbeta, float *W_ckpt, void *stream) {
+  if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return TTT_ERR_ARG;
+  if (T % b != 0) return TTT_ERR_ARG;
+  if (ln && !(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
+  if (d != bwd::D || b > bwd::MAXB) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)B * H;
+  if (units == 0) return TTT_OK;
+  if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  const long long elems = units * T * d;
+  if (elems >= (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+  const bool tok = T > 0;
+  // Required pointers (a stand-in that passes the checks where one is not needed).
+  const void *req[] = {W0, dW0, ln ? (const void *)gamma : W0, ln ? (const void *)beta : W0,
+                       ln ? (const void *)dgamma : dW0, ln ? (const void *)dbeta : dW0,
+                       tok ? Q : W0, tok ? K : W0, tok ? V : W0, tok ? (const void *)eta : W0,
+                       tok ? (const void *)dZ : W0, tok ? (const void *)dQ : dW0,
+                       tok ? (const void *)dK : dW0, tok ? (const void *)dV : dW0,
+                       tok ? (const void *)deta : dW0, tok ? (const void *)W_ckpt : dW0};
+  for (const void *x : req)
+    if (!x) return TTT_ERR_ARG;
+  for (const void *x : req)
+    if (!aligned16(x)) return TTT_ERR_ALIGN;
+  if (dW_T && !aligned16(dW_T)) return TTT_ERR_ALIGN;
+  const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t tbytes = tok ? (size_t)elems * 4 : 0, ibytes = tok ? (size_t)elems * in_elt : 0;
+  const size_t ebytes = tok ? (size_t)units * T * 4 : 0, wbytes = (size_t)units * d * d * 4;
+  const size_t vbytes = ln ? (size_t)units * d * 4 : 0, pbytes = ln ? (size_t)H * d * 4 : 0;
+  const size_t cbytes = tok ? (size_t)units * (T / b) * d * d * 4 : 0;
+  Range ins[9] = {range_of(Q, ibytes), range_of(K, ibytes), range_of(V, ibytes),
+                  range_of(eta, ebytes), range_of(W0, (size_t)H * d * d * 4),
+                  range_of(gamma, pbytes), range_of(beta, pbytes), range_of(dZ, tbytes),
+                  range_of(dW_T, dW_T ? wbytes : 0)};
+  Range outs[8] = {range_of(dQ, tbytes),   range_of(dK, tbytes),     range_of(dV, tbytes),
+                   range_of(deta, ebytes), range_of(dW0, wbytes),    range_of(dgamma, vbytes),
+                   range_of(dbeta, vbytes), range_of(W_ckpt, cbytes)};
+  for (int o = 0; o < 8; ++o) {
+    for (int i = 0; i < 9; ++i)
+      if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
+    for (int o2 = o + 1; o2 < 8; ++o2)
+      if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
+  }
+  bwd::Params p{Q, K, V, eta, W0, gamma, beta, eps, dZ, dW_T, H, T, b,
+                dQ, dK, dV, deta, dW0, dgamma, dbeta, W_ckpt};
+  auto kernel = ln ? (qkv_dtype == TTT_BF16 ? bwd::linear_bwd_kernel<true, __nv_bfloat16>
+                                            : bwd::linear_bwd_kernel<true, float>)
+                   : (qkv_dtype == TTT_BF16 ? bwd::linear_bwd_kernel<false, __nv_bfloat16>
+                                            : bwd::linear_bwd_kernel<false, float>);
+  const size_t smem = bwd::smem_bytes();
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return TTT_ERR_CUDA;
+  kernel<<<(unsigned)units, bwd::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 int run(const Call &c) {
   const int st = validate(c);
   if (st != TTT_OK) return st;
@@ -455,6 +518,23 @@ int ttt_mlp_momentum_decode(const void *q, const void *k, const void *v, int qkv
                             int d, int hidden, int b, int pos, float *z, void *stream) {
   return run_mlp_decode(q, k, v, qkv_dtype, eta, W1, W2, W1_base, W2_base, ln_gamma, ln_beta, ln_eps,
                         B, H, d, hidden, b, pos, z, stream, true, alpha, lambda, S1, S2);
+}
+
+int ttt_linear_bwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                   const float *W0, const float *dZ, const float *dW_T, int B, int H, int T, int d,
+                   int b, float *dQ, float *dK, float *dV, float *deta, float *dW0, float *W_ckpt,
+                   void *stream) {
+  return run_bwd(false, Q, K, V, qkv_dtype, eta, W0, nullptr, nullptr, 1.f, dZ, dW_T, B, H, T, d, b,
+                 dQ, dK, dV, deta, dW0, nullptr, nullptr, W_ckpt, stream);
+}
+
+int ttt_linear_ln_bwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                      const float *W0, const float *ln_gamma, const float *ln_beta, float ln_eps,
+                      const float *dZ, const float *dW_T, int B, int H, int T, int d, int b,
+                      float *dQ, float *dK, float *dV, float *deta, float *dW0, float *dgamma,
+                      float *dbeta, float *W_ckpt, void *stream) {
+  return run_bwd(true, Q, K, V, qkv_dtype, eta, W0, ln_gamma, ln_beta, ln_eps, dZ, dW_T, B, H, T, d,
+                 b, dQ, dK, dV, deta, dW0, dgamma, dbeta, W_ckpt, stream);
 }
 
 int ttt_linear_ln_decode(const void *q, const void *k, const void *v, int qkv_dtype,

@@ -173,6 +173,15 @@ def momentum_rates(cfg: TTTConfig, seed: int = 0):
     return alpha, lam
 
 
+def cotangents(cfg: TTTConfig, seed: int = 0):
+    """Incoming gradients for the backward pass: dZ [B, H, T, d] ~ N(0, 1/d) and
+    dW_T [B, H, d, d] ~ N(0, 1/d^2), float32."""
+    rng = np.random.default_rng([cfg.seed, 4, seed])
+    dZ = (rng.standard_normal((cfg.B, cfg.H, cfg.T, cfg.d), dtype=np.float32) / np.float32(math.sqrt(cfg.d)))
+    dWT = (rng.standard_normal((cfg.B, cfg.H, cfg.d, cfg.d), dtype=np.float32) / np.float32(cfg.d))
+    return dZ, dWT
+
+
 def unit_as_f64(cfg: TTTConfig, bi: int, hi: int, T: int | None = None) -> dict:
     """One unit's inputs and its head's parameters in float64, shaped [1,1,T,d] and
     [1,...] for feeding a per-unit reference computation."""

@@ -111,6 +111,52 @@ def ttt_mlp_fwd(Q, K, V, eta, W1, W2, gamma, beta, b, eps=1e-6, Z=None, W1_out=N
     return Z, W1_out, W2_out
 
 
+def ttt_linear_bwd(Q, K, V, eta, W0, dZ, b, dW_T=None, gamma=None, beta=None, eps=1e-6, stream=None):
+    """Backward of ttt_linear_fwd (or, with gamma and beta, of ttt_linear_ln_fwd): the
+    gradients of <dZ, Z> + <dW_T, W_T>.  dZ [B,H,T,d] f32, dW_T [B,H,d,d] f32 or None.
+    Returns a dict: dQ, dK, dV, deta, dW0 (per unit [B,H,d,d]), W_ckpt [B,H,T/b,d,d]
+    (the state at every mini-batch start) and, with LN, dgamma, dbeta [B,H,d]."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    ln = gamma is not None
+    _cuda(eta, "eta", torch.float32)
+    _cuda(W0, "W0", torch.float32)
+    _cuda(dZ, "dZ", torch.float32)
+    if tuple(dZ.shape) != (B, H, T, d):
+        raise ValueError(f"dZ must have shape {(B, H, T, d)}")
+    if dW_T is not None:
+        _cuda(dW_T, "dW_T", torch.float32)
+        if tuple(dW_T.shape) != (B, H, d, d):
+            raise ValueError(f"dW_T must have shape {(B, H, d, d)}")
+    if ln:
+        for n, t in (("gamma", gamma), ("beta", beta)):
+            _cuda(t, n, torch.float32)
+    if b <= 0 or T % b:
+        raise ValueError("T must be a multiple of b")
+    dev = Q.device
+    out = {n: torch.empty(B, H, T, d, device=dev) for n in ("dQ", "dK", "dV")}
+    out["deta"] = torch.empty(B, H, T, device=dev)
+    out["dW0"] = torch.empty(B, H, d, d, device=dev)
+    out["W_ckpt"] = torch.empty(B, H, T // b, d, d, device=dev)
+    if ln:
+        out["dgamma"] = torch.empty(B, H, d, device=dev)
+        out["dbeta"] = torch.empty(B, H, d, device=dev)
+    o = {k: _ptr(v) for k, v in out.items()}
+    dwt = _ptr(dW_T)
+    with torch.cuda.device(dev):
+        if ln:
+            st = _lib.load().ttt_linear_ln_bwd(
+                _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W0), _ptr(gamma), _ptr(beta), float(eps),
+                _ptr(dZ), dwt, B, H, T, d, int(b), o["dQ"], o["dK"], o["dV"], o["deta"], o["dW0"],
+                o["dgamma"], o["dbeta"], o["W_ckpt"], _stream(stream, dev))
+        else:
+            st = _lib.load().ttt_linear_bwd(
+                _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W0), _ptr(dZ), dwt, B, H, T, d, int(b),
+                o["dQ"], o["dK"], o["dV"], o["deta"], o["dW0"], o["W_ckpt"], _stream(stream, dev))
+    check(st, "ttt_linear_ln_bwd" if ln else "ttt_linear_bwd")
+    return out
+
+
 def _decode_args(q, k, v, eta, W, W_base, z):
     for n, t in (("q", q), ("k", k), ("v", v)):
         _cuda(t, n)

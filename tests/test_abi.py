@@ -233,3 +233,43 @@ def test_mlp_decode_argument_errors(lib):
     assert call(w2b=w1b + 4096) == L.TTT_ERR_ARG      # the two bases overlap
     assert call(B=0) == L.TTT_OK
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
+
+
+def bwd(lib, ln=False, **kw):
+    q, k, v, eta, w0, dz, dwt, dq, dk, dv, de, dw0, ck, g, bt, dg, db = _ptrs(17)
+    a = dict(q=q, k=k, v=v, dt=L.TTT_BF16, eta=eta, w0=w0, dz=dz, dwt=dwt, B=2, H=3, T=64, d=64, b=16,
+             dq=dq, dk=dk, dv=dv, de=de, dw0=dw0, ck=ck, g=g, bt=bt, dg=dg, db=db, eps=1e-6)
+    a.update(kw)
+    if ln:
+        return lib.ttt_linear_ln_bwd(a["q"], a["k"], a["v"], a["dt"], a["eta"], a["w0"], a["g"], a["bt"],
+                                     a["eps"], a["dz"], a["dwt"], a["B"], a["H"], a["T"], a["d"], a["b"],
+                                     a["dq"], a["dk"], a["dv"], a["de"], a["dw0"], a["dg"], a["db"],
+                                     a["ck"], None)
+    return lib.ttt_linear_bwd(a["q"], a["k"], a["v"], a["dt"], a["eta"], a["w0"], a["dz"], a["dwt"],
+                              a["B"], a["H"], a["T"], a["d"], a["b"], a["dq"], a["dk"], a["dv"], a["de"],
+                              a["dw0"], a["ck"], None)
+
+
+@pytest.mark.parametrize("ln", [False, True])
+def test_backward_argument_errors(lib, ln):
+    n0 = lib.ttt_launch_count()
+    p = _ptrs(17)
+    assert bwd(lib, ln, b=32) == L.TTT_ERR_UNSUPPORTED      # mini-batch above 16
+    assert bwd(lib, ln, d=32) == L.TTT_ERR_UNSUPPORTED
+    assert bwd(lib, ln, T=40) == L.TTT_ERR_ARG              # T not a multiple of b
+    assert bwd(lib, ln, b=0) == L.TTT_ERR_ARG
+    assert bwd(lib, ln, dt=7) == L.TTT_ERR_ARG
+    assert bwd(lib, ln, dz=None) == L.TTT_ERR_ARG
+    assert bwd(lib, ln, ck=None) == L.TTT_ERR_ARG
+    assert bwd(lib, ln, dw0=None) == L.TTT_ERR_ARG
+    assert bwd(lib, ln, dq=A + 4) == L.TTT_ERR_ALIGN
+    assert bwd(lib, ln, dwt=A + 8) == L.TTT_ERR_ALIGN
+    assert bwd(lib, ln, dk=p[7] + 4096) == L.TTT_ERR_ARG    # dK overlaps dQ
+    assert bwd(lib, ln, ck=p[5] + 64) == L.TTT_ERR_ARG      # W_ckpt overlaps dZ
+    assert bwd(lib, ln, de=p[6] + 16) == L.TTT_ERR_ARG      # deta overlaps dW_T
+    assert bwd(lib, ln, B=0) == L.TTT_OK
+    if ln:
+        assert bwd(lib, ln, eps=0.0) == L.TTT_ERR_ARG
+        assert bwd(lib, ln, dg=None) == L.TTT_ERR_ARG
+        assert bwd(lib, ln, db=p[15] + 16) == L.TTT_ERR_ARG  # dbeta overlaps dgamma
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
