@@ -78,15 +78,30 @@ struct Smem {
 
 inline size_t smem_bytes() { return sizeof(Smem); }
 
+// The [row][D] products are register-blocked over the four rows rq + 4k of a
+// thread: one column operand load serves four FMAs (the row operands are
+// warp-wide broadcasts).  Rows at or beyond b hold stale values; their sums are
+// computed and dropped.
+//
+// acc[k] += sum_i in[rq + 4k][i] W[i][c]
+__device__ __forceinline__ void rows_W(const float *in, const float *W, int rq, int c,
+                                       float (&acc)[4]) {
+#pragma unroll 8
+  for (int i = 0; i < D; ++i) {
+    const float w = W[i * LD + c];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = fmaf(in[(rq + 4 * k) * LD + i], w, acc[k]);
+  }
+}
+
 // out[r][c] = sum_i in[r][i] W[i][c] for the rows r = rq, rq + 4, ... < b.
 __device__ __forceinline__ void rows_times_W(const float *in, const float *W, float *out, int b,
                                              int rq, int c) {
-  for (int r = rq; r < b; r += 4) {
-    float acc = 0.f;
-#pragma unroll 16
-    for (int i = 0; i < D; ++i) acc = fmaf(in[r * LD + i], W[i * LD + c], acc);
-    out[r * LD + c] = acc;
-  }
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  rows_W(in, W, rq, c, acc);
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (rq + 4 * k < b) out[(rq + 4 * k) * LD + c] = acc[k];
 }
 
 // G (and E = eta G) of the rows warp, warp + 8 < b, from Y in s.X.  With LN the
@@ -182,11 +197,18 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
     __syncthreads();
     grad_rows<LN>(s, b, warp, lane, g0, g1, be0, be1, p.eps);
     __syncthreads();
-    // W -= K^T E
-    for (int i = rq; i < D; i += 4) {
-      float acc = 0.f;
-      for (int r = 0; r < b; ++r) acc = fmaf(s.K[r * LD + i], s.E[r * LD + col], acc);
-      s.W[i * LD + col] -= acc;
+    // W -= K^T E; this thread's rows i = rq + 4k of column col.
+    {
+      float acc[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+      for (int r = 0; r < b; ++r) {
+        const float e = s.E[r * LD + col];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc[k] = fmaf(s.K[r * LD + rq + 4 * k], e, acc[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < 16; ++k) s.W[(rq + 4 * k) * LD + col] -= acc[k];
     }
     __syncthreads();
   }
@@ -225,12 +247,18 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
 
     if (LN) {
       // Zpre = Q W - A E, then P = dL/dZpre through the output LN.
-      for (int r = rq; r < b; r += 4) {
-        float acc = 0.f;
-#pragma unroll 16
-        for (int i = 0; i < D; ++i) acc = fmaf(s.Q[r * LD + i], s.W[i * LD + col], acc);
-        for (int u = 0; u <= r; ++u) acc = fmaf(-s.A[r * BLD + u], s.E[u * LD + col], acc);
-        s.Zh[r * LD + col] = acc;
+      {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        rows_W(s.Q, s.W, rq, col, acc);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = rq + 4 * k;
+          if (r < b) {
+            float z = acc[k];
+            for (int u = 0; u <= r; ++u) z = fmaf(-s.A[r * BLD + u], s.E[u * LD + col], z);
+            s.Zh[r * LD + col] = z;
+          }
+        }
       }
       __syncthreads();
       for (int r = warp; r < b; r += 8) {
@@ -271,17 +299,29 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
     __syncthreads();
 
     // dQ (to global) and dE.  Here col is the output column (i for dQ, j for dE).
-    for (int r = rq; r < b; r += 4) {
-      float q = LN ? s.dZ[r * LD + col] : 0.f;
-#pragma unroll 16
-      for (int j = 0; j < D; ++j) q = fmaf(P[r * LD + j], s.W[col * LD + j], q);
-      for (int u = 0; u <= r; ++u) q = fmaf(-s.M[r * BLD + u], s.K[u * LD + col], q);
-      p.dQ[(tok0 + row0 + r) * D + col] = q;
-      float e = 0.f;
-      for (int t = r; t < b; ++t) e = fmaf(-s.A[t * BLD + r], P[t * LD + col], e);
-#pragma unroll 16
-      for (int i = 0; i < D; ++i) e = fmaf(-s.K[r * LD + i], s.dW[i * LD + col], e);
-      s.dE[r * LD + col] = e;
+    {
+      float q[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int j = 0; j < D; ++j) {
+        const float w = s.W[col * LD + j], dw = s.dW[j * LD + col];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          q[k] = fmaf(P[(rq + 4 * k) * LD + j], w, q[k]);
+          e[k] = fmaf(-s.K[(rq + 4 * k) * LD + j], dw, e[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = rq + 4 * k;
+        if (r < b) {
+          float qq = LN ? q[k] + s.dZ[r * LD + col] : q[k];
+          for (int u = 0; u <= r; ++u) qq = fmaf(-s.M[r * BLD + u], s.K[u * LD + col], qq);
+          p.dQ[(tok0 + row0 + r) * D + col] = qq;
+          float ee = e[k];
+          for (int t = r; t < b; ++t) ee = fmaf(-s.A[t * BLD + r], P[t * LD + col], ee);
+          s.dE[r * LD + col] = ee;
+        }
+      }
     }
     __syncthreads();
 
@@ -334,26 +374,44 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
     __syncthreads();
 
     // dK (to global); col is the output column i.
-    for (int r = rq; r < b; r += 4) {
-      float k = LN ? s.R[r * LD + col] : 0.f;
-      for (int t = r; t < b; ++t) k = fmaf(-s.M[t * BLD + r], s.Q[t * LD + col], k);
-#pragma unroll 16
+    {
+      float kk[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
       for (int j = 0; j < D; ++j) {
-        k = fmaf(-s.E[r * LD + j], s.dW[col * LD + j], k);
-        k = fmaf(s.dY[r * LD + j], s.W[col * LD + j], k);
+        const float dw = s.dW[col * LD + j], w = s.W[col * LD + j];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          kk[k] = fmaf(-s.E[(rq + 4 * k) * LD + j], dw, kk[k]);
+          kk[k] = fmaf(s.dY[(rq + 4 * k) * LD + j], w, kk[k]);
+        }
       }
-      p.dK[(tok0 + row0 + r) * D + col] = k;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int r = rq + 4 * k;
+        if (r < b) {
+          float v = LN ? kk[k] + s.R[r * LD + col] : kk[k];
+          for (int t = r; t < b; ++t) v = fmaf(-s.M[t * BLD + r], s.Q[t * LD + col], v);
+          p.dK[(tok0 + row0 + r) * D + col] = v;
+        }
+      }
     }
     __syncthreads();
 
-    // dW_n = dW_{n+1} + Q^T P + K^T dY.
-    for (int i = rq; i < D; i += 4) {
-      float acc = 0.f;
+    // dW_n = dW_{n+1} + Q^T P + K^T dY; this thread's rows i = rq + 4k of column col.
+    {
+      float acc[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) acc[k] = 0.f;
       for (int r = 0; r < b; ++r) {
-        acc = fmaf(s.Q[r * LD + i], P[r * LD + col], acc);
-        acc = fmaf(s.K[r * LD + i], s.dY[r * LD + col], acc);
+        const float pr = P[r * LD + col], dyr = s.dY[r * LD + col];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          acc[k] = fmaf(s.Q[r * LD + rq + 4 * k], pr, acc[k]);
+          acc[k] = fmaf(s.K[r * LD + rq + 4 * k], dyr, acc[k]);
+        }
       }
-      s.dW[i * LD + col] += acc;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) s.dW[(rq + 4 * k) * LD + col] += acc[k];
     }
     __syncthreads();
   }
