@@ -17,7 +17,8 @@ all in float64 on the CPU.  No blocking, no dual form, no hand-written adjoint.
 
 f is  x W            (TTT-Linear), or
       x + LN(x W)    (TTT-Linear with LayerNorm and residual, §03.9; population
-                      variance, eps inside the square root, affine gamma, beta).
+                      variance, eps inside the square root, affine gamma, beta),
+      x + LN(GELU(x W1) W2)   (TTT-MLP, §03.9: hidden width 4d, exact GELU).
 """
 from __future__ import annotations
 
@@ -38,22 +39,33 @@ def _f(x, W, ln, gamma, beta, eps):
     return x + _ln(y, gamma, beta, eps) if ln else y
 
 
-def _unit_forward(q, k, v, eta, W0, b, ln, gamma, beta, eps):
-    """Primal rule for one (batch, head) unit; returns Z [T, d] and the final W.
-    W0 must require grad (every state is then a node of the graph)."""
-    T = q.shape[0]
-    W = W0
-    Wbase = W0
+def _f_mlp(x, Ws, gamma, beta, eps):
+    return x + _ln(torch.nn.functional.gelu(x @ Ws[0]) @ Ws[1], gamma, beta, eps)
+
+
+def _unit_forward_states(q, k, v, eta, W0s, b, f):
+    """Primal rule for one (batch, head) unit with the state a list of matrices
+    and f(x, states); returns Z [T, d] and the final states.  Every W0 must
+    require grad (every state is then a node of the graph)."""
+    Ws = list(W0s)
+    base = Ws
     Z = []
-    for t in range(T):
+    for t in range(q.shape[0]):
         if t % b == 0:
-            Wbase = W
+            base = Ws
         # grad_W l(W_base; k_t, v_t), kept differentiable in W_base, k, v, gamma, beta.
-        loss = ((_f(k[t], Wbase, ln, gamma, beta, eps) - v[t]) ** 2).sum()
-        g, = torch.autograd.grad(loss, Wbase, create_graph=True)
-        W = W - eta[t] * g
-        Z.append(_f(q[t], W, ln, gamma, beta, eps))
-    return torch.stack(Z), W
+        loss = ((f(k[t], base) - v[t]) ** 2).sum()
+        grads = torch.autograd.grad(loss, base, create_graph=True)
+        Ws = [W - eta[t] * g for W, g in zip(Ws, grads)]
+        Z.append(f(q[t], Ws))
+    return torch.stack(Z), Ws
+
+
+def _unit_forward(q, k, v, eta, W0, b, ln, gamma, beta, eps):
+    """TTT-Linear (or with LN) for one unit; returns Z [T, d] and the final W."""
+    Z, Ws = _unit_forward_states(q, k, v, eta, [W0], b,
+                                 lambda x, Ws: _f(x, Ws[0], ln, gamma, beta, eps))
+    return Z, Ws[0]
 
 
 def ttt_linear_backward(Q, K, V, eta, W0, b, dZ, dW_T=None, ln=False, gamma=None, beta=None,
@@ -95,4 +107,42 @@ def ttt_linear_backward(Q, K, V, eta, W0, b, dZ, dW_T=None, ln=False, gamma=None
             out["dW0"][bi, hi] = grads[4]
             if ln:
                 out["dgamma"][bi, hi], out["dbeta"][bi, hi] = grads[5], grads[6]
+    return out
+
+
+def ttt_mlp_backward(Q, K, V, eta, W1, W2, b, dZ, gamma, beta, eps=1e-6, dW1_T=None, dW2_T=None):
+    """Gradients of L = <dZ, Z> + <dW1_T, W1_T> + <dW2_T, W2_T> through the TTT-MLP
+    forward.  Q, K, V, dZ [B,H,T,d]; eta [B,H,T]; W1 [H,d,h], W2 [H,h,d], gamma,
+    beta [H,d] (per head); dW1_T [B,H,d,h], dW2_T [B,H,h,d] or None.  Returns a
+    dict of float64 arrays: dQ, dK, dV, deta, and per (batch, head) unit dW1,
+    dW2 (of the initial states), dgamma, dbeta."""
+    Q, K, V, eta, dZ = (np.asarray(x, np.float64) for x in (Q, K, V, eta, dZ))
+    W1, W2 = np.asarray(W1, np.float64), np.asarray(W2, np.float64)
+    B, H, T, d = Q.shape
+    h = W1.shape[-1]
+    out = {k: np.zeros((B, H, T, d)) for k in ("dQ", "dK", "dV")}
+    out["deta"] = np.zeros((B, H, T))
+    out["dW1"] = np.zeros((B, H, d, h))
+    out["dW2"] = np.zeros((B, H, h, d))
+    out["dgamma"] = np.zeros((B, H, d))
+    out["dbeta"] = np.zeros((B, H, d))
+    for bi in range(B):
+        for hi in range(H):
+            leaves = [torch.tensor(x[bi, hi], dtype=_f64, requires_grad=True) for x in (Q, K, V, eta)]
+            w1 = torch.tensor(W1[hi], requires_grad=True)
+            w2 = torch.tensor(W2[hi], requires_grad=True)
+            g = torch.tensor(np.asarray(gamma, np.float64)[hi], requires_grad=True)
+            bt = torch.tensor(np.asarray(beta, np.float64)[hi], requires_grad=True)
+            Z, (W1T, W2T) = _unit_forward_states(*leaves, [w1, w2], b,
+                                                 lambda x, Ws: _f_mlp(x, Ws, g, bt, eps))
+            L = (Z * torch.tensor(dZ[bi, hi])).sum()
+            if dW1_T is not None:
+                L = L + (W1T * torch.tensor(np.asarray(dW1_T, np.float64)[bi, hi])).sum()
+            if dW2_T is not None:
+                L = L + (W2T * torch.tensor(np.asarray(dW2_T, np.float64)[bi, hi])).sum()
+            wrt = leaves + [w1, w2, g, bt]
+            grads = torch.autograd.grad(L, wrt, allow_unused=True)
+            grads = [np.zeros(x.shape) if gr is None else gr.detach().numpy() for gr, x in zip(grads, wrt)]
+            for key, gr in zip(("dQ", "dK", "dV", "deta", "dW1", "dW2", "dgamma", "dbeta"), grads):
+                out[key][bi, hi] = gr
     return out
