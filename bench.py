@@ -275,6 +275,9 @@ def main():
                          "instead of the forward")
     ap.add_argument("--decode-mlp", action="store_true",
                     help="the same for the TTT-MLP decode step")
+    ap.add_argument("--momentum", action="store_true",
+                    help="time the whole-sequence forward with the momentum and decay update (TTT-Linear + LN, "
+                         "B=16 H=32 T=8192)")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass of TTT-Linear + LN on the bench workload (B=16 H=32 T=8192)")
     ap.add_argument("--decode-momentum", action="store_true",
@@ -283,6 +286,8 @@ def main():
     args = ap.parse_args()
     if args.backward:
         return run_backward(args)
+    if args.momentum:
+        return run_momentum(args)
     if args.decode or args.decode_mlp or args.decode_momentum:
         return run_decode(args, mlp=args.decode_mlp, momentum=args.decode_momentum)
     cfg = I.CONFIGS[args.workload]
@@ -396,6 +401,68 @@ def main():
 
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 FP32 lanes x 2 flops x 1965 MHz.
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_momentum(args):
+    """The momentum and decay forward's own line: one step = one launch of
+    ttt_linear_ln_momentum_fwd over the linear + LN workload (B=16 H=32 T=8192, b=16)."""
+    import torch
+    import test_sequence_modeling_b200 as ttt
+    from test_sequence_modeling_b200 import _lib
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"]
+    data = I.make_inputs(cfg)
+    B, H, T, d, b = cfg.B, cfg.H, cfg.T, cfg.d, cfg.b
+    qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
+    eta = torch.from_numpy(np.ascontiguousarray(data["eta"])).to(dev)
+    W0, gamma, beta = (torch.from_numpy(data[k]).to(dev) for k in ("W0", "gamma", "beta"))
+    alpha, lam = (torch.from_numpy(x).to(dev) for x in I.momentum_rates(cfg))
+    Z = torch.empty(B, H, T, d, device=dev)
+    W_out, S_out = torch.empty(B, H, d, d, device=dev), torch.empty(B, H, d, d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lib = _lib.load()
+
+    def step():
+        ttt.ttt_linear_momentum_fwd(qkv["Q"], qkv["K"], qkv["V"], eta, alpha, lam, W0, b, gamma=gamma,
+                                    beta=beta, eps=cfg.ln_eps, Z=Z, W_out=W_out, S_out=S_out, stream=stream)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_id_for(torch, 0))
+    clocks.start()
+    n0 = lib.ttt_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = lib.ttt_launch_count() - n0
+    clock_info = clocks.stop()
+    if ttt.last_device_status() != 0:
+        raise RuntimeError("device status error")
+    ms = e0.elapsed_time(e1) / args.steps
+    units = B * H
+    # Algorithmic bytes: q, k, v (bf16), eta, alpha, lambda in and Z out per token;
+    # W0 in and W_out, S_out out per unit.
+    nbytes = units * (T * (3 * d * 2 + 3 * 4 + d * 4) + 3 * d * d * 4)
+    peaks, peak_kind = load_peaks()
+    achieved = nbytes / (ms / 1e3) / 1e9
+    line = {
+        "metric": "TTT-Linear+LN momentum/decay forward tokens/s (B x H x T / s)",
+        "value": units * T / (ms / 1e3), "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "momentum_" + cfg.name, "B": B, "H": H, "T": T, "d": d, "b": b,
+                   "qkv_dtype": "bf16", "l2": "inputs larger than L2 (no flush needed)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)", "algorithmic_bytes_per_launch": nbytes},
+        "clocks": clock_info, "gpu_launches": int(launches),
+    }
+    print(json.dumps(line), flush=True)
 
 
 def run_backward(args):

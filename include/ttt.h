@@ -118,6 +118,31 @@ TTT_API int ttt_mlp_fwd(const void *Q, const void *K, const void *V, int qkv_dty
                 float *W1_out, float *W2_out, void *stream);
 
 /*
+ * Forward of TTT-Linear (and, _ln_, TTT-Linear with LN and residual) over whole
+ * sequences with the momentum and decay update of the Titans article (§二.1(2):
+ * momentum on past surprise, weight decay that forgets), kept to the TTT
+ * mini-batch rule: with S_0 = 0 and G_t the loss gradient at the state the
+ * mini-batch of token t started from,
+ *   S_t = alpha_t S_{t-1} - eta_t k_t^T G_t,  W_t = (1 - lambda_t) W_{t-1} + S_t,
+ *   z_t = q_t W_t  (or q_t + LN(q_t W_t)).
+ * Inputs as for the forward, plus alpha, lambda [B][H][T] fp32 (per token, like
+ * eta).  Outputs: Z [B][H][T][d], W_out and S_out [B][H][d][d] (the final state
+ * and momentum), fp32.  1 <= b <= 16 and d = 64 (else TTT_ERR_UNSUPPORTED),
+ * T % b == 0.  alpha = lambda = 0 is the plain TTT forward.  Errors as for the
+ * forward entry points.
+ */
+TTT_API int ttt_linear_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                                    const float *eta, const float *alpha, const float *lambda,
+                                    const float *W0, int B, int H, int T, int d, int b, float *Z,
+                                    float *W_out, float *S_out, void *stream);
+TTT_API int ttt_linear_ln_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                                       const float *eta, const float *alpha, const float *lambda,
+                                       const float *W0, const float *ln_gamma,
+                                       const float *ln_beta, float ln_eps, int B, int H, int T,
+                                       int d, int b, float *Z, float *W_out, float *S_out,
+                                       void *stream);
+
+/*
  * Backward pass of TTT-Linear (and, _ln_, TTT-Linear with LN and residual): the
  * gradients of L = <dZ, Z> + <dW_T, W_T> through the forward of ttt_linear_fwd /
  * ttt_linear_ln_fwd (the write-up trains the layer end to end and computes the

@@ -25,6 +25,10 @@ SIGNATURES = {
     "ttt_set_path": (_i, [_i]),
     "ttt_launch_count": (ctypes.c_longlong, []),
     "ttt_debug_inject_timeout": (_i, [_i]),
+    "ttt_linear_momentum_fwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _fp, _fp,
+                                     _fp, _vp]),
+    "ttt_linear_ln_momentum_fwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i,
+                                        _i, _i, _fp, _fp, _fp, _vp]),
     "ttt_linear_bwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _i, _i, _i, _i, _i, _fp, _fp, _fp,
                             _fp, _fp, _fp, _vp]),
     "ttt_linear_ln_bwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _f, _fp, _fp, _i, _i, _i, _i, _i,

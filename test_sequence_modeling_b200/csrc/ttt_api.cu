@@ -15,6 +15,7 @@
 #include "device_status.cuh"
 #include "backward.cuh"
 #include "decode.cuh"
+#include "momentum.cuh"
 #include "simt.cuh"
 #include "tc_linear.cuh"
 
@@ -22,6 +23,7 @@ namespace simt = ttt::simt;
 namespace tc = ttt::tc;
 namespace decode = ttt::decode;
 namespace bwd = ttt::bwd;
+namespace mom = ttt::mom;
 
 namespace {
 
@@ -408,6 +410,59 @@ int run_bwd(bool ln, const void *Q, const void *K, const void *V, int qkv_dtype,
   return TTT_OK;
 }
 
+int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int qkv_dtype,
+                     const float *eta, const float *alpha, const float *lambda, const float *W0,
+                     const float *gamma, const float *beta, float eps, int B, int H, int T, int d,
+                     int b, float *Z, float *W_out, float *S_out, void *stream) {
+  if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return TTT_ERR_ARG;
+  if (T % b != 0) return TTT_ERR_ARG;
+  if (ln && !(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
+  if (d != mom::D || b > mom::MAXB) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)B * H;
+  if (units == 0) return TTT_OK;
+  if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  const long long elems = units * T * d;
+  if (elems >= (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+  const bool tok = T > 0;
+  const void *req[] = {W0, W_out, S_out, ln ? (const void *)gamma : W0, ln ? (const void *)beta : W0,
+                       tok ? Q : W0, tok ? K : W0, tok ? V : W0, tok ? (const void *)eta : W0,
+                       tok ? (const void *)alpha : W0, tok ? (const void *)lambda : W0,
+                       tok ? (const void *)Z : W_out};
+  for (const void *x : req)
+    if (!x) return TTT_ERR_ARG;
+  for (const void *x : req)
+    if (!aligned16(x)) return TTT_ERR_ALIGN;
+  const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t ibytes = tok ? (size_t)elems * in_elt : 0, ebytes = tok ? (size_t)units * T * 4 : 0;
+  const size_t pbytes = ln ? (size_t)H * d * 4 : 0, wbytes = (size_t)units * d * d * 4;
+  Range ins[9] = {range_of(Q, ibytes),     range_of(K, ibytes),      range_of(V, ibytes),
+                  range_of(eta, ebytes),   range_of(alpha, ebytes),  range_of(lambda, ebytes),
+                  range_of(W0, (size_t)H * d * d * 4), range_of(gamma, pbytes), range_of(beta, pbytes)};
+  Range outs[3] = {range_of(Z, tok ? (size_t)elems * 4 : 0), range_of(W_out, wbytes),
+                   range_of(S_out, wbytes)};
+  for (int o = 0; o < 3; ++o) {
+    for (int i = 0; i < 9; ++i)
+      if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
+    for (int o2 = o + 1; o2 < 3; ++o2)
+      if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
+  }
+  mom::Params p{Q, K, V, eta, alpha, lambda, W0, gamma, beta, eps, H, T, b, Z, W_out, S_out};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = (unsigned)units;
+  const bool bf16 = qkv_dtype == TTT_BF16;
+  if (ln) {
+    if (bf16) mom::momentum_fwd_kernel<true, __nv_bfloat16><<<grid, mom::THREADS, 0, s>>>(p);
+    else mom::momentum_fwd_kernel<true, float><<<grid, mom::THREADS, 0, s>>>(p);
+  } else {
+    if (bf16) mom::momentum_fwd_kernel<false, __nv_bfloat16><<<grid, mom::THREADS, 0, s>>>(p);
+    else mom::momentum_fwd_kernel<false, float><<<grid, mom::THREADS, 0, s>>>(p);
+  }
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 int run(const Call &c) {
   const int st = validate(c);
   if (st != TTT_OK) return st;
@@ -518,6 +573,23 @@ int ttt_mlp_momentum_decode(const void *q, const void *k, const void *v, int qkv
                             int d, int hidden, int b, int pos, float *z, void *stream) {
   return run_mlp_decode(q, k, v, qkv_dtype, eta, W1, W2, W1_base, W2_base, ln_gamma, ln_beta, ln_eps,
                         B, H, d, hidden, b, pos, z, stream, true, alpha, lambda, S1, S2);
+}
+
+int ttt_linear_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                            const float *eta, const float *alpha, const float *lambda,
+                            const float *W0, int B, int H, int T, int d, int b, float *Z,
+                            float *W_out, float *S_out, void *stream) {
+  return run_momentum_fwd(false, Q, K, V, qkv_dtype, eta, alpha, lambda, W0, nullptr, nullptr, 1.f, B,
+                          H, T, d, b, Z, W_out, S_out, stream);
+}
+
+int ttt_linear_ln_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                               const float *eta, const float *alpha, const float *lambda,
+                               const float *W0, const float *ln_gamma, const float *ln_beta,
+                               float ln_eps, int B, int H, int T, int d, int b, float *Z,
+                               float *W_out, float *S_out, void *stream) {
+  return run_momentum_fwd(true, Q, K, V, qkv_dtype, eta, alpha, lambda, W0, ln_gamma, ln_beta, ln_eps,
+                          B, H, T, d, b, Z, W_out, S_out, stream);
 }
 
 int ttt_linear_bwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,

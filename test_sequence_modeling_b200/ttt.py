@@ -111,6 +111,39 @@ def ttt_mlp_fwd(Q, K, V, eta, W1, W2, gamma, beta, b, eps=1e-6, Z=None, W1_out=N
     return Z, W1_out, W2_out
 
 
+def ttt_linear_momentum_fwd(Q, K, V, eta, alpha, lam, W0, b, gamma=None, beta=None, eps=1e-6, Z=None,
+                            W_out=None, S_out=None, stream=None):
+    """Forward of TTT-Linear (with gamma and beta: TTT-Linear + LN) with the momentum and
+    decay update (see include/ttt.h).  alpha, lam [B,H,T] f32 like eta.  Returns
+    (Z [B,H,T,d], W_out [B,H,d,d], S_out [B,H,d,d]), all f32."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    ln = gamma is not None
+    for n, t in (("eta", eta), ("alpha", alpha), ("lam", lam)):
+        _cuda(t, n, torch.float32)
+        if tuple(t.shape) != (B, H, T):
+            raise ValueError(f"{n} must have shape {(B, H, T)}")
+    _cuda(W0, "W0", torch.float32)
+    if ln:
+        for n, t in (("gamma", gamma), ("beta", beta)):
+            _cuda(t, n, torch.float32)
+    Z = _out(Z, (B, H, T, d), Q.device, "Z")
+    W_out = _out(W_out, (B, H, d, d), Q.device, "W_out")
+    S_out = _out(S_out, (B, H, d, d), Q.device, "S_out")
+    with torch.cuda.device(Q.device):
+        if ln:
+            st = _lib.load().ttt_linear_ln_momentum_fwd(
+                _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(W0), _ptr(gamma),
+                _ptr(beta), float(eps), B, H, T, d, int(b), _ptr(Z), _ptr(W_out), _ptr(S_out),
+                _stream(stream, Q.device))
+        else:
+            st = _lib.load().ttt_linear_momentum_fwd(
+                _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(W0), B, H, T, d,
+                int(b), _ptr(Z), _ptr(W_out), _ptr(S_out), _stream(stream, Q.device))
+    check(st, "ttt_linear_ln_momentum_fwd" if ln else "ttt_linear_momentum_fwd")
+    return Z, W_out, S_out
+
+
 def ttt_linear_bwd(Q, K, V, eta, W0, dZ, b, dW_T=None, gamma=None, beta=None, eps=1e-6, stream=None):
     """Backward of ttt_linear_fwd (or, with gamma and beta, of ttt_linear_ln_fwd): the
     gradients of <dZ, Z> + <dW_T, W_T>.  dZ [B,H,T,d] f32, dW_T [B,H,d,d] f32 or None.

@@ -273,3 +273,34 @@ def test_backward_argument_errors(lib, ln):
         assert bwd(lib, ln, dg=None) == L.TTT_ERR_ARG
         assert bwd(lib, ln, db=p[15] + 16) == L.TTT_ERR_ARG  # dbeta overlaps dgamma
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
+
+
+def momentum_fwd(lib, ln=False, **kw):
+    q, k, v, eta, al, lm, w0, z, wo, so, g, bt = _ptrs(12)
+    a = dict(q=q, k=k, v=v, dt=L.TTT_BF16, eta=eta, al=al, lm=lm, w0=w0, g=g, bt=bt, eps=1e-6, B=2, H=3,
+             T=64, d=64, b=16, z=z, wo=wo, so=so)
+    a.update(kw)
+    head = (a["q"], a["k"], a["v"], a["dt"], a["eta"], a["al"], a["lm"], a["w0"])
+    tail = (a["B"], a["H"], a["T"], a["d"], a["b"], a["z"], a["wo"], a["so"], None)
+    if ln:
+        return lib.ttt_linear_ln_momentum_fwd(*head, a["g"], a["bt"], a["eps"], *tail)
+    return lib.ttt_linear_momentum_fwd(*head, *tail)
+
+
+@pytest.mark.parametrize("ln", [False, True])
+def test_momentum_forward_argument_errors(lib, ln):
+    n0 = lib.ttt_launch_count()
+    p = _ptrs(12)
+    assert momentum_fwd(lib, ln, b=32) == L.TTT_ERR_UNSUPPORTED
+    assert momentum_fwd(lib, ln, d=128) == L.TTT_ERR_UNSUPPORTED
+    assert momentum_fwd(lib, ln, T=40) == L.TTT_ERR_ARG
+    assert momentum_fwd(lib, ln, al=None) == L.TTT_ERR_ARG
+    assert momentum_fwd(lib, ln, so=None) == L.TTT_ERR_ARG
+    assert momentum_fwd(lib, ln, lm=A + 4) == L.TTT_ERR_ALIGN
+    assert momentum_fwd(lib, ln, so=p[8] + 256) == L.TTT_ERR_ARG    # S_out overlaps W_out
+    assert momentum_fwd(lib, ln, z=p[4] + 16) == L.TTT_ERR_ARG      # Z overlaps alpha
+    assert momentum_fwd(lib, ln, B=0) == L.TTT_OK
+    if ln:
+        assert momentum_fwd(lib, ln, eps=-1.0) == L.TTT_ERR_ARG
+        assert momentum_fwd(lib, ln, bt=None) == L.TTT_ERR_ARG
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
