@@ -20,6 +20,12 @@
 // of decode calls and this kernel agree to rounding.  HBM traffic is the inputs
 // and outputs once (about 650 B per token with bf16 q, k, v); the time is the
 // per-mini-batch chain of barriers.
+//
+// With MOMENTUM = false the same kernel runs the plain TTT rule
+// (W_t = W_{t-1} - eta_t k_t^T G_t, no S, alpha, lambda): the exact-fp32
+// CUDA-core forward of TTT-Linear (+ LN) for b <= 16.  Per token it computes
+// z_t = q_t W_t from the state itself rather than through the dual form's
+// masked Gram (the two are equal; see the mini-batch rule above).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,13 +42,13 @@ constexpr int THREADS = 256;
 
 struct Params {
   const void *Q, *K, *V;                    // [units][T][D]
-  const float *eta, *alpha, *lambda;        // [units][T]
+  const float *eta, *alpha, *lambda;        // [units][T] (alpha, lambda: MOMENTUM only)
   const float *W0;                          // [H][D][D]
   const float *gamma, *beta;                // [H][D] (LN)
   float eps;
   int H, T, b;
   float *Z;                                 // [units][T][D]
-  float *W_out, *S_out;                     // [units][D][D]
+  float *W_out, *S_out;                     // [units][D][D] (S_out: MOMENTUM only)
 };
 
 struct Smem {
@@ -52,7 +58,7 @@ struct Smem {
   float part[MAXB][4][D];    // per-quarter partial column sums: k_t W_base, then q_t W_t
 };
 
-template <bool LN, typename InT>
+template <bool LN, typename InT, bool MOMENTUM = true>
 __global__ void __launch_bounds__(THREADS) momentum_fwd_kernel(const Params p) {
   __shared__ Smem s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -72,12 +78,12 @@ __global__ void __launch_bounds__(THREADS) momentum_fwd_kernel(const Params p) {
     bet0 = p.beta[head * D + lane];
     bet1 = p.beta[head * D + lane + 32];
   }
-  float wb[16], w[16], sm[16];
+  float wb[16], w[16], sm[MOMENTUM ? 16 : 1];
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     wb[r] = p.W0[(long)head * D * D + (16 * rq + r) * D + j];
     w[r] = wb[r];
-    sm[r] = 0.f;
+    if (MOMENTUM) sm[r] = 0.f;
   }
 
   for (int n = 0; n < N; ++n) {
@@ -90,8 +96,10 @@ __global__ void __launch_bounds__(THREADS) momentum_fwd_kernel(const Params p) {
     }
     if (tid < b) {
       s.eta[tid] = p.eta[row0 + tid];
-      s.alpha[tid] = p.alpha[row0 + tid];
-      s.lambda[tid] = p.lambda[row0 + tid];
+      if (MOMENTUM) {
+        s.alpha[tid] = p.alpha[row0 + tid];
+        s.lambda[tid] = p.lambda[row0 + tid];
+      }
     }
     __syncthreads();
 
@@ -128,14 +136,18 @@ __global__ void __launch_bounds__(THREADS) momentum_fwd_kernel(const Params p) {
 #pragma unroll 1
     for (int t = 0; t < b; ++t) {
       const float gj = s.g[t][j];
-      const float al = s.alpha[t];
-      const float keep = 1.f - s.lambda[t];
+      const float al = MOMENTUM ? s.alpha[t] : 0.f;
+      const float keep = MOMENTUM ? 1.f - s.lambda[t] : 1.f;
       float zacc = 0.f;
 #pragma unroll
       for (int r = 0; r < 16; ++r) {
         const int i = 16 * rq + r;
-        sm[r] = fmaf(al, sm[r], -s.k[t][i] * gj);
-        w[r] = fmaf(keep, w[r], sm[r]);
+        if (MOMENTUM) {
+          sm[r] = fmaf(al, sm[r], -s.k[t][i] * gj);
+          w[r] = fmaf(keep, w[r], sm[r]);
+        } else {
+          w[r] = fmaf(-s.k[t][i], gj, w[r]);
+        }
         zacc = fmaf(s.q[t][i], w[r], zacc);
       }
       s.part[t][rq][j] = zacc;
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__(THREADS) momentum_fwd_kernel(const Params p) {
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     p.W_out[unit * D * D + (16 * rq + r) * D + j] = w[r];
-    p.S_out[unit * D * D + (16 * rq + r) * D + j] = sm[r];
+    if (MOMENTUM) p.S_out[unit * D * D + (16 * rq + r) * D + j] = sm[r];
   }
 }
 

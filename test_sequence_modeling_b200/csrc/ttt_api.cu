@@ -159,6 +159,22 @@ int run_simt(const Call &c) {
     return bf16 ? launch(simt::mlp_kernel<__nv_bfloat16>, grid, smem, s, p, simt::MLP_THREADS)
                 : launch(simt::mlp_kernel<float>, grid, smem, s, p, simt::MLP_THREADS);
   }
+  if (c.b <= mom::MAXB) {
+    // b <= 16: the state stays in registers for the whole sequence (the plain
+    // instantiation of the momentum kernel).
+    mom::Params q{c.Q, c.K, c.V, c.eta, nullptr, nullptr, c.W0, c.gamma, c.beta, c.eps,
+                  c.H, c.T, c.b, c.Z, c.W_out, nullptr};
+    if (c.kind == LINEAR_LN) {
+      if (bf16) mom::momentum_fwd_kernel<true, __nv_bfloat16, false><<<grid, mom::THREADS, 0, s>>>(q);
+      else mom::momentum_fwd_kernel<true, float, false><<<grid, mom::THREADS, 0, s>>>(q);
+    } else {
+      if (bf16) mom::momentum_fwd_kernel<false, __nv_bfloat16, false><<<grid, mom::THREADS, 0, s>>>(q);
+      else mom::momentum_fwd_kernel<false, float, false><<<grid, mom::THREADS, 0, s>>>(q);
+    }
+    if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return TTT_OK;
+  }
   const size_t smem = simt::linear_smem_bytes(c.b);
   if (c.kind == LINEAR_LN)
     return bf16 ? launch(simt::linear_kernel<true, __nv_bfloat16>, grid, smem, s, p)
