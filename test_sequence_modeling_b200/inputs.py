@@ -17,6 +17,11 @@ Distributions (the five workloads of the TTT layer forward):
   gamma    ~ 1 + N(0, 0.01^2), beta ~ N(0, 0.01^2), one per head.
 Draw order within a unit stream: Q, K, V, eta noise.  Within a head stream:
 W0 (or W1 then W2), gamma, beta.
+
+Two more streams serve the widened paths: ``default_rng([seed, 3, s])`` draws the
+momentum factors alpha ~ U[0, 0.9) and weight decays lambda ~ U[0, 0.05) of the
+momentum and decay update, and ``default_rng([seed, 4, s])`` the incoming
+gradients dZ ~ N(0, 1/d), dW_T ~ N(0, 1/d^2) of the backward pass.
 """
 from __future__ import annotations
 
