@@ -1,8 +1,10 @@
-"""TTT layer forward (mini-batch TTT, dual form) on NVIDIA B200, sm_100a.
+"""TTT layers (mini-batch TTT) on NVIDIA B200, sm_100a: the dual-form forward of
+TTT-Linear, TTT-Linear + LN and TTT-MLP, its backward (TTT-Linear, + LN), the
+primal-form decode step, and the momentum and decay (Titans-style) update.
 
 The computation lives in ``libttt.so`` (C ABI in ``include/ttt.h``); the
 functions below are its Python binding over torch CUDA tensors.  ``inputs``
-holds the seeded synthetic workloads.
+holds the seeded synthetic workloads; ``host`` the forward over host buffers.
 """
 from ._lib import (TTT_BF16, TTT_ERR_TIMEOUT, TTT_F32, TTT_OK, TTT_PATH_AUTO,  # noqa: F401
                    TTT_PATH_SIMT, TTT_PATH_TC, TTTError)

@@ -1,4 +1,5 @@
-"""Python binding of the TTT layer forward: marshals torch CUDA tensors into the C ABI.
+"""Python binding of the TTT layer library (forward, backward, decode, momentum and
+decay variants): marshals torch CUDA tensors into the C ABI.
 
 Every step of the computation runs in the CUDA kernels of libttt.so; this module
 only checks shapes and dtypes, allocates outputs when the caller passes none,
