@@ -76,5 +76,45 @@ def test_unmutated_copy_passes(source, tmp_path):
     src = tmp_path / "same.c"
     src.write_text(source)
     orc = oracle.Oracle(oracle.load(oracle.build(str(src), str(tmp_path / "libsame.so"), force=True)))
-    for _, pin in all_pins():
+    from test_oracle_momentum import momentum_pins
+    for _, pin in all_pins() + momentum_pins():
         pin(orc)
+
+
+MOMENTUM_MUTANTS = {
+    "momentum without alpha": ("S[p] = alpha[t] * S[p] - eta[t] * grad[p];", "S[p] = S[p] - eta[t] * grad[p];"),
+    "decay applied to the momentum": ("W[p] = (1.0 - lam[t]) * W[p] + S[p];",
+                                      "W[p] = W[p] + (1.0 - lam[t]) * S[p];"),
+    "momentum gradient at the current state": (
+        "    if (t % b == 0) memcpy(Wbase, W, sizeof(double) * P);\n"
+        "    const double *k = K + (long)t * d, *v = V + (long)t * d, *q = Q + (long)t * d;\n"
+        "    model_loss_grad(m, Wbase, k, v, grad, &sc);\n"
+        "    for (long p = 0; p < P; ++p) {\n      S[p]",
+        "    memcpy(Wbase, W, sizeof(double) * P);\n"
+        "    const double *k = K + (long)t * d, *v = V + (long)t * d, *q = Q + (long)t * d;\n"
+        "    model_loss_grad(m, Wbase, k, v, grad, &sc);\n"
+        "    for (long p = 0; p < P; ++p) {\n      S[p]"),
+    "decay of the previous token": ("W[p] = (1.0 - lam[t]) * W[p] + S[p];",
+                                    "W[p] = (1.0 - lam[t > 0 ? t - 1 : 0]) * W[p] + S[p];"),
+    "state updated with the previous momentum": (
+        "      S[p] = alpha[t] * S[p] - eta[t] * grad[p];\n      W[p] = (1.0 - lam[t]) * W[p] + S[p];",
+        "      W[p] = (1.0 - lam[t]) * W[p] + S[p];\n      S[p] = alpha[t] * S[p] - eta[t] * grad[p];"),
+}
+
+
+@pytest.mark.parametrize("name", list(MOMENTUM_MUTANTS))
+def test_momentum_mutant_is_caught(name, source, tmp_path):
+    """The same for the momentum and decay variant, against its own pins."""
+    from test_oracle_momentum import momentum_pins
+    old, new = MOMENTUM_MUTANTS[name]
+    assert source.count(old) == 1, f"anchor for '{name}' not unique in the oracle source"
+    src = tmp_path / "mutant.c"
+    src.write_text(source.replace(old, new, 1))
+    orc = oracle.Oracle(oracle.load(oracle.build(str(src), str(tmp_path / "libmutant.so"), force=True)))
+    caught = []
+    for pin_name, pin in momentum_pins():
+        try:
+            pin(orc)
+        except (AssertionError, ValueError):
+            caught.append(pin_name)
+    assert caught, f"mutant '{name}' passes every momentum pin"
