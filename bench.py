@@ -127,6 +127,13 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
             text, _ = self.proc.communicate()
+        return self.summarize(text)
+
+    @staticmethod
+    def summarize(text):
+        """Median SM clock under load, the max clock, the throttle reasons seen, and a
+        verdict: "rejected: ..." for a hardware or thermal slowdown, or for an SM clock
+        well below max with no reason (a leftover clock lock); sw_power_cap is kept."""
         rows = [r.split(", ") for r in text.strip().splitlines() if r.count(",") >= 8]
         if not rows:
             return None
@@ -135,8 +142,16 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip() == "Active"})
         loaded = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+        info = {"sm_mhz": statistics.median(loaded) if loaded else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        bad = [r for r in reasons if r != "sw_power_cap"]
+        if bad:
+            info["verdict"] = "rejected: " + ", ".join(bad)
+        elif not reasons and info["sm_mhz"] and info["sm_max_mhz"] and info["sm_mhz"] < 0.85 * info["sm_max_mhz"]:
+            info["verdict"] = "rejected: SM clock well below max with no reason"
+        else:
+            info["verdict"] = "ok"
+        return info
 
 
 def gpu_id_for(torch, device) -> str | None:
