@@ -28,6 +28,15 @@ def _cuda(t, name, dtype=None):
     return t
 
 
+def _shaped(t, name, shape):
+    """A float32 CUDA tensor of exactly this shape: the C ABI reads plain pointers, so
+    a size mismatch has to be caught here."""
+    _cuda(t, name, torch.float32)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
 def _qkv(Q, K, V):
     for n, t in (("Q", Q), ("K", K), ("V", V)):
         _cuda(t, n)
@@ -65,8 +74,8 @@ def ttt_linear_fwd(Q, K, V, eta, W0, b, Z=None, W_out=None, stream=None):
     Returns (Z [B,H,T,d] f32, W_out [B,H,d,d] f32)."""
     dt = _qkv(Q, K, V)
     B, H, T, d = Q.shape
-    _cuda(eta, "eta", torch.float32)
-    _cuda(W0, "W0", torch.float32)
+    _shaped(eta, "eta", (B, H, T))
+    _shaped(W0, "W0", (H, d, d))
     Z = _out(Z, (B, H, T, d), Q.device, "Z")
     W_out = _out(W_out, (B, H, d, d), Q.device, "W_out")
     with torch.cuda.device(Q.device):
@@ -80,8 +89,9 @@ def ttt_linear_ln_fwd(Q, K, V, eta, W0, gamma, beta, b, eps=1e-6, Z=None, W_out=
     """TTT-Linear with LN + residual.  gamma, beta [H,d] f32."""
     dt = _qkv(Q, K, V)
     B, H, T, d = Q.shape
-    for n, t in (("eta", eta), ("W0", W0), ("gamma", gamma), ("beta", beta)):
-        _cuda(t, n, torch.float32)
+    for n, t, shp in (("eta", eta, (B, H, T)), ("W0", W0, (H, d, d)), ("gamma", gamma, (H, d)),
+                      ("beta", beta, (H, d))):
+        _shaped(t, n, shp)
     Z = _out(Z, (B, H, T, d), Q.device, "Z")
     W_out = _out(W_out, (B, H, d, d), Q.device, "W_out")
     with torch.cuda.device(Q.device):
@@ -97,9 +107,11 @@ def ttt_mlp_fwd(Q, K, V, eta, W1, W2, gamma, beta, b, eps=1e-6, Z=None, W1_out=N
     """TTT-MLP forward.  W1 [H,d,h], W2 [H,h,d] f32.  Returns (Z, W1_out, W2_out)."""
     dt = _qkv(Q, K, V)
     B, H, T, d = Q.shape
-    for n, t in (("eta", eta), ("W1", W1), ("W2", W2), ("gamma", gamma), ("beta", beta)):
-        _cuda(t, n, torch.float32)
+    _cuda(W1, "W1", torch.float32)
     hidden = W1.shape[-1]
+    for n, t, shp in (("eta", eta, (B, H, T)), ("W1", W1, (H, d, hidden)), ("W2", W2, (H, hidden, d)),
+                      ("gamma", gamma, (H, d)), ("beta", beta, (H, d))):
+        _shaped(t, n, shp)
     Z = _out(Z, (B, H, T, d), Q.device, "Z")
     W1_out = _out(W1_out, (B, H, d, hidden), Q.device, "W1_out")
     W2_out = _out(W2_out, (B, H, hidden, d), Q.device, "W2_out")
@@ -124,10 +136,10 @@ def ttt_linear_momentum_fwd(Q, K, V, eta, alpha, lam, W0, b, gamma=None, beta=No
         _cuda(t, n, torch.float32)
         if tuple(t.shape) != (B, H, T):
             raise ValueError(f"{n} must have shape {(B, H, T)}")
-    _cuda(W0, "W0", torch.float32)
+    _shaped(W0, "W0", (H, d, d))
     if ln:
         for n, t in (("gamma", gamma), ("beta", beta)):
-            _cuda(t, n, torch.float32)
+            _shaped(t, n, (H, d))
     Z = _out(Z, (B, H, T, d), Q.device, "Z")
     W_out = _out(W_out, (B, H, d, d), Q.device, "W_out")
     S_out = _out(S_out, (B, H, d, d), Q.device, "S_out")
@@ -153,18 +165,16 @@ def ttt_linear_bwd(Q, K, V, eta, W0, dZ, b, dW_T=None, gamma=None, beta=None, ep
     dt = _qkv(Q, K, V)
     B, H, T, d = Q.shape
     ln = gamma is not None
-    _cuda(eta, "eta", torch.float32)
-    _cuda(W0, "W0", torch.float32)
-    _cuda(dZ, "dZ", torch.float32)
-    if tuple(dZ.shape) != (B, H, T, d):
-        raise ValueError(f"dZ must have shape {(B, H, T, d)}")
+    _shaped(eta, "eta", (B, H, T))
+    _shaped(W0, "W0", (H, d, d))
+    _shaped(dZ, "dZ", (B, H, T, d))
     if dW_T is not None:
         _cuda(dW_T, "dW_T", torch.float32)
         if tuple(dW_T.shape) != (B, H, d, d):
             raise ValueError(f"dW_T must have shape {(B, H, d, d)}")
     if ln:
         for n, t in (("gamma", gamma), ("beta", beta)):
-            _cuda(t, n, torch.float32)
+            _shaped(t, n, (H, d))
     if b <= 0 or T % b:
         raise ValueError("T must be a multiple of b")
     dev = Q.device
@@ -226,7 +236,7 @@ def ttt_linear_ln_decode(q, k, v, eta, W, W_base, gamma, beta, b, pos, eps=1e-6,
     """One primal-form decode step of TTT-Linear with LN + residual; gamma, beta [H,d] f32."""
     dt, B, H, d, z = _decode_args(q, k, v, eta, W, W_base, z)
     for n, t in (("gamma", gamma), ("beta", beta)):
-        _cuda(t, n, torch.float32)
+        _shaped(t, n, (H, d))
     with torch.cuda.device(q.device):
         st = _lib.load().ttt_linear_ln_decode(_ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta), _ptr(W),
                                               _ptr(W_base), _ptr(gamma), _ptr(beta), float(eps), B, H,
@@ -265,7 +275,7 @@ def ttt_linear_ln_momentum_decode(q, k, v, eta, alpha, lam, W, W_base, S, gamma,
     dt, B, H, d, z = _decode_args(q, k, v, eta, W, W_base, z)
     _momentum_args(B, H, d, alpha, lam, S)
     for n, t in (("gamma", gamma), ("beta", beta)):
-        _cuda(t, n, torch.float32)
+        _shaped(t, n, (H, d))
     with torch.cuda.device(q.device):
         st = _lib.load().ttt_linear_ln_momentum_decode(
             _ptr(q), _ptr(k), _ptr(v), dt, _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(W), _ptr(W_base),
@@ -320,14 +330,14 @@ def _mlp_decode_args(q, k, v, eta, W1, W2, W1_base, W2_base, gamma, beta, z):
         raise ValueError("q, k, v must have the same shape [B, H, d]")
     B, H, d = q.shape
     hidden = W1.shape[-1]
-    _cuda(eta, "eta", torch.float32)
+    _shaped(eta, "eta", (B, H))
     for n, t, shp in (("W1", W1, (B, H, d, hidden)), ("W1_base", W1_base, (B, H, d, hidden)),
                       ("W2", W2, (B, H, hidden, d)), ("W2_base", W2_base, (B, H, hidden, d))):
         _cuda(t, n, torch.float32)
         if tuple(t.shape) != shp:
             raise ValueError(f"{n} must have shape {shp}")
     for n, t in (("gamma", gamma), ("beta", beta)):
-        _cuda(t, n, torch.float32)
+        _shaped(t, n, (H, d))
     z = _out(z, (B, H, d), q.device, "z")
     return _QKV_DTYPES[q.dtype], B, H, d, hidden, z
 
