@@ -299,6 +299,9 @@ def main():
                     help="the decode step with the momentum and decay update (TTT-Linear + LN, or with "
                          "--decode-mlp TTT-MLP)")
     args = ap.parse_args()
+    single = args.backward or args.momentum or args.decode or args.decode_mlp or args.decode_momentum
+    if single and int(os.environ.get("RANK", "0")) != 0:
+        return 0  # these lines are measured on one GPU: under a multi-rank launch only rank 0 runs
     if args.backward:
         return run_backward(args)
     if args.momentum:

@@ -45,3 +45,14 @@ def test_reference_arm_two_ranks_prints_once():
     lines = _json_lines(r.stdout)
     assert len(lines) == 1
     _check(lines[0], 2)
+
+
+def test_single_gpu_lines_leave_other_ranks_idle():
+    """--backward, --momentum and the decode lines are measured on one GPU: a rank
+    other than 0 exits at once, printing nothing and touching no device."""
+    for flag in ("--backward", "--momentum", "--decode", "--decode-mlp", "--decode-momentum"):
+        env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+        r = subprocess.run([sys.executable, "bench.py", flag, "--steps", "1", "--warmup", "0"], cwd=ROOT,
+                           capture_output=True, text=True, timeout=300, env=env)
+        assert r.returncode == 0, (flag, r.stderr[-1000:])
+        assert _json_lines(r.stdout) == [], flag
