@@ -171,6 +171,45 @@ TTT_API int ttt_linear_ln_bwd(const void *Q, const void *K, const void *V, int q
                               float *dbeta, float *W_ckpt, void *stream);
 
 /*
+ * The backward of TTT-Linear + LN (ttt_linear_ln_bwd) for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is a property of
+ * the library's interface, not of the method.
+ *
+ * Who needs it: code that runs under a device allocator it does not own and may
+ * not call cudaMalloc itself -- an operator hosted inside another framework or
+ * runtime that hands out only its own buffers, or a serving process that
+ * reserves all device memory at start-up, where a later cudaMalloc can fail or
+ * stall the device -- and that has no way to pass the extra workspace
+ * ttt_linear_ln_bwd asks for.  Here the per-mini-batch states that the reverse
+ * pass reads back (W_ckpt of ttt_linear_ln_bwd) live in one fixed array of
+ * device memory inside the library instead.
+ *
+ * Arguments, layouts, outputs and errors are those of ttt_linear_ln_bwd without
+ * W_ckpt; the outputs are identical to that entry point's.  Limits and rules:
+ *   - B * H * (T / b) <= TTT_NOALLOC_BWD_MAX_STATES (4096 states of d x d fp32,
+ *     a 64 MiB array).  A larger call returns TTT_ERR_UNSUPPORTED before
+ *     anything is enqueued.  Every GPU that loads the library holds the array
+ *     until the process exits.
+ *   - The array is shared by every call on a device and keeps the last call's
+ *     contents.  A call writes every state before it reads it, so nothing needs
+ *     clearing, but calls whose kernels overlap on the GPU (different streams,
+ *     or different host threads, without an ordering between them) race on it:
+ *     order them on one stream or with events.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address once and keeps it; make that first call before
+ *     any stream capture.  The lookup follows the size checks and precedes the
+ *     pointer checks; it returns TTT_ERR_CUDA if it fails.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define TTT_NOALLOC_BWD_MAX_STATES 4096
+TTT_API int ttt_linear_ln_bwd_noalloc(const void *Q, const void *K, const void *V, int qkv_dtype,
+                                      const float *eta, const float *W0, const float *ln_gamma,
+                                      const float *ln_beta, float ln_eps, const float *dZ,
+                                      const float *dW_T, int B, int H, int T, int d, int b,
+                                      float *dQ, float *dK, float *dV, float *deta, float *dW0,
+                                      float *dgamma, float *dbeta, void *stream);
+
+/*
  * Primal-form decode step (generation, §04.3 of the TTT write-up: decoding is
  * sequential and takes the primal form): one token per (batch, head) and call,
  * with the state carried in device memory across calls.

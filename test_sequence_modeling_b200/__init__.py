@@ -17,7 +17,8 @@ def __getattr__(name):
                 "last_device_status", "launch_count", "debug_inject_timeout",
                 "ttt_linear_decode", "ttt_linear_ln_decode", "ttt_mlp_decode",
                 "ttt_linear_momentum_decode", "ttt_linear_ln_momentum_decode",
-                "ttt_mlp_momentum_decode", "ttt_linear_bwd", "ttt_linear_momentum_fwd"):
+                "ttt_mlp_momentum_decode", "ttt_linear_bwd", "ttt_linear_momentum_fwd",
+                "ttt_linear_ln_bwd_noalloc"):
         from . import ttt
         return getattr(ttt, name)
     raise AttributeError(name)

@@ -11,6 +11,8 @@ TTT_OK, TTT_ERR_ARG, TTT_ERR_ALIGN, TTT_ERR_UNSUPPORTED, TTT_ERR_CUDA, TTT_ERR_T
     0, -1, -2, -3, -4, -5)
 TTT_F32, TTT_BF16 = 0, 1
 TTT_PATH_AUTO, TTT_PATH_SIMT, TTT_PATH_TC = 0, 1, 2
+# Capacity of ttt_linear_ln_bwd_noalloc's built-in state array (d x d fp32 states).
+TTT_NOALLOC_BWD_MAX_STATES = 4096
 
 _vp, _fp, _i, _f = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 
@@ -33,6 +35,8 @@ SIGNATURES = {
                             _fp, _fp, _fp, _vp]),
     "ttt_linear_ln_bwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _f, _fp, _fp, _i, _i, _i, _i, _i,
                                _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _vp]),
+    "ttt_linear_ln_bwd_noalloc": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _f, _fp, _fp, _i, _i, _i, _i,
+                                       _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _vp]),
     "ttt_linear_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _i, _i, _i, _i, _i, _fp, _vp]),
     "ttt_linear_ln_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i, _i, _i,
                                   _fp, _vp]),

@@ -6,6 +6,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -634,3 +635,77 @@ int ttt_linear_ln_decode(const void *q, const void *k, const void *v, int qkv_dt
 }
 
 }  // extern "C"
+
+// ---- Backward of TTT-Linear + LN without any allocation -------------------------
+//
+// For callers that cannot call cudaMalloc (an operator hosted by a framework
+// that owns the device allocator, or a process that reserves all device memory
+// up front): the per-mini-batch states that the backward's reverse pass reads
+// back live in one fixed device array of this library instead of a caller
+// workspace.  Every device that loads the library holds the array (64 MiB)
+// until the process exits; calls on a device share it, so calls that overlap
+// on the GPU race on it.  A call writes each state before reading it, so the
+// array never needs clearing.
+namespace ttt {
+namespace noalloc {
+
+constexpr long long MAX_STATES = TTT_NOALLOC_BWD_MAX_STATES;  // d x d fp32 states
+static __device__ __align__(256) float g_bwd_states[MAX_STATES * 64 * 64];
+
+}  // namespace noalloc
+}  // namespace ttt
+
+namespace {
+
+constexpr int kNoAllocMaxDevices = 256;
+std::mutex g_noalloc_mu;
+std::atomic<float *> g_noalloc_states[kNoAllocMaxDevices];
+
+// The device address of the state array on the current device, looked up once
+// per device.  In host code the array's name denotes a host-side stand-in, not
+// device memory, so only this address may be handed to a kernel.
+int noalloc_states(float **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return TTT_ERR_CUDA;
+  if (dev >= kNoAllocMaxDevices) return TTT_ERR_UNSUPPORTED;
+  float *ptr = g_noalloc_states[dev].load(std::memory_order_acquire);
+  if (!ptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    ptr = g_noalloc_states[dev].load(std::memory_order_relaxed);
+    if (!ptr) {
+      void *addr = nullptr;
+      if (cudaGetSymbolAddress(&addr, ttt::noalloc::g_bwd_states) != cudaSuccess || !addr)
+        return TTT_ERR_CUDA;
+      ptr = static_cast<float *>(addr);
+      g_noalloc_states[dev].store(ptr, std::memory_order_release);
+    }
+  }
+  *out = ptr;
+  return TTT_OK;
+}
+
+}  // namespace
+
+extern "C" int ttt_linear_ln_bwd_noalloc(const void *Q, const void *K, const void *V,
+                                         int qkv_dtype, const float *eta, const float *W0,
+                                         const float *ln_gamma, const float *ln_beta, float ln_eps,
+                                         const float *dZ, const float *dW_T, int B, int H, int T,
+                                         int d, int b, float *dQ, float *dK, float *dV,
+                                         float *deta, float *dW0, float *dgamma, float *dbeta,
+                                         void *stream) {
+  // The size checks of the backward, then the array's capacity, all before the
+  // one-time address lookup; the pointer checks follow in run_bwd.
+  if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0 || T % b != 0) return TTT_ERR_ARG;
+  if (!(std::isfinite(ln_eps) && ln_eps > 0.f)) return TTT_ERR_ARG;
+  if (d != bwd::D || b > bwd::MAXB) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)B * H;
+  if (units == 0) return TTT_OK;
+  if (units > ttt::noalloc::MAX_STATES || units * (T / b) > ttt::noalloc::MAX_STATES)
+    return TTT_ERR_UNSUPPORTED;
+  float *states = nullptr;
+  const int st = noalloc_states(&states);
+  if (st != TTT_OK) return st;
+  return run_bwd(true, Q, K, V, qkv_dtype, eta, W0, ln_gamma, ln_beta, ln_eps, dZ, dW_T, B, H, T, d,
+                 b, dQ, dK, dV, deta, dW0, dgamma, dbeta, states, stream);
+}

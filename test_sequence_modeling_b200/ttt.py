@@ -201,6 +201,42 @@ def ttt_linear_bwd(Q, K, V, eta, W0, dZ, b, dW_T=None, gamma=None, beta=None, ep
     return out
 
 
+def ttt_linear_ln_bwd_noalloc(Q, K, V, eta, W0, dZ, b, gamma, beta, eps=1e-6, dW_T=None, out=None,
+                              stream=None):
+    """The backward of ttt_linear_ln_fwd for callers that must not allocate device
+    memory: the states its reverse pass reads back stay in the library's own fixed
+    array (B*H*T/b <= TTT_NOALLOC_BWD_MAX_STATES), so no W_ckpt is returned.  Pass
+    preallocated outputs in `out` (dQ, dK, dV, deta, dW0, dgamma, dbeta) to keep the
+    call free of allocation on this side too.  Calls whose kernels overlap on the
+    GPU share that array and race; the first call on a device looks its address up
+    and should come before any stream capture."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    _shaped(eta, "eta", (B, H, T))
+    _shaped(W0, "W0", (H, d, d))
+    _shaped(dZ, "dZ", (B, H, T, d))
+    for n, t in (("gamma", gamma), ("beta", beta)):
+        _shaped(t, n, (H, d))
+    if dW_T is not None:
+        _shaped(dW_T, "dW_T", (B, H, d, d))
+    if b <= 0 or T % b:
+        raise ValueError("T must be a multiple of b")
+    dev = Q.device
+    shapes = {"dQ": (B, H, T, d), "dK": (B, H, T, d), "dV": (B, H, T, d), "deta": (B, H, T),
+              "dW0": (B, H, d, d), "dgamma": (B, H, d), "dbeta": (B, H, d)}
+    out = dict(out or {})
+    for n, shp in shapes.items():
+        out[n] = _out(out.get(n), shp, dev, n)
+    o = {k: _ptr(v) for k, v in out.items()}
+    with torch.cuda.device(dev):
+        st = _lib.load().ttt_linear_ln_bwd_noalloc(
+            _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W0), _ptr(gamma), _ptr(beta), float(eps),
+            _ptr(dZ), _ptr(dW_T), B, H, T, d, int(b), o["dQ"], o["dK"], o["dV"], o["deta"], o["dW0"],
+            o["dgamma"], o["dbeta"], _stream(stream, dev))
+    check(st, "ttt_linear_ln_bwd_noalloc")
+    return out
+
+
 def _decode_args(q, k, v, eta, W, W_base, z):
     for n, t in (("q", q), ("k", k), ("v", v)):
         _cuda(t, n)

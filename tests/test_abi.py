@@ -304,3 +304,24 @@ def test_momentum_forward_argument_errors(lib, ln):
         assert momentum_fwd(lib, ln, eps=-1.0) == L.TTT_ERR_ARG
         assert momentum_fwd(lib, ln, bt=None) == L.TTT_ERR_ARG
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
+
+
+def test_noalloc_backward_checks_sizes_before_any_cuda_call(lib):
+    """ttt_linear_ln_bwd_noalloc rejects a call whose states exceed its built-in
+    array, and malformed sizes, on the host (fake pointers are never touched)."""
+    p = _ptrs(14)
+
+    def call(B, H, T, b=16, d=64, eps=1e-6, dt=L.TTT_BF16):
+        return lib.ttt_linear_ln_bwd_noalloc(p[0], p[1], p[2], dt, p[3], p[4], p[5], p[6], eps, p[7],
+                                             None, B, H, T, d, b, p[8], p[9], p[10], p[11], p[12],
+                                             p[13], p[13] + (1 << 29), None)
+
+    cap = L.TTT_NOALLOC_BWD_MAX_STATES
+    assert call(4, 32, 16 * cap // 128 + 16) == L.TTT_ERR_UNSUPPORTED  # one mini-batch too many
+    assert call(cap + 1, 1, 16) == L.TTT_ERR_UNSUPPORTED
+    assert call(2, 3, 40) == L.TTT_ERR_ARG                  # T % b != 0
+    assert call(2, 3, 48, eps=0.0) == L.TTT_ERR_ARG
+    assert call(2, 3, 48, dt=7) == L.TTT_ERR_ARG
+    assert call(2, 3, 48, d=32) == L.TTT_ERR_UNSUPPORTED
+    assert call(2, 3, 64, b=32) == L.TTT_ERR_UNSUPPORTED
+    assert call(0, 3, 48) == L.TTT_OK                       # no units: nothing to do
