@@ -207,6 +207,15 @@ __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // ---- tcgen05.mma ------------------------------------------------------------------
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled canonical layout.
@@ -224,6 +233,21 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t start, uint32_t lbo
   return d;
 }
 
+// Descriptor of an MN-major operand of 32-bit elements in the "128-byte swizzle
+// with 32-byte base" layout (the only MN-major layout for kind::tf32): rows of
+// 128 bytes (32 elements along MN), the four 32-byte granules of row r stored
+// at granule index g ^ (r % 4); lbo = distance between 32-element MN blocks,
+// sbo = distance between 4-row K groups.
+__device__ __forceinline__ uint64_t smem_desc_sw128_b32(uint32_t start, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((start >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= (uint64_t)1 << 61;  // 128-byte swizzle, 32-byte base
+  return d;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B and an fp32 accumulator.
 // a_mn / b_mn: operand is MN-major (else K-major); neg_a: D += (-A) B.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, bool b_mn,
@@ -236,6 +260,50 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
          | ((b_mn ? 1u : 0u) << 16)        // B major
          | ((uint32_t)(N >> 3) << 17)      // N / 8
          | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
+// Instruction descriptor of kind::tf32 (fp32 containers read as tf32) with an
+// fp32 accumulator; a_mn / b_mn: operand is MN-major (else K-major); neg_a:
+// D += (-A) B.
+__host__ __device__ constexpr uint32_t idesc_tf32_f32(int M, int N, bool a_mn, bool b_mn,
+                                                      bool neg_a) {
+  return (1u << 4)                         // D format: f32
+         | (2u << 7)                       // A format: tf32
+         | (2u << 10)                      // B format: tf32
+         | ((neg_a ? 1u : 0u) << 13)       // negate A
+         | ((a_mn ? 1u : 0u) << 15)        // A major
+         | ((b_mn ? 1u : 0u) << 16)        // B major
+         | ((uint32_t)(N >> 3) << 17)      // N / 8
+         | ((uint32_t)(M >> 4) << 24);     // M / 16
+}
+
+// kind::tf32 products (K = 8 per instruction): both operands from shared
+// memory, or A from tensor memory (one fp32 element per column).
+__device__ __forceinline__ void umma_ss_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_tf32(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
+// Rounds an fp32 value to tf32 (nearest, ties away from zero), returned as an
+// fp32 bit pattern whose 13 low mantissa bits are zero.
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
 }
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]; issued by one thread.

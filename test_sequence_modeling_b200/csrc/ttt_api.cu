@@ -19,9 +19,11 @@
 #include "momentum.cuh"
 #include "simt.cuh"
 #include "tc_linear.cuh"
+#include "tc_mlp.cuh"
 
 namespace simt = ttt::simt;
 namespace tc = ttt::tc;
+namespace tcmlp = ttt::tcmlp;
 namespace decode = ttt::decode;
 namespace bwd = ttt::bwd;
 namespace mom = ttt::mom;
@@ -215,7 +217,8 @@ bool make_qkv_map(CUtensorMap *map, const void *base, int T, long long units, in
 }
 
 bool tc_supported(const Call &c) {
-  return c.kind != MLP_LN && c.qkv_dtype == TTT_BF16 && c.b == tc::MB && c.T > 0;
+  if (c.qkv_dtype != TTT_BF16 || c.T <= 0) return false;
+  return c.kind == MLP_LN ? c.b == tcmlp::MB : c.b == tc::MB;
 }
 
 template <bool LN>
@@ -246,6 +249,37 @@ int launch_linear_tc(const Call &c) {
     return TTT_ERR_CUDA;
   kernel<<<(unsigned)units, tc::THREADS, tc::SMEM_BYTES, static_cast<cudaStream_t>(c.stream)>>>(
       mq, mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
+int launch_mlp_tc(const Call &c) {
+  const long long units = (long long)c.B * c.H;
+  CUtensorMap mq, mk, mv;
+  if (!make_qkv_map(&mq, c.Q, c.T, units, tcmlp::CHUNK) ||
+      !make_qkv_map(&mk, c.K, c.T, units, tcmlp::CHUNK) ||
+      !make_qkv_map(&mv, c.V, c.T, units, tcmlp::CHUNK))
+    return TTT_ERR_CUDA;
+  tcmlp::Params p;
+  p.eta = c.eta;
+  p.W1_0 = c.W0;
+  p.W2_0 = c.W2_0;
+  p.gamma = c.gamma;
+  p.beta = c.beta;
+  p.eps = c.eps;
+  p.H = c.H;
+  p.T = c.T;
+  p.Z = c.Z;
+  p.W1_out = c.W_out;
+  p.W2_out = c.W2_out;
+  p.inject_timeout = g_inject_timeout.load();
+  auto kernel = tcmlp::mlp_tc_kernel;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)tcmlp::SMEM_BYTES) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  kernel<<<(unsigned)units, tcmlp::THREADS, tcmlp::SMEM_BYTES,
+           static_cast<cudaStream_t>(c.stream)>>>(mq, mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return TTT_OK;
@@ -487,8 +521,10 @@ int run(const Call &c) {
   const int path = g_path.load();
   const bool tc_ok = tc_supported(c);
   if (path == TTT_PATH_TC && !tc_ok) return TTT_ERR_UNSUPPORTED;
-  if (path != TTT_PATH_SIMT && tc_ok)
+  if (path != TTT_PATH_SIMT && tc_ok) {
+    if (c.kind == MLP_LN) return launch_mlp_tc(c);
     return c.kind == LINEAR_LN ? launch_linear_tc<true>(c) : launch_linear_tc<false>(c);
+  }
   return run_simt(c);
 }
 

@@ -43,12 +43,15 @@ class HostForward:
     def run(self, Q, K, V, eta, params, b, eps, Z, W_outs, after=None):
         """params: the per-head inputs on the host (W0; or W0, gamma, beta; or W1,
         W2, gamma, beta), copied with the first chunk.  Z, W_outs: host outputs.
-        ``after``: an event the first copy waits for (the start of a timed region)."""
+        ``after``: an event the first copy waits for (the start of a timed region).
+        The first copy also waits for the previous call's last copy back, so that
+        back-to-back calls never overwrite device buffers still in use."""
         dq, dk, dv = self.d_qkv
         P = self.d_params
         for i, (b0, b1) in enumerate(self.slices):
             with torch.cuda.stream(self.s_in):
                 if i == 0:
+                    self.s_in.wait_event(self.done)  # no-op before the first call
                     if after is not None:
                         self.s_in.wait_event(after)
                     for dst, src in zip(self.d_params, params):

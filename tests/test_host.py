@@ -35,3 +35,30 @@ def test_host_forward_equals_device_forward(name, chunks):
     assert np.array_equal(Z.numpy(), ref["Z"])
     for k, o in zip(keys, outs):
         assert np.array_equal(o.numpy(), ref[k]), k
+
+
+def test_back_to_back_calls_do_not_overlap():
+    """Two calls in a row on different inputs (no event passed between them): each
+    output equals the device forward of its own inputs."""
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=6, H=4, T=256)
+    runs = []
+    for seed in (11, 12):
+        c = cfg.replace(seed=seed)
+        dev = to_device(c, I.make_inputs(c))
+        runs.append((dev, run_gpu(c, dev)))
+    fwd = None
+    outs = []
+    for dev, _ in runs:
+        host = {k: v.cpu().pin_memory() for k, v in dev.items()}
+        params = [host["W0"], host["gamma"], host["beta"]]
+        if fwd is None:
+            fwd = HostForward("linear_ln", host["Q"], [(cfg.H, cfg.d, cfg.d)], [p.shape for p in params],
+                              chunks=3)
+        Z = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d, pin_memory=True)
+        W = torch.empty(cfg.B, cfg.H, cfg.d, cfg.d, pin_memory=True)
+        fwd.run(host["Q"], host["K"], host["V"], host["eta"], params, cfg.b, cfg.ln_eps, Z, [W])
+        outs.append((Z, W))
+    fwd.done.synchronize()
+    for (Z, W), (_, ref) in zip(outs, runs):
+        assert np.array_equal(Z.numpy(), ref["Z"])
+        assert np.array_equal(W.numpy(), ref["W"])

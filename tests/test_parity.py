@@ -17,7 +17,7 @@ PATHS = {"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT, "tc": ttt.TTT_PAT
 
 
 def tc_capable(cfg):
-    return cfg.dtype == "bf16" and cfg.variant != "mlp" and cfg.b == 16
+    return cfg.dtype == "bf16" and cfg.b == 16
 
 
 @pytest.fixture(autouse=True)
@@ -47,6 +47,15 @@ def test_reduced_config_every_unit(name, path):
     assert max(worst.values()) <= tol, (name, path, worst)
 
 
+# Regression bounds of the default path at full size, a few times the error each
+# path measures (printed by the test): the exact-fp32 path for fp32 inputs, bf16
+# hi + lo operands for TTT-Linear, tf32 operands for TTT-MLP.  A precision change
+# shows here long before it reaches the oracle tolerance.
+REGRESSION = {"linear_f32_B1H1T256": 1e-6, "linear_bf16_B16H12T2048": 3e-5,
+              "linear_ln_B16H32T8192": 3e-5, "linear_ln_B1H32T32768": 3e-5,
+              "mlp_B8H32T8192": 1.5e-3}
+
+
 @pytest.mark.parametrize("name", I.CONFIG_ORDER)
 def test_full_size_sampled_units(name):
     cfg = I.CONFIGS[name]
@@ -54,7 +63,9 @@ def test_full_size_sampled_units(name):
     out = run_gpu(cfg, dev)
     n = 6 if cfg.variant != "mlp" else 3
     worst = compare(cfg, out, sample_units(cfg, n))
+    print(f"{name}: max relative Frobenius error per output {worst}")
     assert max(worst.values()) <= TOL[cfg.dtype], (name, worst)
+    assert max(worst.values()) <= REGRESSION[name], (name, worst)
     # Properties that hold at any size: finite everywhere, no unit left unwritten.
     for k, v in out.items():
         assert np.all(np.isfinite(v)), k
@@ -121,11 +132,15 @@ def test_device_status_clean_after_runs():
     assert ttt.last_device_status() == 0
 
 
-@pytest.mark.parametrize("variant", ["linear", "linear_ln"])
+BASES = {"linear": "linear_bf16_B16H12T2048", "linear_ln": "linear_ln_B16H32T8192",
+         "mlp": "mlp_B8H32T8192"}
+
+
+@pytest.mark.parametrize("variant", ["linear", "linear_ln", "mlp"])
 @pytest.mark.parametrize("T", [16, 48, 80, 208, 1040])
 def test_tensor_core_ragged_chunks(variant, T):
     """Sequences whose length is not a multiple of the 64-token chunk."""
-    base = {"linear": "linear_bf16_B16H12T2048", "linear_ln": "linear_ln_B16H32T8192"}[variant]
+    base = BASES[variant]
     cfg = I.CONFIGS[base].replace(B=2, H=3, T=T)
     ttt.set_path(ttt.TTT_PATH_TC)
     dev = to_device(cfg, I.make_inputs(cfg))
@@ -133,10 +148,16 @@ def test_tensor_core_ragged_chunks(variant, T):
     assert max(worst.values()) <= TOL[cfg.dtype], (variant, T, worst)
 
 
-@pytest.mark.parametrize("name", ["linear_bf16_B16H12T2048", "linear_ln_B16H32T8192"])
+# Agreement of the tensor-core path with the exact-fp32 CUDA-core path: bf16
+# hi + lo operands (~2^-16) for TTT-Linear, tf32 operands (10-bit mantissa) for
+# TTT-MLP, both far below the oracle tolerance.
+AGREE = {"linear_bf16_B16H12T2048": 2e-4, "linear_ln_B16H32T8192": 2e-4, "mlp_B8H32T8192": 1e-3}
+
+
+@pytest.mark.parametrize("name", list(AGREE))
 def test_tensor_core_matches_cuda_core_path(name):
     """The two CUDA paths agree far below the oracle tolerance."""
-    cfg = I.CONFIGS[name].replace(B=2, H=4, T=1024)
+    cfg = I.CONFIGS[name].replace(B=2, H=4, T=1024 if not name.startswith("mlp") else 512)
     dev = to_device(cfg, I.make_inputs(cfg))
     ttt.set_path(ttt.TTT_PATH_TC)
     a = run_gpu(cfg, dev)
@@ -144,15 +165,15 @@ def test_tensor_core_matches_cuda_core_path(name):
     b = run_gpu(cfg, dev)
     for k in a:
         rel = np.linalg.norm(a[k] - b[k]) / np.linalg.norm(b[k])
-        assert rel < 2e-4, (k, rel)
+        assert rel < AGREE[name], (k, rel)
 
 
-@pytest.mark.parametrize("variant", ["linear", "linear_ln"])
+@pytest.mark.parametrize("variant", ["linear", "linear_ln", "mlp"])
 def test_bounded_wait_expiry_is_reported_and_recoverable(variant):
     """The timeout path without a fault: every CTA waits on a barrier that nothing
     arrives at, the bounded wait expires, the status word reports it, and the
     context stays usable (the next call is exact again)."""
-    base = {"linear": "linear_bf16_B16H12T2048", "linear_ln": "linear_ln_B16H32T8192"}[variant]
+    base = BASES[variant]
     cfg = I.CONFIGS[base].replace(B=2, H=3, T=320)
     dev = to_device(cfg, I.make_inputs(cfg))
     ttt.set_path(ttt.TTT_PATH_TC)
