@@ -1,4 +1,4 @@
-// tc_mlp.cuh - tensor-core (tcgen05, kind::tf32) kernel of TTT-MLP,
+// tc_mlp.cuh - tensor-core (tcgen05) kernel of TTT-MLP,
 // f(x) = x + LN(GELU(x W1) W2), d = 64, hidden h = 256, bf16 Q, K, V, b = 16.
 //
 // Method: the dual form of the TTT write-up (§03.7) over mini-batches of b = 16
@@ -13,44 +13,49 @@
 // Every product is exact in the dual form: each layer is linear in its weight
 // and all the mini-batch's gradients are taken at its base state.
 //
-// Work decomposition.  One CTA of 8 warps owns one (batch, head) sequence for
-// its whole length; thread i owns hidden unit i (TMEM lane i % 128 of column
-// half i / 128).  The fp32 state lives in tensor memory for the whole sequence:
-// W1^T and W2 as [hidden][d] (lanes = hidden unit), and the two state updates
-// are tensor-core products that accumulate into it in place.  Products whose
-// output has a hidden dimension are computed hidden-major (M = 256 as two
-// M = 128 halves), the two whose output is [d x tokens] with M = 64.  Operands
-// that contract over d with the hidden units as rows (W1^T, W2, X2^T, E2^T) are
-// read from tensor memory; the products that contract W2 over the hidden width
-// read a tf32 copy of W2 in shared memory, refreshed after each update.
-// kind::tf32 takes a shared-memory operand either K-major (128-byte swizzle) or
-// MN-major (128-byte swizzle on a 32-byte base), so each buffer is stored in
-// the one form its products need.  Per mini-batch:
-//   P1  = W1^T [K;Q]^T               (hidden x 32 tokens; A from TMEM)
-//   X3^T = W2^T X2^T                  (d x 16, M = 64)
-//   GW^T = W2 G3^T                    (hidden x 16; A from TMEM)
-//   W2 -= X2^T E3,  W1^T -= E2^T K    (A from TMEM, accumulated into the state)
-//   P1_q -= E2^T tril(Q K^T)^T        (Zq1: the Q columns of P1)
-//   S2   = Zq2 X2^T                   (the 16 x 16 Gram over the hidden width:
-//                                     8 blocks of 32 hidden units, each an
-//                                     M = 64 product whose diagonal 16 x 16
-//                                     blocks are summed)
-//   Zq3^T = W2'^T Zq2^T + E3^T striu(S2)^T  (W2' = W2 after this mini-batch's
-//                                     update, hence the strictly upper mask:
-//                                     Zq2 W2 = Zq2 W2' + S2 E3)
+// Work decomposition.  One CTA of 16 warps owns one (batch, head) sequence for
+// its whole length; thread (i, j) owns hidden unit i (TMEM lane i % 128 of
+// column half i / 128) and tokens 8 j .. 8 j + 7 of each mini-batch (or d
+// columns 32 j .. 32 j + 31 of the state).  The fp32 state lives in tensor
+// memory for the whole sequence: W1^T and W2 as [hidden][d] (lanes = hidden
+// unit), and the two state updates are tensor-core products that accumulate
+// into it in place.  Products whose output has a hidden dimension are computed
+// hidden-major (M = 256 as two M = 128 halves), the two whose output is
+// [d x tokens] with M = 64.  Per mini-batch:
+//   P1   = W1^T [K;Q]^T                 (hidden x 32 tokens; A from TMEM)
+//   X3^T = W2^T X2^T                    (d x 16, M = 64)
+//   GW^T = W2 G3^T                      (hidden x 16; A from TMEM)
+//   W2 -= X2^T E3,  W1^T -= E2^T K      (A from TMEM, accumulated into the state)
+//   P1_q -= E2^T tril(Q K^T)^T          (Zq1: the Q columns of P1)
+//   S2   = Zq2 X2^T                     (the 16 x 16 Gram over the hidden width:
+//                                       4 blocks of 64 hidden units as one
+//                                       M = 64 product whose diagonal 16 x 16
+//                                       blocks are summed)
+//   Zq3^T = W2'^T Zq2^T + E3^T striu(S2)^T   (W2' = W2 after this mini-batch's
+//                                       update, hence the strictly upper mask:
+//                                       Zq2 W2 = Zq2 W2' + S2 E3)
 // and once per chunk of 64 tokens S1 = [K;Q] K^T for the masked Q K^T blocks.
 // GELU, GELU', the LN forward and backward and the output LN run on the CUDA
 // cores between the products.
 //
-// Precision: tf32 operands (10-bit mantissa), fp32 accumulation and fp32
-// state.  Activations, gradients, the masked Grams and the W2 copy are rounded
-// to tf32 (nearest) when they are written; W1 is read from tensor memory at
-// full precision, which the tensor core truncates to tf32.  K and Q (bf16) are
-// exact in tf32.
+// Operand precision.  The products that contract over the hidden width (X3,
+// Zq3, the Gram) take fp16 operands (kind::f16, 10-bit mantissa, 16 elements
+// of K per instruction): a copy of W2 refreshed after each update, X2 and Zq2.
+// Every other product is kind::tf32 (10-bit mantissa, fp32 range) with the
+// fp32 state read from tensor memory (truncated to tf32 by the tensor core) and
+// the activations, gradients and masked Grams rounded to tf32 where they are
+// written.  Accumulation is fp32; K and Q (bf16) are exact in tf32.  fp16
+// overflows above 65504: the W2 copy and the activations X2, Zq2 stay far below
+// that unless the inner model diverges.
+//
+// Product issue.  A tcgen05.mma instruction costs ~45 SM cycles to issue
+// whatever its size, so the products are shaped for few instructions, and every
+// product is issued by warp 0 converged (one lane elected inside the asm).
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "device_status.cuh"
@@ -65,7 +70,7 @@ constexpr int D = 64;
 constexpr int HID = 256;
 constexpr int MB = 16;      // mini-batch size of this kernel
 constexpr int CHUNK = 64;   // tokens per TMA chunk (4 mini-batches)
-constexpr int THREADS = 256;
+constexpr int THREADS = 512;
 constexpr uint32_t TMEM_COLS = 512;
 
 // TMEM columns (lane = hidden unit within a half unless noted).
@@ -76,29 +81,30 @@ constexpr uint32_t C_P1 = 256;   // P1 = W1^T [K;Q]^T, half h at 256 + 32 h; its
 constexpr uint32_t C_GW = 320;   // GW^T, half h at 320 + 16 h; then E2^T
 constexpr uint32_t C_X3 = 352;   // X3^T (M = 64, lane offset 0) and Zq3^T (lane offset 16)
 constexpr uint32_t C_S1 = 368;   // S1 = [K;Q] K^T of the chunk (M = 128, 64 columns)
-constexpr uint32_t C_S2 = 432;   // the Gram blocks (M = 64 at lane offsets 0 and 16, 64 columns)
+constexpr uint32_t C_S2 = 432;   // the Gram blocks (M = 64, 64 columns)
 
 // Shared-memory map (bytes from a 1024-byte aligned base).  "[a][r][128B]" means
-// 32 fp32 of row r of column block a; K-major tiles use the 128-byte swizzle
-// (swz32), MN-major ones the 32-byte-base swizzle (swzb32).
-constexpr uint32_t OFF_W2 = 0;          // W2 copy [d-block 2][hidden 256][128B], tf32, MN-major
-constexpr uint32_t OFF_KQ = 65536;      // [K;Q] of the chunk [d-block 2][row 128][128B], K-major
-constexpr uint32_t OFF_X2 = 98304;      // X2  [hidden-block 8][token 16][128B], K-major
-constexpr uint32_t OFF_KM = 114688;     // K of the mini-batch [d-block 2][token 16][128B], MN-major
-constexpr uint32_t OFF_Z2 = 131072;     // Zq2 [hidden-block 8][token 16][128B], K-major
-constexpr uint32_t OFF_G3 = 147456;     // G3  [d-block 2][token 16][128B], K-major
-constexpr uint32_t OFF_E3 = 151552;     // E3  same shape, MN-major
-constexpr uint32_t OFF_S1 = 155648;     // masked Q K^T in P1's column order [row 32][128B]
-constexpr uint32_t OFF_S2U = 159744;    // striu(S2) [query token 16][128B]
-constexpr uint32_t OFF_STG = 161792;    // 2 stages x {K, Q, V} bf16 [64][128B] (TMA)
+// 128 bytes of row r of column block a.  K-major tiles and fp16 tiles use the
+// 128-byte swizzle (16-byte granules), MN-major fp32 tiles the 128-byte swizzle
+// on a 32-byte base (the only MN-major layout of kind::tf32).
+constexpr uint32_t OFF_W2 = 0;          // W2 copy [hidden 256][64 d fp16], MN-major for W2^T
+constexpr uint32_t OFF_KQ = 32768;      // [K;Q] of the chunk [d-block 2][row 128][128B] fp32, K-major
+constexpr uint32_t OFF_X2 = 65536;      // X2  [hidden-block 4][token 16][64 fp16], K-major
+constexpr uint32_t OFF_Z2 = 73728;      // Zq2 same layout
+constexpr uint32_t OFF_KM = 81920;      // K of the mini-batch [d-block 2][token 16][128B] fp32, MN-major
+constexpr uint32_t OFF_G3 = 86016;      // G3  [d-block 2][token 16][128B] fp32, K-major
+constexpr uint32_t OFF_E3 = 90112;      // E3  same shape, MN-major
+constexpr uint32_t OFF_S1 = 94208;      // masked Q K^T in P1's column order [row 32][128B]
+constexpr uint32_t OFF_S2U = 98304;     // striu(S2) [query token 16][128B]
+constexpr uint32_t OFF_STG = 100352;    // 2 stages x {K, Q, V} bf16 [64][128B] (TMA)
 constexpr uint32_t STG_BYTES = 24576;
-constexpr uint32_t OFF_ETA = 210944;    // 2 stages x 64 eta
-constexpr uint32_t OFF_RED = 211456;    // [16][RS] fp32 rows (X3, Zq3) / Gram partials [8][16][17]
-constexpr uint32_t OFF_GB = 220160;     // gamma [64], beta [64]
-constexpr uint32_t OFF_BAR = 220672;    // mbarriers
-constexpr uint32_t OFF_TSLOT = 220800;  // TMEM base address
-constexpr uint32_t OFF_ABORT = 220804;  // set when a bounded wait expired
-constexpr uint32_t SMEM_USED = 220808;
+constexpr uint32_t OFF_ETA = 149504;    // 2 stages x 64 eta
+constexpr uint32_t OFF_RED = 150016;    // [16][RS] fp32 rows (X3, Zq3) / Gram partials [4][16][17]
+constexpr uint32_t OFF_GB = 154368;     // gamma [64], beta [64]
+constexpr uint32_t OFF_BAR = 154880;    // mbarriers
+constexpr uint32_t OFF_TSLOT = 154976;  // TMEM base address
+constexpr uint32_t OFF_ABORT = 154980;  // set when a bounded wait expired
+constexpr uint32_t SMEM_USED = 154984;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 constexpr int RS = 68;                  // row stride (floats) of the [token][d] staging rows
 
@@ -120,34 +126,47 @@ struct Params {
   int inject_timeout;
 };
 
-// Byte offset of fp32 element (row, col) in a [rows][128B] block of 32 columns
-// with the 128-byte swizzle (col < 32).
+// Byte offset of 4-byte element (row, col) in a [rows][128B] block of 32
+// columns with the 128-byte swizzle (col < 32).
 __device__ __forceinline__ uint32_t swz32(uint32_t row, uint32_t col) {
   return row * 128u + ((((col >> 2) ^ row) & 7u) << 4) + ((col & 3u) << 2);
 }
-
-// Byte offset of fp32 element (row, col) in a [rows][128B] block of 32 columns
-// with the 32-byte-base swizzle (col < 32).
+// The same for 2-byte elements, 64 columns per row (col < 64).
+__device__ __forceinline__ uint32_t swz16(uint32_t row, uint32_t col) {
+  return row * 128u + ((((col >> 3) ^ row) & 7u) << 4) + ((col & 7u) << 1);
+}
+// 4-byte element (row, col) with the 32-byte-base swizzle (col < 32).
 __device__ __forceinline__ uint32_t swzb32(uint32_t row, uint32_t col) {
   return row * 128u + ((((col >> 3) ^ row) & 3u) << 5) + ((col & 7u) << 2);
 }
 
-__device__ __forceinline__ float sum16(float x) {
-  x += __shfl_xor_sync(0xffffffffu, x, 1);
-  x += __shfl_xor_sync(0xffffffffu, x, 2);
-  x += __shfl_xor_sync(0xffffffffu, x, 4);
-  x += __shfl_xor_sync(0xffffffffu, x, 8);
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
   return x;
 }
 
-// GELU(x) = x Phi(x) (exact erf form) and its derivative Phi(x) + x phi(x).
-__device__ __forceinline__ void gelu2(float x, float &g, float &dg) {
-  const float cdf = normcdff(x);
-  const float pdf = 0.398942280401432678f * expf(-0.5f * x * x);
-  g = x * cdf;
-  dg = fmaf(x, pdf, cdf);
+// Phi(x) and phi(x) of the standard normal, for GELU(x) = x Phi(x) (the exact
+// erf form) and GELU'(x) = Phi(x) + x phi(x).  erfc(z), z = |x| / sqrt(2), by
+// the rational approximation of Abramowitz and Stegun, Handbook of Mathematical
+// Functions, formula 7.1.26 (absolute error at most 1.5e-7):
+//   erfc(z) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),
+//   t = 1 / (1 + p z),
+// so that Phi(x) = 1 - erfc(z) / 2 for x >= 0 and erfc(z) / 2 otherwise, with no
+// cancellation on either side; exp(-z^2) = exp(-x^2 / 2) also gives phi.
+__device__ __forceinline__ void normal_cdf_pdf(float x, float &cdf, float &pdf) {
+  constexpr float P = 0.3275911f;
+  constexpr float A1 = 0.254829592f, A2 = -0.284496736f, A3 = 1.421413741f;
+  constexpr float A4 = -1.453152027f, A5 = 1.061405429f;
+  constexpr float RSQRT2 = 0.70710678118654752f, RSQRT2PI = 0.39894228040143268f;
+  const float z = fabsf(x) * RSQRT2;
+  const float t = __fdividef(1.f, fmaf(P, z, 1.f));
+  const float poly = t * fmaf(t, fmaf(t, fmaf(t, fmaf(t, A5, A4), A3), A2), A1);
+  const float e = __expf(-0.5f * x * x);
+  const float half_erfc = 0.5f * poly * e;
+  cdf = x >= 0.f ? 1.f - half_erfc : half_erfc;
+  pdf = RSQRT2PI * e;
 }
-__device__ __forceinline__ float gelu(float x) { return x * normcdff(x); }
 
 __device__ __forceinline__ void mma_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                          long long limit = WAIT_LIMIT) {
@@ -166,8 +185,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3;    // TMEM lane quarter of this warp
-  const int half = warp >> 2; // hidden half of this thread
+  const int qd = warp & 3;           // TMEM lane quarter of this warp
+  const int half = (warp >> 2) & 1;  // hidden half of this thread
+  const int th = warp >> 3;          // token half (tokens 8 th .. 8 th + 7) / d block
   const int hid = 128 * half + 32 * qd + lane;
   const int unit = blockIdx.x;
   const int head = unit % p.H;
@@ -205,37 +225,42 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t tb = *tslot;
   const uint32_t tq = tmem_addr(tb, 32 * qd, 0);  // this warp's lane quarter
 
-  // Initial state: W1^T row `hid` and W2 row `hid` into TMEM; W2 (tf32) into the
-  // shared copy.
-  {
-    const float *w1 = p.W1_0 + (size_t)head * D * HID;
-    const float *w2 = p.W2_0 + ((size_t)head * HID + hid) * D;
+  // Writes 32 consecutive d of this thread's W2 row as fp16 into the W2 copy
+  // (MN-major for W2^T: row = hidden unit, 64 d per 128-byte row).
+  auto store_w2_row = [&](const uint32_t (&r)[32]) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t r[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(w1[(16 * k + e) * HID + hid]);
-      tmem_st_32x32b_x16(tq + C_W1 + 64 * half + 16 * k, r);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint32_t r[16];
-      float4 v[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = reinterpret_cast<const float4 *>(w2 + 16 * k)[e];
+    for (int u = 0; u < 4; ++u) {
+      uint32_t h2[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        r[4 * e + 0] = __float_as_uint(v[e].x);
-        r[4 * e + 1] = __float_as_uint(v[e].y);
-        r[4 * e + 2] = __float_as_uint(v[e].z);
-        r[4 * e + 3] = __float_as_uint(v[e].w);
-        const int col = 16 * k + 4 * e;  // d of v[e].x
-        *reinterpret_cast<float4 *>(sm + OFF_W2 + (col >> 5) * 32768u + swzb32(hid, col & 31)) =
-            make_float4(round_tf32(v[e].x), round_tf32(v[e].y), round_tf32(v[e].z),
-                        round_tf32(v[e].w));
+        __half2 v = __floats2half2_rn(__uint_as_float(r[8 * u + 2 * e]), __uint_as_float(r[8 * u + 2 * e + 1]));
+        h2[e] = *reinterpret_cast<uint32_t *>(&v);
       }
-      tmem_st_32x32b_x16(tq + C_W2 + 64 * half + 16 * k, r);
+      *reinterpret_cast<uint4 *>(sm + OFF_W2 + swz16(hid, 32 * th + 8 * u)) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
     }
+  };
+
+  // Initial state: this thread's 32 d of W1^T row `hid` and of W2 row `hid` into
+  // TMEM; the W2 row also into the fp16 copy.
+  {
+    const float *w1 = p.W1_0 + (size_t)head * D * HID;
+    const float *w2 = p.W2_0 + ((size_t)head * HID + hid) * D + 32 * th;
+    uint32_t r[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(w1[(32 * th + e) * HID + hid]);
+    tmem_st_32x32b_x16(tq + C_W1 + 64 * half + 32 * th, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
+    tmem_st_32x32b_x16(tq + C_W1 + 64 * half + 32 * th + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float4 v = reinterpret_cast<const float4 *>(w2)[e];
+      r[4 * e] = __float_as_uint(v.x);
+      r[4 * e + 1] = __float_as_uint(v.y);
+      r[4 * e + 2] = __float_as_uint(v.z);
+      r[4 * e + 3] = __float_as_uint(v.w);
+    }
+    tmem_st_32x32b_x16(tq + C_W2 + 64 * half + 32 * th, *reinterpret_cast<const uint32_t(*)[16]>(&r[0]));
+    tmem_st_32x32b_x16(tq + C_W2 + 64 * half + 32 * th + 16, *reinterpret_cast<const uint32_t(*)[16]>(&r[16]));
+    store_w2_row(r);
     tmem_wait_st();
   }
 
@@ -262,12 +287,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // Instruction descriptors.
   constexpr uint32_t ID_P1 = idesc_tf32_f32(128, 32, false, false, false);   // W1^T(TMEM) x [K;Q]
-  constexpr uint32_t ID_X3 = idesc_tf32_f32(64, 16, true, false, false);     // W2^T x X2 (and Zq2)
+  constexpr uint32_t ID_X3 = idesc_f16_f32(64, 16, true, false, false);      // W2^T x X2 (and Zq2)
   constexpr uint32_t ID_GW = idesc_tf32_f32(128, 16, false, false, false);   // W2(TMEM) x G3
   constexpr uint32_t ID_UPD = idesc_tf32_f32(128, 64, false, true, true);    // state -= A(TMEM) B
   constexpr uint32_t ID_ZQ1 = idesc_tf32_f32(128, 32, false, false, true);   // P1 -= E2^T(TMEM) S1^T
   constexpr uint32_t ID_S1 = idesc_tf32_f32(128, 64, false, false, false);   // [K;Q] x K
-  constexpr uint32_t ID_G2 = idesc_tf32_f32(64, 64, false, false, false);    // Gram blocks
+  constexpr uint32_t ID_G2 = idesc_f16_f32(64, 64, false, false, false);     // Gram blocks
   constexpr uint32_t ID_ZC = idesc_tf32_f32(64, 16, true, false, false);     // Zq3 += E3^T S2u^T
 
   const uint32_t aW2 = sbase + OFF_W2, aKQ = sbase + OFF_KQ, aX2 = sbase + OFF_X2;
@@ -278,24 +303,25 @@ __global__ void __launch_bounds__(THREADS, 1)
   uint32_t n_s1c = 0, n_p1 = 0, n_x3 = 0, n_gw = 0, n_upd = 0, n_s2 = 0, n_zq3 = 0;
   int issued_mma = 0;  // whether warp 0 has issued products (for the drain)
 
-  // Products are issued by one elected lane of warp 0 after a CTA barrier.
-  auto issue_p1 = [&](int m, bool elected) {
+  // Products are issued by warp 0 (one lane elected inside each instruction's asm
+  // block, the warp converged) after a CTA barrier.
+  auto issue_p1 = [&](int m) {
 #pragma unroll
     for (int h = 0; h < 2; ++h)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint64_t b = smem_desc_sw128(aKQ + m * 4096 + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
-        if (elected) umma_ts_tf32(tb + C_P1 + 32 * h, tb + C_W1 + 64 * h + 8 * i, b, ID_P1, i > 0);
+        umma_ts_tf32_w(tb + C_P1 + 32 * h, tb + C_W1 + 64 * h + 8 * i, b, ID_P1, i > 0);
       }
-    if (elected) umma_commit(&bars[BAR_P1]);
+    umma_commit_w(&bars[BAR_P1]);
   };
-  // W2^T (M = d) against a [16 token][hidden] operand (X2 or Zq2).
-  auto issue_w2t = [&](uint32_t d_tmem, uint32_t aB, bool elected) {
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) {
-      const uint64_t a = smem_desc_sw128_b32(aW2 + i * 1024, 32768, 512);
+  // W2^T (M = d, fp16) against a [16 token][hidden] fp16 operand (X2 or Zq2).
+  auto issue_w2t = [&](uint32_t d_tmem, uint32_t aB) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint64_t a = smem_desc_sw128(aW2 + i * 2048, 8192, 1024);
       const uint64_t b = smem_desc_sw128(aB + (i >> 2) * 2048 + (i & 3) * 32, 16, 1024);
-      if (elected) umma_ss_tf32(d_tmem, a, b, ID_X3, i > 0);
+      umma_ss_w(d_tmem, a, b, ID_X3, i > 0);
     }
   };
 
@@ -327,46 +353,43 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after_sync();
     if (warp == 0) {
       __syncwarp();
-      const bool el = elect_one_sync();
       tc_fence_after_sync();
+      issue_p1(0);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t off = (i >> 2) * 16384 + (i & 3) * 32;
-        if (el)
-          umma_ss_tf32(tb + C_S1, smem_desc_sw128(aKQ + off, 16, 1024),
+        umma_ss_tf32_w(tb + C_S1, smem_desc_sw128(aKQ + off, 16, 1024),
                        smem_desc_sw128(aKQ + off, 16, 2048), ID_S1, i > 0);
       }
-      if (el) umma_commit(&bars[BAR_S1C]);
-      issue_p1(0, el);
+      umma_commit_w(&bars[BAR_S1C]);
       issued_mma = 1;
       __syncwarp();
     }
 
     for (int m = 0; m < nmb; ++m) {
       const int t0 = MB * m;  // first token of the mini-batch within the chunk
-      // ---- X1 -> X2 = GELU(X1), GELU'(X1) (thread = hidden unit, 16 tokens) ----
+      // ---- X1 -> X2 = GELU(X1), GELU'(X1) (thread: hidden unit, 8 tokens) ----------
       mma_wait(&bars[BAR_P1], n_p1++ & 1u, abort);
       tc_fence_after_sync();
       __syncwarp();
-      float d2[16];
+      float d2[8];
       {
-        uint32_t ra[8], rb[8];
-        tmem_ld_32x32b_x8(tq + C_P1 + 32 * half, ra);       // K tokens 0-7
-        tmem_ld_32x32b_x8(tq + C_P1 + 32 * half + 16, rb);  // K tokens 8-15
+        uint32_t r[8];
+        tmem_ld_32x32b_x8(tq + C_P1 + 32 * half + 16 * th, r);  // K tokens 8 th .. 8 th + 7
         tmem_wait_ld();
-        const uint32_t xb = OFF_X2 + (4 * half + qd) * 2048u;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float x1 = __uint_as_float(j < 8 ? ra[j] : rb[j - 8]);
-          float g;
-          gelu2(x1, g, d2[j]);
-          g = round_tf32(g);
-          *reinterpret_cast<float *>(sm + xb + swz32(j, lane)) = g;
-          if (j < 8) ra[j] = __float_as_uint(g); else rb[j - 8] = __float_as_uint(g);
+        for (int j = 0; j < 8; ++j) {
+          const float x1 = __uint_as_float(r[j]);
+          float cdf, pdf;
+          normal_cdf_pdf(x1, cdf, pdf);
+          const float g = x1 * cdf;
+          d2[j] = fmaf(x1, pdf, cdf);
+          const int t = 8 * th + j;
+          *reinterpret_cast<__half *>(sm + OFF_X2 + (hid >> 6) * 2048u + swz16(t, hid & 63)) = __float2half_rn(g);
+          r[j] = __float_as_uint(round_tf32(g));
         }
         // X2^T over the consumed X1 columns: the A operand of the W2 update.
-        tmem_st_32x32b_x8(tq + C_P1 + 32 * half, ra);
-        tmem_st_32x32b_x8(tq + C_P1 + 32 * half + 16, rb);
+        tmem_st_32x32b_x8(tq + C_P1 + 32 * half + 16 * th, r);
         tmem_wait_st();
       }
       fence_proxy_async_smem();
@@ -376,11 +399,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---- X3^T = W2^T X2^T ----------------------------------------------------
       if (warp == 0) {
         __syncwarp();
-        const bool el = elect_one_sync();
         tc_fence_after_sync();
-        issue_w2t(tb + C_X3, aX2, el);
-        if (el) umma_commit(&bars[BAR_X3]);
+        issue_w2t(tb + C_X3, aX2);
+        umma_commit_w(&bars[BAR_X3]);
         __syncwarp();
+      }
+      // K of the mini-batch, MN-major, for the W1 update (one float4 per thread).
+      if (tid < 256) {
+        const int t = tid >> 4, u = tid & 15, tc = t0 + t;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(
+            stg + tc * 128 + ((((u >> 1) ^ tc) & 7) << 4) + (u & 1) * 8);
+        const float2 lo = unpack_bf16x2(raw.x), hi = unpack_bf16x2(raw.y);
+        *reinterpret_cast<float4 *>(sm + OFF_KM + (u >> 3) * 2048u + swzb32(t, 4 * (u & 7))) =
+            make_float4(lo.x, lo.y, hi.x, hi.y);
       }
       mma_wait(&bars[BAR_X3], n_x3++ & 1u, abort);
       tc_fence_after_sync();
@@ -396,37 +427,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before_sync();
       __syncthreads();
-      // ---- LN forward and backward of X3 (16 threads per token, 4 d each) -------
+      // ---- LN forward and backward of X3 (one warp per token, 2 d per lane) ------
       {
-        const int t = tid >> 4, sub = tid & 15, tc = t0 + t;
-        const float4 x = *reinterpret_cast<const float4 *>(red + t * RS + 4 * sub);
-        const float4 gm = *reinterpret_cast<const float4 *>(gam + 4 * sub);
-        const float4 bt = *reinterpret_cast<const float4 *>(bet + 4 * sub);
-        const uint32_t kvo = tc * 128 + ((((sub >> 1) ^ tc) & 7) << 4) + (sub & 1) * 8;
-        const uint2 kr = *reinterpret_cast<const uint2 *>(stg + kvo);
-        const uint2 vr = *reinterpret_cast<const uint2 *>(stg + 16384 + kvo);
-        const float2 k01 = unpack_bf16x2(kr.x), k23 = unpack_bf16x2(kr.y);
-        const float2 v01 = unpack_bf16x2(vr.x), v23 = unpack_bf16x2(vr.y);
-        const float mean = sum16((x.x + x.y) + (x.z + x.w)) * (1.f / D);
-        const float d0 = x.x - mean, d1 = x.y - mean, dd2 = x.z - mean, d3 = x.w - mean;
-        const float var = sum16((d0 * d0 + d1 * d1) + (dd2 * dd2 + d3 * d3)) * (1.f / D);
-        const float r = rsqrtf(var + p.eps);
-        const float h0 = d0 * r, h1 = d1 * r, h2 = dd2 * r, h3 = d3 * r;
+        const int t = warp, tc = t0 + t, dc = 2 * lane;
+        const float2 x = *reinterpret_cast<const float2 *>(red + t * RS + dc);
+        const float2 gm = *reinterpret_cast<const float2 *>(gam + dc);
+        const float2 bt = *reinterpret_cast<const float2 *>(bet + dc);
+        const uint32_t kvo = tc * 128 + ((((dc >> 3) ^ tc) & 7) << 4) + (dc & 7) * 2;
+        const float2 kk = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(stg + kvo));
+        const float2 vv = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(stg + 16384 + kvo));
+        const float mean = warp_sum(x.x + x.y) * (1.f / D);
+        const float d0 = x.x - mean, d1 = x.y - mean;
+        const float r = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / D) + p.eps);
+        const float h0 = d0 * r, h1 = d1 * r;
         // g = 2 (k + gamma xhat + beta - v); dl/dxhat = g gamma.
-        const float a0 = 2.f * (k01.x + fmaf(gm.x, h0, bt.x) - v01.x) * gm.x;
-        const float a1 = 2.f * (k01.y + fmaf(gm.y, h1, bt.y) - v01.y) * gm.y;
-        const float a2 = 2.f * (k23.x + fmaf(gm.z, h2, bt.z) - v23.x) * gm.z;
-        const float a3 = 2.f * (k23.y + fmaf(gm.w, h3, bt.w) - v23.y) * gm.w;
-        const float ma = sum16((a0 + a1) + (a2 + a3)) * (1.f / D);
-        const float mb = sum16((a0 * h0 + a1 * h1) + (a2 * h2 + a3 * h3)) * (1.f / D);
+        const float a0 = 2.f * (kk.x + fmaf(gm.x, h0, bt.x) - vv.x) * gm.x;
+        const float a1 = 2.f * (kk.y + fmaf(gm.y, h1, bt.y) - vv.y) * gm.y;
+        const float ma = warp_sum(a0 + a1) * (1.f / D);
+        const float mb = warp_sum(a0 * h0 + a1 * h1) * (1.f / D);
         const float g0 = r * (a0 - ma - h0 * mb), g1 = r * (a1 - ma - h1 * mb);
-        const float g2 = r * (a2 - ma - h2 * mb), g3 = r * (a3 - ma - h3 * mb);
         const float e = eta_s[tc];
-        const uint32_t blk = (sub >> 3) * 2048u;
-        *reinterpret_cast<float4 *>(sm + OFF_G3 + blk + swz32(t, 4 * (sub & 7))) =
-            make_float4(round_tf32(g0), round_tf32(g1), round_tf32(g2), round_tf32(g3));
-        *reinterpret_cast<float4 *>(sm + OFF_E3 + blk + swzb32(t, 4 * (sub & 7))) = make_float4(
-            round_tf32(e * g0), round_tf32(e * g1), round_tf32(e * g2), round_tf32(e * g3));
+        const uint32_t blk = (dc >> 5) * 2048u;
+        *reinterpret_cast<float2 *>(sm + OFF_G3 + blk + swz32(t, dc & 31)) =
+            make_float2(round_tf32(g0), round_tf32(g1));
+        *reinterpret_cast<float2 *>(sm + OFF_E3 + blk + swzb32(t, dc & 31)) =
+            make_float2(round_tf32(e * g0), round_tf32(e * g1));
       }
       fence_proxy_async_smem();
       tc_fence_before_sync();
@@ -435,28 +460,18 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---- GW^T = W2 G3^T (A = the W2 state in TMEM) --------------------------------
       if (warp == 0) {
         __syncwarp();
-        const bool el = elect_one_sync();
         tc_fence_after_sync();
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const uint64_t b = smem_desc_sw128(aG3 + (i >> 2) * 2048 + (i & 3) * 32, 16, 1024);
-            if (el) umma_ts_tf32(tb + C_GW + 16 * h, tb + C_W2 + 64 * h + 8 * i, b, ID_GW, i > 0);
+            umma_ts_tf32_w(tb + C_GW + 16 * h, tb + C_W2 + 64 * h + 8 * i, b, ID_GW, i > 0);
           }
-        if (el) umma_commit(&bars[BAR_GW]);
+        umma_commit_w(&bars[BAR_GW]);
         __syncwarp();
       }
-      // K of the mini-batch, MN-major, for the W1 update (one float4 per thread).
-      {
-        const int t = tid >> 4, u = tid & 15, tc = t0 + t;
-        const uint2 raw = *reinterpret_cast<const uint2 *>(
-            stg + tc * 128 + ((((u >> 1) ^ tc) & 7) << 4) + (u & 1) * 8);
-        const float2 lo = unpack_bf16x2(raw.x), hi = unpack_bf16x2(raw.y);
-        *reinterpret_cast<float4 *>(sm + OFF_KM + (u >> 3) * 2048u + swzb32(t, 4 * (u & 7))) =
-            make_float4(lo.x, lo.y, hi.x, hi.y);
-      }
-      // ---- the masked Q K^T block of this mini-batch (warp m % 4: its Q lanes) ---
+      // ---- the masked Q K^T block of this mini-batch (warp m: its Q lanes) ---------
       if (m == 0) mma_wait(&bars[BAR_S1C], n_s1c++ & 1u, abort);
       tc_fence_after_sync();
       __syncwarp();
@@ -477,20 +492,18 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
       }
-      // ---- G2 = GW * GELU'(X1), E2 = eta G2 ---------------------------------------
+      // ---- G2 = GW * GELU'(X1), E2 = eta G2 (into TMEM over GW) ----------------------
       mma_wait(&bars[BAR_GW], n_gw++ & 1u, abort);
       tc_fence_after_sync();
       __syncwarp();
       {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(tq + C_GW + 16 * half, r);
+        uint32_t r[8];
+        tmem_ld_32x32b_x8(tq + C_GW + 16 * half + 8 * th, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float g2 = __uint_as_float(r[j]) * d2[j];
-          r[j] = __float_as_uint(round_tf32(eta_s[t0 + j] * g2));
-        }
-        tmem_st_32x32b_x16(tq + C_GW + 16 * half, r);  // E2^T over the consumed GW
+        for (int j = 0; j < 8; ++j)
+          r[j] = __float_as_uint(round_tf32(eta_s[t0 + 8 * th + j] * (__uint_as_float(r[j]) * d2[j])));
+        tmem_st_32x32b_x8(tq + C_GW + 16 * half + 8 * th, r);
         tmem_wait_st();
       }
       fence_proxy_async_smem();
@@ -500,7 +513,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---- W1^T -= E2^T K; W2 -= X2^T E3; Zq1 = P1_q - E2^T S1^T ----------------------
       if (warp == 0) {
         __syncwarp();
-        const bool el = elect_one_sync();
         tc_fence_after_sync();
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -509,61 +521,54 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint64_t bk = smem_desc_sw128_b32(aKM + j * 1024, 2048, 512);
             const uint64_t be = smem_desc_sw128_b32(aE3 + j * 1024, 2048, 512);
             const uint64_t bs = smem_desc_sw128(aS1 + j * 32, 16, 1024);
-            const uint32_t e2 = tb + C_GW + 16 * h + 8 * j;        // E2^T, tokens 8j..8j+7
-            const uint32_t x2 = tb + C_P1 + 32 * h + 16 * j;       // X2^T, tokens 8j..8j+7
-            if (el) umma_ts_tf32(tb + C_W1 + 64 * h, e2, bk, ID_UPD, true);
-            if (el) umma_ts_tf32(tb + C_W2 + 64 * h, x2, be, ID_UPD, true);
-            if (el) umma_ts_tf32(tb + C_P1 + 32 * h, e2, bs, ID_ZQ1, true);
+            const uint32_t e2 = tb + C_GW + 16 * h + 8 * j;   // E2^T, tokens 8j..8j+7
+            const uint32_t x2 = tb + C_P1 + 32 * h + 16 * j;  // X2^T, tokens 8j..8j+7
+            umma_ts_tf32_w(tb + C_W1 + 64 * h, e2, bk, ID_UPD, true);
+            umma_ts_tf32_w(tb + C_W2 + 64 * h, x2, be, ID_UPD, true);
+            umma_ts_tf32_w(tb + C_P1 + 32 * h, e2, bs, ID_ZQ1, true);
           }
-        if (el) umma_commit(&bars[BAR_UPD]);
+        umma_commit_w(&bars[BAR_UPD]);
         __syncwarp();
       }
       // ---- refresh the W2 copy from the updated state; Zq2 = GELU(Zq1) -------------
       mma_wait(&bars[BAR_UPD], n_upd++ & 1u, abort);
       tc_fence_after_sync();
       __syncwarp();
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
+      {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tq + C_W2 + 64 * half + 32 * k, r);
+        tmem_ld_32x32b_x32(tq + C_W2 + 64 * half + 32 * th, r);
         tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          *reinterpret_cast<float4 *>(sm + OFF_W2 + k * 32768u + swzb32(hid, 4 * e)) =
-              make_float4(round_tf32(__uint_as_float(r[4 * e])), round_tf32(__uint_as_float(r[4 * e + 1])),
-                          round_tf32(__uint_as_float(r[4 * e + 2])), round_tf32(__uint_as_float(r[4 * e + 3])));
+        store_w2_row(r);
       }
       {
-        uint32_t ra[8], rb[8];
-        tmem_ld_32x32b_x8(tq + C_P1 + 32 * half + 8, ra);   // Q tokens 0-7
-        tmem_ld_32x32b_x8(tq + C_P1 + 32 * half + 24, rb);  // Q tokens 8-15
+        uint32_t r[8];
+        tmem_ld_32x32b_x8(tq + C_P1 + 32 * half + 8 + 16 * th, r);  // Q tokens 8 th .. 8 th + 7
         tmem_wait_ld();
-        const uint32_t zb = OFF_Z2 + (4 * half + qd) * 2048u;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          *reinterpret_cast<float *>(sm + zb + swz32(j, lane)) =
-              round_tf32(gelu(__uint_as_float(j < 8 ? ra[j] : rb[j - 8])));
+        for (int j = 0; j < 8; ++j) {
+          const float z1 = __uint_as_float(r[j]);
+          float cdf, pdf;
+          normal_cdf_pdf(z1, cdf, pdf);
+          *reinterpret_cast<__half *>(sm + OFF_Z2 + (hid >> 6) * 2048u + swz16(8 * th + j, hid & 63)) =
+              __float2half_rn(z1 * cdf);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before_sync();
       __syncthreads();
       tc_fence_after_sync();
-      // ---- Gram blocks of Zq2 X2^T; Zq3^T = W2'^T Zq2^T; next P1 ----------------------
+      // ---- next P1 first (it starts the next mini-batch's chain), then the Gram of
+      // Zq2 X2^T and Zq3^T = W2'^T Zq2^T ------------------------------------------------
       if (warp == 0) {
         __syncwarp();
-        const bool el = elect_one_sync();
         tc_fence_after_sync();
+        if (m + 1 < nmb) issue_p1(m + 1);
 #pragma unroll
-        for (int g = 0; g < 2; ++g)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint64_t a = smem_desc_sw128(aZ2 + g * 8192 + i * 32, 16, 1024);
-            const uint64_t b = smem_desc_sw128(aX2 + g * 8192 + i * 32, 16, 1024);
-            if (el) umma_ss_tf32(tmem_addr(tb, 16 * g, C_S2), a, b, ID_G2, i > 0);
-          }
-        if (el) umma_commit(&bars[BAR_S2]);
-        issue_w2t(tmem_addr(tb, 16, C_X3), aZ2, el);
-        if (m + 1 < nmb) issue_p1(m + 1, el);
+        for (int i = 0; i < 4; ++i)
+          umma_ss_w(tb + C_S2, smem_desc_sw128(aZ2 + i * 32, 16, 1024),
+                    smem_desc_sw128(aX2 + i * 32, 16, 1024), ID_G2, i > 0);
+        umma_commit_w(&bars[BAR_S2]);
+        issue_w2t(tmem_addr(tb, 16, C_X3), aZ2);
         __syncwarp();
       }
       mma_wait(&bars[BAR_S2], n_s2++ & 1u, abort);
@@ -571,19 +576,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (warp < 4) {
         uint32_t r[16];
-        tmem_ld_32x32b_x16(tq + C_S2 + 16 * qd, r);  // lanes 0-15: block qd, 16-31: block 4 + qd
+        tmem_ld_32x32b_x16(tq + C_S2 + 16 * qd, r);  // lanes 0-15: block qd, token lane
         tmem_wait_ld();
-        const int blk = qd + 4 * (lane >> 4), t = lane & 15;
+        if (lane < 16) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) red[(blk * 16 + t) * 17 + j] = __uint_as_float(r[j]);
+          for (int j = 0; j < 16; ++j) red[(qd * 16 + lane) * 17 + j] = __uint_as_float(r[j]);
+        }
       }
       tc_fence_before_sync();
       __syncthreads();
-      {
+      if (tid < 256) {
         const int t = tid >> 4, sj = tid & 15;
         float v = 0.f;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) v += red[(g * 16 + t) * 17 + sj];
+        for (int g = 0; g < 4; ++g) v += red[(g * 16 + t) * 17 + sj];
         *reinterpret_cast<float *>(sm + OFF_S2U + swz32(t, sj)) = sj > t ? round_tf32(v) : 0.f;
       }
       fence_proxy_async_smem();
@@ -593,15 +599,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ---- Zq3^T += E3^T striu(S2)^T ------------------------------------------------
       if (warp == 0) {
         __syncwarp();
-        const bool el = elect_one_sync();
         tc_fence_after_sync();
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           const uint64_t a = smem_desc_sw128_b32(aE3 + j * 1024, 2048, 512);
           const uint64_t b = smem_desc_sw128(aS2U + j * 32, 16, 1024);
-          if (el) umma_ss_tf32(tmem_addr(tb, 16, C_X3), a, b, ID_ZC, true);
+          umma_ss_tf32_w(tmem_addr(tb, 16, C_X3), a, b, ID_ZC, true);
         }
-        if (el) umma_commit(&bars[BAR_ZQ3]);
+        umma_commit_w(&bars[BAR_ZQ3]);
         __syncwarp();
       }
       mma_wait(&bars[BAR_ZQ3], n_zq3++ & 1u, abort);
@@ -618,25 +623,19 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       tc_fence_before_sync();
       __syncthreads();
-      // ---- Z = Q + LN(Zq3) ---------------------------------------------------------
+      // ---- Z = Q + LN(Zq3) (one warp per token) --------------------------------------
       {
-        const int t = tid >> 4, sub = tid & 15, tc = t0 + t;
-        const float4 x = *reinterpret_cast<const float4 *>(red + t * RS + 4 * sub);
-        const float4 gm = *reinterpret_cast<const float4 *>(gam + 4 * sub);
-        const float4 bt = *reinterpret_cast<const float4 *>(bet + 4 * sub);
-        const uint2 qr = *reinterpret_cast<const uint2 *>(
-            stg + 8192 + tc * 128 + ((((sub >> 1) ^ tc) & 7) << 4) + (sub & 1) * 8);
-        const float2 q01 = unpack_bf16x2(qr.x), q23 = unpack_bf16x2(qr.y);
-        const float mean = sum16((x.x + x.y) + (x.z + x.w)) * (1.f / D);
-        const float d0 = x.x - mean, d1 = x.y - mean, dd2 = x.z - mean, d3 = x.w - mean;
-        const float var = sum16((d0 * d0 + d1 * d1) + (dd2 * dd2 + d3 * d3)) * (1.f / D);
-        const float r = rsqrtf(var + p.eps);
-        float4 z;
-        z.x = q01.x + fmaf(gm.x, d0 * r, bt.x);
-        z.y = q01.y + fmaf(gm.y, d1 * r, bt.y);
-        z.z = q23.x + fmaf(gm.z, dd2 * r, bt.z);
-        z.w = q23.y + fmaf(gm.w, d3 * r, bt.w);
-        *reinterpret_cast<float4 *>(p.Z + (tok_base + (size_t)c * CHUNK + tc) * D + 4 * sub) = z;
+        const int t = warp, tc = t0 + t, dc = 2 * lane;
+        const float2 x = *reinterpret_cast<const float2 *>(red + t * RS + dc);
+        const float2 gm = *reinterpret_cast<const float2 *>(gam + dc);
+        const float2 bt = *reinterpret_cast<const float2 *>(bet + dc);
+        const float2 qq = unpack_bf16x2(*reinterpret_cast<const uint32_t *>(
+            stg + 8192 + tc * 128 + ((((dc >> 3) ^ tc) & 7) << 4) + (dc & 7) * 2));
+        const float mean = warp_sum(x.x + x.y) * (1.f / D);
+        const float d0 = x.x - mean, d1 = x.y - mean;
+        const float r = rsqrtf(warp_sum(d0 * d0 + d1 * d1) * (1.f / D) + p.eps);
+        *reinterpret_cast<float2 *>(p.Z + (tok_base + (size_t)c * CHUNK + tc) * D + dc) =
+            make_float2(qq.x + fmaf(gm.x, d0 * r, bt.x), qq.y + fmaf(gm.y, d1 * r, bt.y));
       }
       __syncthreads();  // the staging rows are rewritten by the next mini-batch
     }
@@ -653,7 +652,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (warp == 0 && issued_mma) {
       __syncwarp();
-      if (elect_one_sync()) umma_commit(&bars[BAR_DRAIN]);
+      umma_commit_w(&bars[BAR_DRAIN]);
       __syncwarp();
     }
     if (issued_mma) mbar_wait(&bars[BAR_DRAIN], 0, WAIT_LIMIT);
@@ -665,26 +664,19 @@ __global__ void __launch_bounds__(THREADS, 1)
   // Final state (every update has completed: each was waited on above).
   {
     float *w1 = p.W1_out + (size_t)unit * D * HID;
-    float *w2 = p.W2_out + ((size_t)unit * HID + hid) * D;
+    float *w2 = p.W2_out + ((size_t)unit * HID + hid) * D + 32 * th;
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(tq + C_W1 + 64 * half + 32 * th, r);
+    tmem_wait_ld();
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tq + C_W1 + 64 * half + 32 * k, r);
-      tmem_wait_ld();
+    for (int e = 0; e < 32; ++e) w1[(32 * th + e) * HID + hid] = __uint_as_float(r[e]);
+    tmem_ld_32x32b_x32(tq + C_W2 + 64 * half + 32 * th, r);
+    tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) w1[(32 * k + e) * HID + hid] = __uint_as_float(r[e]);
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      uint32_t r[32];
-      tmem_ld_32x32b_x32(tq + C_W2 + 64 * half + 32 * k, r);
-      tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        reinterpret_cast<float4 *>(w2 + 32 * k)[e] =
-            make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                        __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
-    }
+    for (int e = 0; e < 8; ++e)
+      reinterpret_cast<float4 *>(w2)[e] =
+          make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                      __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
   }
   tc_fence_before_sync();
   __syncthreads();
