@@ -71,9 +71,9 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(sources=KERNEL_SOURCES) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(os.path.basename(rel).encode() + b"\0" + f.read())
     return h.hexdigest()[:16]
@@ -87,7 +87,7 @@ def committed_traffic(workload: str):
         with open(path) as f:
             t = json.load(f)
         e = t[workload]
-        if e.get("kernel_source_sha") == kernel_source_sha():
+        if e.get("kernel_source_sha") == kernel_source_sha(tuple(e["kernel_sources"])):
             return float(e["dram_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         pass
@@ -254,12 +254,36 @@ def run_reference(args, cfg):
     return 0
 
 
+def tc_path(cfg, path):
+    return cfg.dtype == "bf16" and cfg.b == 16 and path != "simt"
+
+
 def dtype_of(cfg, path):
-    """Arithmetic type of the path that runs: tensor-core products take bf16 operands
-    (fp32 values split into bf16 hi + lo) with fp32 accumulation; the CUDA-core path
-    is fp32 throughout."""
-    tc = cfg.dtype == "bf16" and cfg.b == 16 and cfg.variant != "mlp" and path != "simt"
-    return "bf16" if tc else "f32"
+    """Arithmetic type of the path that runs.  TTT-Linear on tensor cores: bf16
+    operands (fp32 values split into bf16 hi + lo), fp32 accumulation.  TTT-MLP on
+    tensor cores: tf32 operands, fp16 for the three contractions over the hidden
+    width, fp32 accumulation.  The CUDA-core paths are fp32 throughout."""
+    if not tc_path(cfg, path):
+        return "f32"
+    return "tf32+f16" if cfg.variant == "mlp" else "bf16"
+
+
+# Nominal dense tf32 : bf16 tensor throughput of a B200 (1.1 vs 2.25 PFLOP/s).
+TF32_PER_BF16 = 1.1 / 2.25
+
+
+def tensor_peak_scale(cfg, path):
+    """Peak of the path's contractions relative to the measured bf16 peak.  The
+    TTT-MLP tensor-core path runs, per head-token, 10 d h + 4 b d + 2 b h FLOPs as
+    tf32 ([K;Q] W1, G3 W2^T, both state updates, the masked Q K^T products) and
+    4 d h + 2 b h as fp16 (X2 W2, Zq2 W2 and the Gram Zq2 X2^T); each kind at its
+    own peak gives the time at the roofline."""
+    if cfg.variant != "mlp" or not tc_path(cfg, path):
+        return 1.0
+    d, b, h = cfg.d, cfg.b, cfg.hidden
+    tf32 = 10.0 * d * h + 4.0 * b * d + 2.0 * b * h
+    f16 = 4.0 * d * h + 2.0 * b * h
+    return (tf32 + f16) / (tf32 / TF32_PER_BF16 + f16)
 
 
 def workload_config(cfg, args, world=1):
@@ -430,6 +454,7 @@ def run_momentum(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     cfg = I.CONFIGS["linear_ln_B16H32T8192"]
+    cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T)  # smaller profiling cases
     data = I.make_inputs(cfg)
     B, H, T, d, b = cfg.B, cfg.H, cfg.T, cfg.d, cfg.b
     qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
@@ -492,6 +517,7 @@ def run_backward(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     cfg = I.CONFIGS["linear_ln_B16H32T8192"]
+    cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T)  # smaller profiling cases
     data = I.make_inputs(cfg)
     B, H, T, d, b = cfg.B, cfg.H, cfg.T, cfg.d, cfg.b
     qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
@@ -561,6 +587,8 @@ def run_decode(args, mlp=False, momentum=False):
     else:
         name = "decode_momentum_linear_ln_B512H32" if momentum else "decode_linear_ln_B512H32"
         cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=512, T=16, name=name)
+    if args.batch:  # smaller profiling cases
+        cfg = cfg.replace(B=args.batch)
     data = I.make_inputs(cfg)
     B, H, T, d = cfg.B, cfg.H, cfg.T, cfg.d
     qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
@@ -702,15 +730,21 @@ def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, 
 def finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info, launches, e2e,
            peaks, peak_kind, nbytes, nflops, dist):
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
-    t_tc = nflops / (peaks["bf16_tflops_sustained"] * 1e12)
+    scale = tensor_peak_scale(cfg, args.path)
+    tensor_peak = peaks["bf16_tflops_sustained"] * scale
+    t_tc = nflops / (tensor_peak * 1e12)
     if t_hbm >= t_tc:
         achieved = nbytes / (kernel_avg_ms / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"]}
     else:
         achieved = nflops / (kernel_avg_ms / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops_sustained"]}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": achieved / tensor_peak}
+        if scale != 1.0:
+            roof["peak_mix"] = (f"sustained bf16 x {scale:.3f}: tf32 products at the nominal "
+                                f"{TF32_PER_BF16:.3f} of bf16, fp16 products at the bf16 rate")
+            roof["frac_vs_bf16_peak"] = achieved / peaks["bf16_tflops_sustained"]
     traffic = committed_traffic(cfg.name)
     roof.update({"traffic": traffic, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)"
                  if peak_kind == "measured" else "fallback",
