@@ -171,6 +171,33 @@ TTT_API int ttt_linear_ln_bwd(const void *Q, const void *K, const void *V, int q
                               float *dbeta, float *W_ckpt, void *stream);
 
 /*
+ * Backward pass of TTT-MLP (the gradients of L = <dZ, Z> + <dW1_T, W1_T> +
+ * <dW2_T, W2_T> through the forward of ttt_mlp_fwd; the write-up trains the layer
+ * end to end and computes the backward in the dual form too, §04.3).  Inputs as
+ * for ttt_mlp_fwd, plus
+ *   dZ      [B][H][T][d] fp32: the cotangent of Z.
+ *   dW1_T   [B][H][d][hidden], dW2_T [B][H][hidden][d] fp32, or NULL (zero): the
+ *           cotangents of the final states.
+ * Outputs (fp32, caller-owned, fully written):
+ *   dQ, dK, dV [B][H][T][d];  deta [B][H][T];
+ *   dW1_0 [B][H][d][hidden], dW2_0 [B][H][hidden][d]: per (batch, head) unit (the
+ *           gradient of a state shared by the batch is the sum over the batch);
+ *   dgamma, dbeta [B][H][d]: per unit likewise;
+ *   W1_ckpt [B][H][T/b][d][hidden], W2_ckpt [B][H][T/b][hidden][d]: the state at
+ *           the start of every mini-batch (index 0 = the initial state), which the
+ *           reverse pass reads.
+ * 1 <= b <= 16, d = 64, hidden = 4 d (else TTT_ERR_UNSUPPORTED); T % b == 0.  No
+ * output may overlap an input or another output.  fp32 arithmetic on the CUDA
+ * cores.  Errors as for the forward.
+ */
+TTT_API int ttt_mlp_bwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                        const float *W1_0, const float *W2_0, const float *ln_gamma,
+                        const float *ln_beta, float ln_eps, const float *dZ, const float *dW1_T,
+                        const float *dW2_T, int B, int H, int T, int d, int hidden, int b, float *dQ,
+                        float *dK, float *dV, float *deta, float *dW1_0, float *dW2_0,
+                        float *dgamma, float *dbeta, float *W1_ckpt, float *W2_ckpt, void *stream);
+
+/*
  * The backward of TTT-Linear + LN (ttt_linear_ln_bwd) for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is a property of
  * the library's interface, not of the method.

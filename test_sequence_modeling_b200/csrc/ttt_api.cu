@@ -15,6 +15,7 @@
 #include "ttt.h"
 #include "device_status.cuh"
 #include "backward.cuh"
+#include "backward_mlp.cuh"
 #include "decode.cuh"
 #include "momentum.cuh"
 #include "simt.cuh"
@@ -26,6 +27,7 @@ namespace tc = ttt::tc;
 namespace tcmlp = ttt::tcmlp;
 namespace decode = ttt::decode;
 namespace bwd = ttt::bwd;
+namespace bwdmlp = ttt::bwdmlp;
 namespace mom = ttt::mom;
 
 namespace {
@@ -461,6 +463,67 @@ int run_bwd(bool ln, const void *Q, const void *K, const void *V, int qkv_dtype,
   return TTT_OK;
 }
 
+int run_mlp_bwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                const float *W1_0, const float *W2_0, const float *gamma, const float *beta, float eps,
+                const float *dZ, const float *dW1_T, const float *dW2_T, int B, int H, int T, int d,
+                int hidden, int b, float *dQ, float *dK, float *dV, float *deta, float *dW1,
+                float *dW2, float *dgamma, float *dbeta, float *W1_ckpt, float *W2_ckpt,
+                void *stream) {
+  if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || d <= 0 || hidden <= 0 || b <= 0) return TTT_ERR_ARG;
+  if (T % b != 0) return TTT_ERR_ARG;
+  if (!(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
+  if (d != bwdmlp::D || hidden != bwdmlp::HID || b > bwdmlp::MAXB) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)B * H;
+  if (units == 0) return TTT_OK;
+  if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  const long long elems = units * T * d;
+  if (elems >= (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+  const bool tok = T > 0;
+  const void *req[] = {W1_0, W2_0, gamma, beta, dW1, dW2, dgamma, dbeta,
+                       tok ? Q : W1_0, tok ? K : W1_0, tok ? V : W1_0, tok ? (const void *)eta : W1_0,
+                       tok ? (const void *)dZ : W1_0, tok ? (const void *)dQ : dW1,
+                       tok ? (const void *)dK : dW1, tok ? (const void *)dV : dW1,
+                       tok ? (const void *)deta : dW1, tok ? (const void *)W1_ckpt : dW1,
+                       tok ? (const void *)W2_ckpt : dW1};
+  for (const void *x : req)
+    if (!x) return TTT_ERR_ARG;
+  for (const void *x : req)
+    if (!aligned16(x)) return TTT_ERR_ALIGN;
+  if ((dW1_T && !aligned16(dW1_T)) || (dW2_T && !aligned16(dW2_T))) return TTT_ERR_ALIGN;
+  const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t tbytes = tok ? (size_t)elems * 4 : 0, ibytes = tok ? (size_t)elems * in_elt : 0;
+  const size_t ebytes = tok ? (size_t)units * T * 4 : 0, wbytes = (size_t)units * d * hidden * 4;
+  const size_t hbytes = (size_t)H * d * hidden * 4, pbytes = (size_t)H * d * 4;
+  const size_t vbytes = (size_t)units * d * 4;
+  const size_t cbytes = tok ? (size_t)units * (T / b) * d * hidden * 4 : 0;
+  Range ins[11] = {range_of(Q, ibytes),   range_of(K, ibytes),   range_of(V, ibytes),
+                   range_of(eta, ebytes), range_of(W1_0, hbytes), range_of(W2_0, hbytes),
+                   range_of(gamma, pbytes), range_of(beta, pbytes), range_of(dZ, tbytes),
+                   range_of(dW1_T, dW1_T ? wbytes : 0), range_of(dW2_T, dW2_T ? wbytes : 0)};
+  Range outs[10] = {range_of(dQ, tbytes),      range_of(dK, tbytes),      range_of(dV, tbytes),
+                    range_of(deta, ebytes),    range_of(dW1, wbytes),     range_of(dW2, wbytes),
+                    range_of(dgamma, vbytes),  range_of(dbeta, vbytes),   range_of(W1_ckpt, cbytes),
+                    range_of(W2_ckpt, cbytes)};
+  for (int o = 0; o < 10; ++o) {
+    for (int i = 0; i < 11; ++i)
+      if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
+    for (int o2 = o + 1; o2 < 10; ++o2)
+      if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
+  }
+  bwdmlp::Params p{Q,  K,  V,    eta,  W1_0, W2_0, gamma,  beta,  eps,     dZ,     dW1_T,
+                   dW2_T, H, T, b, dQ,   dK,   dV,    deta,  dW1,    dW2,   dgamma,  dbeta,
+                   W1_ckpt, W2_ckpt};
+  auto kernel = qkv_dtype == TTT_BF16 ? bwdmlp::mlp_bwd_kernel<__nv_bfloat16> : bwdmlp::mlp_bwd_kernel<float>;
+  const size_t smem = bwdmlp::smem_bytes();
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  kernel<<<(unsigned)units, bwdmlp::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int qkv_dtype,
                      const float *eta, const float *alpha, const float *lambda, const float *W0,
                      const float *gamma, const float *beta, float eps, int B, int H, int T, int d,
@@ -660,6 +723,17 @@ int ttt_linear_ln_bwd(const void *Q, const void *K, const void *V, int qkv_dtype
                       float *dbeta, float *W_ckpt, void *stream) {
   return run_bwd(true, Q, K, V, qkv_dtype, eta, W0, ln_gamma, ln_beta, ln_eps, dZ, dW_T, B, H, T, d,
                  b, dQ, dK, dV, deta, dW0, dgamma, dbeta, W_ckpt, stream);
+}
+
+int ttt_mlp_bwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                const float *W1_0, const float *W2_0, const float *ln_gamma, const float *ln_beta,
+                float ln_eps, const float *dZ, const float *dW1_T, const float *dW2_T, int B, int H,
+                int T, int d, int hidden, int b, float *dQ, float *dK, float *dV, float *deta,
+                float *dW1_0, float *dW2_0, float *dgamma, float *dbeta, float *W1_ckpt,
+                float *W2_ckpt, void *stream) {
+  return run_mlp_bwd(Q, K, V, qkv_dtype, eta, W1_0, W2_0, ln_gamma, ln_beta, ln_eps, dZ, dW1_T, dW2_T,
+                     B, H, T, d, hidden, b, dQ, dK, dV, deta, dW1_0, dW2_0, dgamma, dbeta, W1_ckpt,
+                     W2_ckpt, stream);
 }
 
 int ttt_linear_ln_decode(const void *q, const void *k, const void *v, int qkv_dtype,

@@ -20,8 +20,10 @@ W0 (or W1 then W2), gamma, beta.
 
 Two more streams serve the widened paths: ``default_rng([seed, 3, s])`` draws the
 momentum factors alpha ~ U[0, 0.9) and weight decays lambda ~ U[0, 0.05) of the
-momentum and decay update, and ``default_rng([seed, 4, s])`` the incoming
-gradients dZ ~ N(0, 1/d), dW_T ~ N(0, 1/d^2) of the backward pass.
+momentum and decay update, ``default_rng([seed, 4, s])`` the incoming gradients
+dZ ~ N(0, 1/d), dW_T ~ N(0, 1/d^2) of the TTT-Linear backward pass, and
+``default_rng([seed, 5, s])`` those of the TTT-MLP backward (dZ ~ N(0, 1/d),
+dW1_T, dW2_T ~ N(0, 1/(d h))).
 """
 from __future__ import annotations
 
@@ -185,6 +187,18 @@ def cotangents(cfg: TTTConfig, seed: int = 0):
     dZ = (rng.standard_normal((cfg.B, cfg.H, cfg.T, cfg.d), dtype=np.float32) / np.float32(math.sqrt(cfg.d)))
     dWT = (rng.standard_normal((cfg.B, cfg.H, cfg.d, cfg.d), dtype=np.float32) / np.float32(cfg.d))
     return dZ, dWT
+
+
+def mlp_cotangents(cfg: TTTConfig, seed: int = 0):
+    """Incoming gradients for the TTT-MLP backward: dZ [B, H, T, d] ~ N(0, 1/d) and
+    dW1_T [B, H, d, h], dW2_T [B, H, h, d] ~ N(0, 1/(d h)), float32, from the stream
+    default_rng([seed, 5, s])."""
+    rng = np.random.default_rng([cfg.seed, 5, seed])
+    dZ = (rng.standard_normal((cfg.B, cfg.H, cfg.T, cfg.d), dtype=np.float32) / np.float32(math.sqrt(cfg.d)))
+    sc = np.float32(1.0 / math.sqrt(cfg.d * cfg.hidden))
+    dW1 = rng.standard_normal((cfg.B, cfg.H, cfg.d, cfg.hidden), dtype=np.float32) * sc
+    dW2 = rng.standard_normal((cfg.B, cfg.H, cfg.hidden, cfg.d), dtype=np.float32) * sc
+    return dZ, dW1, dW2
 
 
 def unit_as_f64(cfg: TTTConfig, bi: int, hi: int, T: int | None = None) -> dict:

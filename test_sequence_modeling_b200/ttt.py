@@ -201,6 +201,46 @@ def ttt_linear_bwd(Q, K, V, eta, W0, dZ, b, dW_T=None, gamma=None, beta=None, ep
     return out
 
 
+def ttt_mlp_bwd(Q, K, V, eta, W1, W2, gamma, beta, dZ, b, eps=1e-6, dW1_T=None, dW2_T=None, stream=None):
+    """Backward of ttt_mlp_fwd: the gradients of <dZ, Z> + <dW1_T, W1_T> + <dW2_T, W2_T>.
+    dZ [B,H,T,d] f32; dW1_T [B,H,d,h], dW2_T [B,H,h,d] f32 or None.  Returns a dict:
+    dQ, dK, dV, deta, dW1, dW2 (per unit), dgamma, dbeta [B,H,d] and the per-mini-batch
+    states W1_ckpt [B,H,T/b,d,h], W2_ckpt [B,H,T/b,h,d]."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    h = W1.shape[-1]
+    _shaped(eta, "eta", (B, H, T))
+    _shaped(W1, "W1", (H, d, h))
+    _shaped(W2, "W2", (H, h, d))
+    _shaped(dZ, "dZ", (B, H, T, d))
+    for n, t in (("gamma", gamma), ("beta", beta)):
+        _shaped(t, n, (H, d))
+    if dW1_T is not None:
+        _shaped(dW1_T, "dW1_T", (B, H, d, h))
+    if dW2_T is not None:
+        _shaped(dW2_T, "dW2_T", (B, H, h, d))
+    if b <= 0 or T % b:
+        raise ValueError("T must be a multiple of b")
+    dev = Q.device
+    out = {n: torch.empty(B, H, T, d, device=dev) for n in ("dQ", "dK", "dV")}
+    out["deta"] = torch.empty(B, H, T, device=dev)
+    out["dW1"] = torch.empty(B, H, d, h, device=dev)
+    out["dW2"] = torch.empty(B, H, h, d, device=dev)
+    out["dgamma"] = torch.empty(B, H, d, device=dev)
+    out["dbeta"] = torch.empty(B, H, d, device=dev)
+    out["W1_ckpt"] = torch.empty(B, H, T // b, d, h, device=dev)
+    out["W2_ckpt"] = torch.empty(B, H, T // b, h, d, device=dev)
+    o = {k: _ptr(v) for k, v in out.items()}
+    with torch.cuda.device(dev):
+        st = _lib.load().ttt_mlp_bwd(
+            _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W1), _ptr(W2), _ptr(gamma), _ptr(beta),
+            float(eps), _ptr(dZ), _ptr(dW1_T), _ptr(dW2_T), B, H, T, d, h, int(b), o["dQ"], o["dK"],
+            o["dV"], o["deta"], o["dW1"], o["dW2"], o["dgamma"], o["dbeta"], o["W1_ckpt"], o["W2_ckpt"],
+            _stream(stream, dev))
+    check(st, "ttt_mlp_bwd")
+    return out
+
+
 def ttt_linear_ln_bwd_noalloc(Q, K, V, eta, W0, dZ, b, gamma, beta, eps=1e-6, dW_T=None, out=None,
                               stream=None):
     """The backward of ttt_linear_ln_fwd for callers that must not allocate device
