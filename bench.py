@@ -445,6 +445,69 @@ def main():
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
+def run_momentum_mlp(args):
+    """One launch of ttt_mlp_momentum_fwd over the TTT-MLP workload (B=8 H=32 T=8192, b=16)."""
+    import torch
+    import test_sequence_modeling_b200 as ttt
+    from test_sequence_modeling_b200 import _lib
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    cfg = I.CONFIGS["mlp_B8H32T8192"]
+    cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T)  # smaller profiling cases
+    data = I.make_inputs(cfg)
+    B, H, T, d, b, h = cfg.B, cfg.H, cfg.T, cfg.d, cfg.b, cfg.hidden
+    qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
+    t = {k: torch.from_numpy(np.ascontiguousarray(data[k])).to(dev) for k in ("eta", "W1", "W2", "gamma", "beta")}
+    alpha, lam = (torch.from_numpy(x).to(dev) for x in I.momentum_rates(cfg))
+    stream = torch.cuda.current_stream(dev)
+    lib = _lib.load()
+
+    def step():
+        return ttt.ttt_mlp_momentum_fwd(qkv["Q"], qkv["K"], qkv["V"], t["eta"], alpha, lam, t["W1"], t["W2"],
+                                        t["gamma"], t["beta"], b, cfg.ln_eps, stream=stream)
+
+    outs = step()
+    del outs
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(gpu_id_for(torch, 0))
+    clocks.start()
+    n0 = lib.ttt_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    launches = lib.ttt_launch_count() - n0
+    clock_info = clocks.stop()
+    if ttt.last_device_status() != 0:
+        raise RuntimeError("device status error")
+    ms = e0.elapsed_time(e1) / args.steps
+    units, N = B * H, T // b
+    # Multiply-adds per mini-batch: K W1, X2 W2, G3 W2^T (3 b d h), Q W1 + Q S1 and
+    # Zq2 W2 + Zq2 S2 (4 b d h), the two rank-b updates of W and S of both layers
+    # (4 b d h), the masked Grams and their products (b^2 (2 h + 2 d)).
+    flops = 2.0 * units * N * (11 * b * d * h + 2 * b * b * (h + d))
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {
+        "metric": "TTT-MLP momentum/decay forward tokens/s (B x H x T / s)",
+        "value": units * T / (ms / 1e3), "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "momentum_" + cfg.name, "B": B, "H": H, "T": T, "d": d, "b": b,
+                   "hidden": h, "qkv_dtype": "bf16", "l2": "inputs larger than L2 (no flush needed)"},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": ALU_F32_TFLOPS, "unit": "TFLOP/s",
+                     "frac": achieved / ALU_F32_TFLOPS, "traffic": None,
+                     "peak_source": "148 SMs x 128 FP32 lanes x 2 x 1965 MHz (CUDA-core fp32 FMA)",
+                     "flops_per_launch": flops},
+        "clocks": clock_info, "gpu_launches": int(launches),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_backward_mlp(args):
     """One launch of ttt_mlp_bwd over the TTT-MLP workload (B=8 H=32 T=8192, b=16)."""
     import torch
@@ -511,7 +574,10 @@ def run_backward_mlp(args):
 
 def run_momentum(args):
     """The momentum and decay forward's own line: one step = one launch of
-    ttt_linear_ln_momentum_fwd over the linear + LN workload (B=16 H=32 T=8192, b=16)."""
+    ttt_linear_ln_momentum_fwd over the linear + LN workload (B=16 H=32 T=8192, b=16),
+    or (``--workload mlp_B8H32T8192``) of ttt_mlp_momentum_fwd over the TTT-MLP one."""
+    if args.workload.startswith("mlp"):
+        return run_momentum_mlp(args)
     import torch
     import test_sequence_modeling_b200 as ttt
     from test_sequence_modeling_b200 import _lib

@@ -143,6 +143,24 @@ TTT_API int ttt_linear_ln_momentum_fwd(const void *Q, const void *K, const void 
                                        void *stream);
 
 /*
+ * The same momentum and decay forward on the TTT-MLP memory, f(x) = x + LN(GELU(x
+ * W1) W2) (the Titans article's memory is an MLP, §二.1(3)): both layers follow
+ *   S_t = alpha_t S_{t-1} - eta_t g_t,  W_t = (1 - lambda_t) W_{t-1} + S_t,
+ * with g_t the loss gradient at the mini-batch base, z_t = f(q_t; W1_t, W2_t).
+ * Inputs as for ttt_mlp_fwd plus alpha, lambda [B][H][T] fp32.  Outputs: Z
+ * [B][H][T][d]; W1_out, S1_out [B][H][d][hidden]; W2_out, S2_out [B][H][hidden][d]
+ * (the final states and momenta), fp32.  1 <= b <= 16, d = 64, hidden = 4 d (else
+ * TTT_ERR_UNSUPPORTED), T % b == 0.  fp32 arithmetic on the CUDA cores.  Errors as
+ * for the forward entry points.
+ */
+TTT_API int ttt_mlp_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                                 const float *eta, const float *alpha, const float *lambda,
+                                 const float *W1_0, const float *W2_0, const float *ln_gamma,
+                                 const float *ln_beta, float ln_eps, int B, int H, int T, int d,
+                                 int hidden, int b, float *Z, float *W1_out, float *W2_out,
+                                 float *S1_out, float *S2_out, void *stream);
+
+/*
  * Backward pass of TTT-Linear (and, _ln_, TTT-Linear with LN and residual): the
  * gradients of L = <dZ, Z> + <dW_T, W_T> through the forward of ttt_linear_fwd /
  * ttt_linear_ln_fwd (the write-up trains the layer end to end and computes the

@@ -35,6 +35,8 @@ SIGNATURES = {
                             _fp, _fp, _fp, _vp]),
     "ttt_linear_ln_bwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _f, _fp, _fp, _i, _i, _i, _i, _i,
                                _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _vp]),
+    "ttt_mlp_momentum_fwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i, _i,
+                                  _i, _i, _fp, _fp, _fp, _fp, _fp, _vp]),
     "ttt_mlp_bwd": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _f, _fp, _fp, _fp, _i, _i, _i, _i,
                          _i, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _vp]),
     "ttt_linear_ln_bwd_noalloc": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _f, _fp, _fp, _i, _i, _i, _i,

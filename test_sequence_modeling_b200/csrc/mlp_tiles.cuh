@@ -1,0 +1,147 @@
+// mlp_tiles.cuh - fp32 CUDA-core building blocks of the TTT-MLP kernels that
+// keep one mini-batch's [b x hidden] and [b x d] tiles in shared memory and
+// stream the [d x hidden] matrices (state, cotangents, momenta) from global
+// memory: products of a tile with such a matrix (coalesced matrix loads,
+// warp-wide broadcast tile reads), rank-b updates of a matrix, masked b x b
+// Grams and their products, for a CTA of 16 warps and b <= 16.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace ttt {
+namespace mlptile {
+
+constexpr int D = 64;
+constexpr int HID = 256;
+constexpr int MAXB = 16;     // largest mini-batch of this kernel
+constexpr int THREADS = 512;
+constexpr int LDD = D + 4;   // row stride of the [b][d] tiles (16-byte aligned rows)
+constexpr int LDH = HID + 4; // row stride of the [b][hidden] tiles
+constexpr int LDB = MAXB + 1;
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ float wsum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+__device__ __forceinline__ float phi(float x) { return 0.398942280401432678f * expf(-0.5f * x * x); }
+__device__ __forceinline__ float gelu(float x) { return x * normcdff(x); }
+__device__ __forceinline__ float gelu_d(float x) { return normcdff(x) + x * phi(x); }
+
+// out[t][j] (+/-)= sum_k A[t][k] W[k][j]   (W global, row-major [Kd][N], written
+// earlier in this kernel or by the caller: plain loads, not the read-only path).
+template <int N>
+__device__ void mm_W(float *out, int ldo, const float *A, int lda, const float *W, int Kd, int b,
+                     float sign, bool acc, int tid) {
+  constexpr int TPC = THREADS / N, RPT = MAXB / TPC;
+  const int j = tid % N, g = tid / N;
+  float a[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) a[r] = 0.f;
+#pragma unroll 4
+  for (int k = 0; k < Kd; ++k) {
+    const float w = W[(size_t)k * N + j];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) a[r] = fmaf(A[(g * RPT + r) * lda + k], w, a[r]);
+  }
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int t = g * RPT + r;
+    if (t < b) out[t * ldo + j] = (acc ? out[t * ldo + j] : 0.f) + sign * a[r];
+  }
+}
+
+// out[t][j] (+/-)= sum_k A[t][k] W[j][k]   (W global, row-major [N][Kd]).
+template <int N>
+__device__ void mm_WT(float *out, int ldo, const float *A, int lda, const float *W, int Kd, int b,
+                      float sign, bool acc, int tid) {
+  constexpr int TPC = THREADS / N, RPT = MAXB / TPC;
+  const int j = tid % N, g = tid / N;
+  float a[RPT];
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) a[r] = 0.f;
+  const float4 *wr = reinterpret_cast<const float4 *>(W + (size_t)j * Kd);
+#pragma unroll 2
+  for (int k = 0; k < Kd; k += 4) {
+    const float4 w = wr[k >> 2];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+      const float4 x = *reinterpret_cast<const float4 *>(A + (g * RPT + r) * lda + k);
+      a[r] = fmaf(x.x, w.x, fmaf(x.y, w.y, fmaf(x.z, w.z, fmaf(x.w, w.w, a[r]))));
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int t = g * RPT + r;
+    if (t < b) out[t * ldo + j] = (acc ? out[t * ldo + j] : 0.f) + sign * a[r];
+  }
+}
+
+// out[t][j] += sign sum_{s<b} S[t][s] B[s][j]  (or S[s][t] when trans); the same
+// (t, j) ownership as mm_W / mm_WT with this N, so it may follow them without a
+// barrier.
+template <int N>
+__device__ void small_corr(float *out, int ldo, const float *S, bool trans, const float *B, int ldb,
+                           int b, float sign, int tid) {
+  constexpr int TPC = THREADS / N, RPT = MAXB / TPC;
+  const int j = tid % N, g = tid / N;
+#pragma unroll
+  for (int r = 0; r < RPT; ++r) {
+    const int t = g * RPT + r;
+    if (t >= b) continue;
+    float v = 0.f;
+    for (int s = 0; s < b; ++s) v = fmaf(trans ? S[s * LDB + t] : S[t * LDB + s], B[s * ldb + j], v);
+    out[t * ldo + j] += sign * v;
+  }
+}
+
+// dst[r][c] = src[r][c] + sign sum_{t<b} L[t][r] Rt[t][c]   (dst, src global [R][C];
+// dst may be src: each thread reads and writes only its own entries).
+template <int R, int C>
+__device__ void outer(float *dst, const float *src, const float *L, int ldl, const float *Rt, int ldr,
+                      int b, float sign, int tid) {
+  constexpr int GROUPS = THREADS / C, RPG = R / GROUPS;
+  const int c = tid % C, g = tid / C;
+  float rt[MAXB];
+#pragma unroll
+  for (int t = 0; t < MAXB; ++t) rt[t] = t < b ? Rt[t * ldr + c] : 0.f;
+  for (int i = 0; i < RPG; ++i) {
+    const int r = g * RPG + i;
+    float a = 0.f;
+#pragma unroll
+    for (int t = 0; t < MAXB; ++t)
+      if (t < b) a = fmaf(L[t * ldl + r], rt[t], a);
+    dst[(size_t)r * C + c] = src[(size_t)r * C + c] + sign * a;
+  }
+}
+
+// S[t][s] = sum_k A[t][k] B[s][k] for s <= t < b (zero elsewhere).
+__device__ void gram_tril(float *S, const float *A, int lda, const float *B, int ldb, int Kd, int b,
+                          int tid) {
+  const int p = tid >> 1, hf = tid & 1;
+  const int t = p >> 4, s = p & 15;
+  float v = 0.f;
+  if (t < b && s <= t) {
+    const int k0 = hf * (Kd / 2);
+    for (int k = k0; k < k0 + Kd / 2; k += 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(A + t * lda + k);
+      const float4 y = *reinterpret_cast<const float4 *>(B + s * ldb + k);
+      v = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, v))));
+    }
+  }
+  v += __shfl_xor_sync(0xffffffffu, v, 1);
+  if (hf == 0) S[t * LDB + s] = (t < b && s <= t) ? v : 0.f;
+}
+
+template <typename InT>
+__device__ void load_rows(float *dst, const InT *src, long row0, int b, int tid) {
+  for (int x = tid; x < b * D; x += THREADS) dst[(x / D) * LDD + x % D] = to_f(src[(row0 + x / D) * D + x % D]);
+}
+
+}  // namespace mlptile
+}  // namespace ttt

@@ -18,6 +18,7 @@
 #include "backward_mlp.cuh"
 #include "decode.cuh"
 #include "momentum.cuh"
+#include "momentum_mlp.cuh"
 #include "simt.cuh"
 #include "tc_linear.cuh"
 #include "tc_mlp.cuh"
@@ -29,6 +30,7 @@ namespace decode = ttt::decode;
 namespace bwd = ttt::bwd;
 namespace bwdmlp = ttt::bwdmlp;
 namespace mom = ttt::mom;
+namespace mommlp = ttt::mommlp;
 
 namespace {
 
@@ -577,6 +579,58 @@ int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int q
   return TTT_OK;
 }
 
+int run_mlp_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                         const float *eta, const float *alpha, const float *lambda,
+                         const float *W1_0, const float *W2_0, const float *gamma, const float *beta,
+                         float eps, int B, int H, int T, int d, int hidden, int b, float *Z,
+                         float *W1, float *W2, float *S1, float *S2, void *stream) {
+  if (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) return TTT_ERR_ARG;
+  if (B < 0 || H < 0 || T < 0 || d <= 0 || hidden <= 0 || b <= 0) return TTT_ERR_ARG;
+  if (T % b != 0) return TTT_ERR_ARG;
+  if (!(std::isfinite(eps) && eps > 0.f)) return TTT_ERR_ARG;
+  if (d != mommlp::D || hidden != mommlp::HID || b > mommlp::MAXB) return TTT_ERR_UNSUPPORTED;
+  const long long units = (long long)B * H;
+  if (units == 0) return TTT_OK;
+  if (units > 0x7fffffffLL) return TTT_ERR_UNSUPPORTED;
+  const long long elems = units * T * d;
+  if (elems >= (1LL << 40)) return TTT_ERR_UNSUPPORTED;
+  const bool tok = T > 0;
+  const void *req[] = {W1_0, W2_0, gamma, beta, W1, W2, S1, S2,
+                       tok ? Q : W1_0, tok ? K : W1_0, tok ? V : W1_0, tok ? (const void *)eta : W1_0,
+                       tok ? (const void *)alpha : W1_0, tok ? (const void *)lambda : W1_0,
+                       tok ? (const void *)Z : W1};
+  for (const void *x : req)
+    if (!x) return TTT_ERR_ARG;
+  for (const void *x : req)
+    if (!aligned16(x)) return TTT_ERR_ALIGN;
+  const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t ibytes = tok ? (size_t)elems * in_elt : 0, ebytes = tok ? (size_t)units * T * 4 : 0;
+  const size_t hbytes = (size_t)H * d * hidden * 4, pbytes = (size_t)H * d * 4;
+  const size_t wbytes = (size_t)units * d * hidden * 4;
+  Range ins[10] = {range_of(Q, ibytes),    range_of(K, ibytes),      range_of(V, ibytes),
+                   range_of(eta, ebytes),  range_of(alpha, ebytes),  range_of(lambda, ebytes),
+                   range_of(W1_0, hbytes), range_of(W2_0, hbytes),   range_of(gamma, pbytes),
+                   range_of(beta, pbytes)};
+  Range outs[5] = {range_of(Z, tok ? (size_t)elems * 4 : 0), range_of(W1, wbytes), range_of(W2, wbytes),
+                   range_of(S1, wbytes), range_of(S2, wbytes)};
+  for (int o = 0; o < 5; ++o) {
+    for (int i = 0; i < 10; ++i)
+      if (overlap(outs[o], ins[i])) return TTT_ERR_ARG;
+    for (int o2 = o + 1; o2 < 5; ++o2)
+      if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
+  }
+  mommlp::Params p{Q, K, V, eta, alpha, lambda, W1_0, W2_0, gamma, beta, eps, H, T, b, Z, W1, W2, S1, S2};
+  auto kernel = qkv_dtype == TTT_BF16 ? mommlp::mlp_momentum_fwd_kernel<__nv_bfloat16>
+                                      : mommlp::mlp_momentum_fwd_kernel<float>;
+  const size_t smem = mommlp::smem_bytes();
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  kernel<<<(unsigned)units, mommlp::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 int run(const Call &c) {
   const int st = validate(c);
   if (st != TTT_OK) return st;
@@ -723,6 +777,16 @@ int ttt_linear_ln_bwd(const void *Q, const void *K, const void *V, int qkv_dtype
                       float *dbeta, float *W_ckpt, void *stream) {
   return run_bwd(true, Q, K, V, qkv_dtype, eta, W0, ln_gamma, ln_beta, ln_eps, dZ, dW_T, B, H, T, d,
                  b, dQ, dK, dV, deta, dW0, dgamma, dbeta, W_ckpt, stream);
+}
+
+int ttt_mlp_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
+                         const float *eta, const float *alpha, const float *lambda,
+                         const float *W1_0, const float *W2_0, const float *ln_gamma,
+                         const float *ln_beta, float ln_eps, int B, int H, int T, int d, int hidden,
+                         int b, float *Z, float *W1_out, float *W2_out, float *S1_out, float *S2_out,
+                         void *stream) {
+  return run_mlp_momentum_fwd(Q, K, V, qkv_dtype, eta, alpha, lambda, W1_0, W2_0, ln_gamma, ln_beta,
+                              ln_eps, B, H, T, d, hidden, b, Z, W1_out, W2_out, S1_out, S2_out, stream);
 }
 
 int ttt_mlp_bwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,

@@ -201,6 +201,32 @@ def ttt_linear_bwd(Q, K, V, eta, W0, dZ, b, dW_T=None, gamma=None, beta=None, ep
     return out
 
 
+def ttt_mlp_momentum_fwd(Q, K, V, eta, alpha, lam, W1, W2, gamma, beta, b, eps=1e-6, stream=None):
+    """TTT-MLP forward with the momentum and decay update.  Q, K, V [B,H,T,d]; eta,
+    alpha, lam [B,H,T] f32; W1 [H,d,h], W2 [H,h,d]; gamma, beta [H,d].  Returns
+    (Z [B,H,T,d], W1 [B,H,d,h], W2 [B,H,h,d], S1 [B,H,d,h], S2 [B,H,h,d])."""
+    dt = _qkv(Q, K, V)
+    B, H, T, d = Q.shape
+    h = W1.shape[-1]
+    for n, t in (("eta", eta), ("alpha", alpha), ("lambda", lam)):
+        _shaped(t, n, (B, H, T))
+    _shaped(W1, "W1", (H, d, h))
+    _shaped(W2, "W2", (H, h, d))
+    for n, t in (("gamma", gamma), ("beta", beta)):
+        _shaped(t, n, (H, d))
+    dev = Q.device
+    Z = torch.empty(B, H, T, d, device=dev)
+    W1o, S1o = (torch.empty(B, H, d, h, device=dev) for _ in range(2))
+    W2o, S2o = (torch.empty(B, H, h, d, device=dev) for _ in range(2))
+    with torch.cuda.device(dev):
+        st = _lib.load().ttt_mlp_momentum_fwd(
+            _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(alpha), _ptr(lam), _ptr(W1), _ptr(W2),
+            _ptr(gamma), _ptr(beta), float(eps), B, H, T, d, h, int(b), _ptr(Z), _ptr(W1o), _ptr(W2o),
+            _ptr(S1o), _ptr(S2o), _stream(stream, dev))
+    check(st, "ttt_mlp_momentum_fwd")
+    return Z, W1o, W2o, S1o, S2o
+
+
 def ttt_mlp_bwd(Q, K, V, eta, W1, W2, gamma, beta, dZ, b, eps=1e-6, dW1_T=None, dW2_T=None, stream=None):
     """Backward of ttt_mlp_fwd: the gradients of <dZ, Z> + <dW1_T, W1_T> + <dW2_T, W2_T>.
     dZ [B,H,T,d] f32; dW1_T [B,H,d,h], dW2_T [B,H,h,d] f32 or None.  Returns a dict:

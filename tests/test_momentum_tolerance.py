@@ -20,9 +20,9 @@ def _ln(y, g, bt, eps):
     return g * (y - mu) / torch.sqrt(var + eps) + bt
 
 
-def fp32_spread(b, B=2, H=3, T=32):
+def fp32_spread(b, B=2, H=3, T=32, dtype="bf16"):
     """Max relative Frobenius error of the fp32 evaluation against the oracle, per output."""
-    cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=B, H=H, T=T, b=b)
+    cfg = I.CONFIGS["mlp_B8H32T8192"].replace(B=B, H=H, T=T, b=b, dtype=dtype)
     alpha, lam = I.momentum_rates(cfg)
     gelu = torch.nn.functional.gelu
     worst = {}
@@ -71,3 +71,13 @@ def test_fp32_spread_of_the_mlp_momentum_recursion():
     assert max(spread.values()) > 1e-5, spread
     # ... and the tolerance leaves no more than a small factor above it.
     assert max(spread.values()) * 1.5 <= MLP_MOMENTUM_TOL, spread
+
+
+def test_fp32_spread_of_the_whole_sequence_mlp_momentum_forward():
+    """The same recursion as the TTT-MLP momentum forward runs it: over longer
+    sequences (T = 256, b = 16) and with fp32 inputs (b = 4) the fp32 spread also
+    exceeds 1e-5, so that forward's GPU test uses MLP_MOMENTUM_TOL throughout."""
+    for kw in (dict(b=16, B=1, H=2, T=256), dict(b=4, T=48, dtype="f32")):
+        spread = fp32_spread(**kw)
+        assert max(spread.values()) > 1e-5, (kw, spread)
+        assert max(spread.values()) * 1.5 <= MLP_MOMENTUM_TOL, (kw, spread)
