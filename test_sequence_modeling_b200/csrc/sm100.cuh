@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace ttt {
 namespace sm100 {
@@ -336,6 +337,17 @@ __device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+      : "memory");
+}
+
 // tcgen05.commit by the lane elect.sync picks (the same lane that issued the
 // products above), executed by the whole converged warp.
 __device__ __forceinline__ void umma_commit_w(uint64_t *bar) {
@@ -410,6 +422,12 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t &hi, uin
   __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
   hi = *reinterpret_cast<uint32_t *>(&h);
   lo = *reinterpret_cast<uint32_t *>(&l);
+}
+
+// Packs two floats as fp16 (round to nearest even): a in the low half, b in the high.
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 v = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&v);
 }
 
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {

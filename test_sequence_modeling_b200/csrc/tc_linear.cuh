@@ -29,27 +29,27 @@
 //   1. TMA: K and Q (8-row boxes into that layout, 128-byte swizzle), V
 //      (64 x 64), eta.
 //   2. tcgen05: S = [K;Q] K^T (TMEM cols 64..127) and P = [K;Q] W_c (cols 0..63).
-//   3. Every thread masks its own row of S in TMEM, in place, into the A operand
-//      of step 4 (bf16 hi in the columns of the first half of each mini-batch,
-//      lo in those of the second): K rows keep the columns of earlier
-//      mini-batches, Q rows keep s <= t (the causal mask of the dual form,
-//      diagonal included).
+//   3. Every thread masks its own row of S in TMEM, in place, into the fp16 A
+//      operand of step 4: K rows keep the columns of earlier mini-batches, Q
+//      rows keep s <= t (the causal mask of the dual form, diagonal included).
 //   4. For m = 0..3, the two warps that hold mini-batch m read its K rows of P
 //      (already corrected for mini-batches < m), compute G_m (LN backward in
-//      registers, 16 elements per thread), write eta*G_m as bf16 hi + lo, meet
-//      at a named barrier, and one of them issues P -= A[:, m] (eta G_m) (A read
-//      from TMEM), which applies mini-batch m's update to every later K row and
-//      every Q row at once.  Once their chain steps are issued, the warps write
-//      the outputs of their Q rows, which are final after their mini-batch's
-//      update (later updates add exactly zero to them).
-//   5. dW = K^T (eta G) on the tensor core into the S columns (free again);
-//      every thread updates its 32 fp32 state elements and rewrites the bf16
-//      hi + lo operand copy of W; then steps 1-3 of the next chunk follow
+//      registers, 16 elements per thread), write eta*G_m as fp16, turn their K
+//      rows into fp16 in place, meet at a named barrier, and one of them issues
+//      P -= A[:, m] (eta G_m) (A read from TMEM), which applies mini-batch m's
+//      update to every later K row and every Q row at once.  Once their chain
+//      steps are issued, the warps write the outputs of their Q rows, which are
+//      final after their mini-batch's update (later updates add exactly zero to
+//      them).
+//   5. dW = K^T (eta G) on the tensor core (fp16) into the S columns (free
+//      again); every thread updates its 32 fp32 state elements and rewrites the
+//      bf16 hi + lo operand copy of W; then steps 1-3 of the next chunk follow
 //      directly (the next K, V are fetched as soon as dW is done, each warp's Q
 //      rows as soon as it has written its outputs).
-// Precision: every fp32 operand (W, eta*G, the masked Q K^T) enters the tensor
-// core as a bf16 pair hi + lo (error ~2^-16 relative); K and Q are exact bf16;
-// accumulation is fp32.
+// Precision: W enters P = [K;Q] W as a bf16 pair hi + lo (~2^-16 relative) against
+// the exact bf16 K and Q; the masked Q K^T, eta*G and K enter the chain's
+// corrections and dW as fp16 (2^-11 relative); accumulation is fp32 and the
+// state stays fp32 in registers.
 #pragma once
 
 #include <cuda.h>
@@ -74,8 +74,8 @@ constexpr uint32_t TMEM_COLS = 128;
 constexpr uint32_t OFF_A = 0;          // [K;Q] rows of the chunk in 8-row groups (see kq_group)
 constexpr uint32_t OFF_WHI = 16384;    // W hi [d_in][d_out] bf16
 constexpr uint32_t OFF_WLO = 24576;    // W lo
-constexpr uint32_t OFF_GHI = 32768;    // eta*G hi [token][d_out] bf16
-constexpr uint32_t OFF_GLO = 40960;    // V tile on arrival; eta*G lo once a mini-batch is done
+constexpr uint32_t OFF_GHI = 32768;    // eta*G [token][d_out] fp16
+constexpr uint32_t OFF_GLO = 40960;    // V tile
 constexpr uint32_t OFF_ETA = 49152;    // eta of the chunk, 64 floats
 constexpr uint32_t OFF_GB = 49408;     // per column pair {gamma x2, beta x2}, 32 x 16 bytes
 constexpr uint32_t OFF_UC = 49920;     // per column pair {2 gamma x2, 2 gamma beta x2}
@@ -166,8 +166,9 @@ __global__ void __launch_bounds__(THREADS, 4)
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, as an offset into the shared array so that every
+  // access through it stays a shared-memory access.
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int unit = blockIdx.x;
   const int head = unit % p.H;
@@ -282,8 +283,8 @@ __global__ void __launch_bounds__(THREADS, 4)
 
   constexpr uint32_t ID_P = idesc_bf16_f32(128, 64, false, true, false);   // [K;Q] x W
   constexpr uint32_t ID_S = idesc_bf16_f32(128, 64, false, false, false);  // [K;Q] x K^T
-  constexpr uint32_t ID_UPD = idesc_bf16_f32(128, 64, false, true, true);  // P -= A x (eta G)
-  constexpr uint32_t ID_DW = idesc_bf16_f32(128, 64, true, true, false);   // [K^T;K^T] x (eta G)
+  constexpr uint32_t ID_UPD = idesc_f16_f32(128, 64, false, true, true);   // P -= A x (eta G), fp16
+  constexpr uint32_t ID_DW = idesc_f16_f32(128, 64, true, true, false);    // [K^T;K^T] x (eta G), fp16
 
   // The P-independent part of the LN backward of this thread's K row of token
   // tk: u = 2 gamma (k + beta - v) = g2 (k - v) + g2b (or v for the plain linear
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(THREADS, 4)
     for (int j = 0; j < 8; ++j) {
       const int col = 8 * j + 2 * q4;
       vr[j] = lds_u32(aGlo + sw128_offset(tk, col));
-      if (LN) kr[j] = lds_u32(sbase + kq_offset(tk, 0, col));
+      kr[j] = lds_u32(sbase + kq_offset(tk, 0, col));
     }
   };
   auto make_u = [&]() {
@@ -329,29 +330,26 @@ __global__ void __launch_bounds__(THREADS, 4)
     // drain at the end waits for them).
     if (warp == 0) {
       __syncwarp();
-      const bool issue = elect_one_sync();
       tc_fence_after_sync();
       // S = [K;Q] K^T: B = the K rows alone (every other 8-row group, 2 KB apart).
 #pragma unroll
       for (int k = 0; k < 4; ++k)
-        if (issue)
-          umma_ss(tS, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aA + 32 * k, 16, 2048), ID_S,
+        umma_ss_w(tS, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aA + 32 * k, 16, 2048), ID_S,
                   k > 0);
-      if (issue) umma_commit(&bars[BAR_S]);
+      umma_commit_w(&bars[BAR_S]);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint64_t ak = smem_desc_sw128(aA + 32 * k, 16, 1024);
-        if (issue) umma_ss(tP, ak, smem_desc_sw128(aWhi + 2048 * k, 8192, 1024), ID_P, k > 0);
-        if (issue) umma_ss(tP, ak, smem_desc_sw128(aWlo + 2048 * k, 8192, 1024), ID_P, true);
+        umma_ss_w(tP, ak, smem_desc_sw128(aWhi + 2048 * k, 8192, 1024), ID_P, k > 0);
+        umma_ss_w(tP, ak, smem_desc_sw128(aWlo + 2048 * k, 8192, 1024), ID_P, true);
       }
-      if (issue) umma_commit(&bars[BAR_P]);
+      umma_commit_w(&bars[BAR_P]);
       __syncwarp();
     }
     if (ntok < CHUNK) {  // ragged last chunk: absent tokens contribute nothing to dW
       for (int x = tid; x < (CHUNK - ntok) * 32; x += THREADS) {
         const int row = ntok + x / 32, col = 2 * (x % 32);
         *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(row, col)) = 0u;
-        *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(row, col)) = 0u;
       }
     }
     wait_or_abort(&bars[BAR_S], par, abort);
@@ -364,12 +362,11 @@ __global__ void __launch_bounds__(THREADS, 4)
       const int t = MB * mrow + 8 * hh + (lane & 7);  // its token
       // A block j (tokens 16j..16j+15, natural order) is read from S columns
       // 8j..8j+7 (first half) and 32+8j..32+8j+7 (second half) and written back
-      // in place: hi over the first, lo over the second.  Blocks j > mb0 + 1 are
-      // zero for every row of this warp (the choice is per warp: TMEM access is
-      // warp-collective).
+      // as fp16 pairs over the first.  Blocks j > mb0 + 1 are zero for every row
+      // of this warp (the choice is per warp: TMEM access is warp-collective).
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        uint32_t hi[8], lo[8];
+        uint32_t pk[8];
         if (j <= mb0 + 1) {
           uint32_t v0[8], v1[8];
           tmem_ld_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), v0);
@@ -384,14 +381,13 @@ __global__ void __launch_bounds__(THREADS, 4)
             const uint32_t b1 = e < 4 ? v0[2 * e + 1] : v1[2 * e - 7];
             const float a0 = (full || (diag && s0 <= t)) ? __uint_as_float(b0) : 0.f;
             const float a1 = (full || (diag && s0 + 1 <= t)) ? __uint_as_float(b1) : 0.f;
-            split_bf16x2(a0, a1, hi[e], lo[e]);
+            pk[e] = pack_f16x2(a0, a1);
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) hi[e] = lo[e] = 0u;
+          for (int e = 0; e < 8; ++e) pk[e] = 0u;
         }
-        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), hi);
-        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 32 + 8 * j), lo);
+        tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), pk);
       }
       tmem_wait_st();
     }
@@ -425,13 +421,9 @@ __global__ void __launch_bounds__(THREADS, 4)
       __syncwarp();
       float2 y[8];
       tmem_rows_16x256b(tmem_addr(tP, 32 * warp + 16 * i, 0), 0, y);
-      // Stores eta * (dl/dy) of one column pair as bf16 hi + lo; the lo half
-      // overwrites V, which this thread has read for exactly these cells.
+      // Stores eta * (dl/dy) of one column pair as fp16.
       auto store_grad = [&](int col, float2 g) {
-        uint32_t h, l;
-        split_bf16x2(g.x, g.y, h, l);
-        *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(tk, col)) = h;
-        *reinterpret_cast<uint32_t *>(sm + OFF_GLO + sw128_offset(tk, col)) = l;
+        *reinterpret_cast<uint32_t *>(sm + OFF_GHI + sw128_offset(tk, col)) = pack_f16x2(g.x, g.y);
       };
       if (!LN) {
         // dl/dy = 2 (y - v)
@@ -472,20 +464,22 @@ __global__ void __launch_bounds__(THREADS, 4)
           store_grad(8 * j + 2 * q4, __fmul2_rn(f, __fadd2_rn(__ffma2_rn(xh, __fadd2_rn(w2[j], nB), u[j]), nA)));
         }
       }
+      // This thread's K row elements become fp16 in place (the dW operand); P and
+      // S, the bf16 readers, are complete.
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float2 k2 = unpack_bf16x2(kr[j]);
+        *reinterpret_cast<uint32_t *>(sm + kq_offset(tk, 0, 8 * j + 2 * q4)) = pack_f16x2(k2.x, k2.y);
+      }
       // Both halves of eta*G_m written: the pair's first warp issues the update.
       fence_proxy_async_smem();
       tc_fence_before_sync();
       named_barrier_sync(1 + (warp & 1), 64);
       if (hh == 0) {
         __syncwarp();
-        const bool issue = elect_one_sync();
         tc_fence_after_sync();
-        const uint64_t bhi = smem_desc_sw128(aGhi + 2048 * m, 8192, 1024);
-        const uint64_t blo = smem_desc_sw128(aGlo + 2048 * m, 8192, 1024);
-        if (issue) umma_ts(tP, tS + 8 * m, bhi, ID_UPD, true);       // A hi x G hi
-        if (issue) umma_ts(tP, tS + 8 * m, blo, ID_UPD, true);       // A hi x G lo
-        if (issue) umma_ts(tP, tS + 32 + 8 * m, bhi, ID_UPD, true);  // A lo x G hi
-        if (issue) umma_commit(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
+        umma_ts_w(tP, tS + 8 * m, smem_desc_sw128(aGhi + 2048 * m, 8192, 1024), ID_UPD, true);
+        umma_commit_w(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
         __syncwarp();
       }
     }
@@ -549,7 +543,6 @@ __global__ void __launch_bounds__(THREADS, 4)
     tc_fence_after_sync();
     if (warp == 0) {
       __syncwarp();
-      const bool issue = elect_one_sync();
       // dW = K^T (eta G) into the S columns (their operand is consumed).  Step k
       // takes the K rows of groups 4k and 4k + 2 (tokens of mini-batches
       // 2(k % 2), 2(k % 2) + 1, half k / 2), read twice (lbo 0) so that rows
@@ -559,16 +552,15 @@ __global__ void __launch_bounds__(THREADS, 4)
       for (int k = 0; k < 4; ++k) {
         const uint64_t ak = smem_desc_sw128(aA + 4096 * k, 0, 2048);
         const uint32_t gk = 4096u * (k & 1) + 1024u * (k >> 1);
-        if (issue) umma_ss(tS, ak, smem_desc_sw128(aGhi + gk, 8192, 2048), ID_DW, k > 0);
-        if (issue) umma_ss(tS, ak, smem_desc_sw128(aGlo + gk, 8192, 2048), ID_DW, true);
+        umma_ss_w(tS, ak, smem_desc_sw128(aGhi + gk, 8192, 2048), ID_DW, k > 0);
       }
-      if (issue) umma_commit(&bars[BAR_DW]);
+      umma_commit_w(&bars[BAR_DW]);
       __syncwarp();
     }
     wait_or_abort(&bars[BAR_DW], par, abort);
     tc_fence_after_sync();
     __syncwarp();
-    // K, V (lo half of eta*G) and eta are free once dW is done; every thread passed
+    // K, V and eta are free once dW is done; every thread passed
     // this chunk's wait on their barrier in the chunk head.
     if (tid == 0 && c + 1 < nchunks && !*abort) issue_loads_kv(c + 1);
     {

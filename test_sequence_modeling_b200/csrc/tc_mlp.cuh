@@ -182,8 +182,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     mlp_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const Params p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, as an offset into the shared array so that every
+  // access through it stays a shared-memory access.
+  uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3;           // TMEM lane quarter of this warp
   const int half = (warp >> 2) & 1;  // hidden half of this thread

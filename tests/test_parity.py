@@ -48,11 +48,12 @@ def test_reduced_config_every_unit(name, path):
 
 
 # Regression bounds of the default path at full size, a few times the error each
-# path measures (printed by the test): the exact-fp32 path for fp32 inputs, bf16
-# hi + lo operands for TTT-Linear, tf32 operands for TTT-MLP.  A precision change
-# shows here long before it reaches the oracle tolerance.
-REGRESSION = {"linear_f32_B1H1T256": 1e-6, "linear_bf16_B16H12T2048": 3e-5,
-              "linear_ln_B16H32T8192": 3e-5, "linear_ln_B1H32T32768": 3e-5,
+# path measures (printed by the test): the exact-fp32 path for fp32 inputs; for
+# TTT-Linear, W as bf16 hi + lo and fp16 chain and update operands (measured
+# 2.2e-4 plain, 7.4e-5 with LN); tf32 and fp16 operands for TTT-MLP.  A
+# precision change shows here long before it reaches the oracle tolerance.
+REGRESSION = {"linear_f32_B1H1T256": 1e-6, "linear_bf16_B16H12T2048": 1e-3,
+              "linear_ln_B16H32T8192": 3e-4, "linear_ln_B1H32T32768": 3e-4,
               "mlp_B8H32T8192": 1.5e-3}
 
 
@@ -148,10 +149,10 @@ def test_tensor_core_ragged_chunks(variant, T):
     assert max(worst.values()) <= TOL[cfg.dtype], (variant, T, worst)
 
 
-# Agreement of the tensor-core path with the exact-fp32 CUDA-core path: bf16
-# hi + lo operands (~2^-16) for TTT-Linear, tf32 operands (10-bit mantissa) for
-# TTT-MLP, both far below the oracle tolerance.
-AGREE = {"linear_bf16_B16H12T2048": 2e-4, "linear_ln_B16H32T8192": 2e-4, "mlp_B8H32T8192": 1e-3}
+# Agreement of the tensor-core path with the exact-fp32 CUDA-core path: fp16
+# chain and update operands (11-bit significand) for TTT-Linear, tf32 and fp16
+# operands for TTT-MLP, both far below the oracle tolerance.
+AGREE = {"linear_bf16_B16H12T2048": 1e-3, "linear_ln_B16H32T8192": 5e-4, "mlp_B8H32T8192": 1e-3}
 
 
 @pytest.mark.parametrize("name", list(AGREE))
