@@ -818,9 +818,9 @@ def run_decode(args, mlp=False, momentum=False):
 
 
 def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, torch, dist):
-    """Through the public host-memory API (test_sequence_modeling_b200.host): pinned
-    host inputs in, host outputs back, every step; the copies of one batch chunk
-    overlap the forward of the next."""
+    """Through the C ABI's host-memory forward (ttt_fwd_host, via
+    test_sequence_modeling_b200.host): pinned host inputs in, host outputs back,
+    every step; the copies of one batch chunk overlap the forward of the next."""
     from test_sequence_modeling_b200.host import HostForward
     pin = {k: v.pin_memory() for k, v in host.items()}
     h_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
@@ -857,7 +857,8 @@ def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, 
     e2e_value = world * cfg.head_tokens * args.e2e_steps / (te / 1e3)
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
-            "api": "test_sequence_modeling_b200.host.HostForward (4 batch chunks, copies overlapped)"}
+            "api": "ttt_fwd_host (C ABI, host buffers; 4 batch chunks, copies overlapped) through "
+                   "test_sequence_modeling_b200.host.HostForward"}
 
 
 def finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info, launches, e2e,

@@ -63,6 +63,8 @@
 #define TTT_API
 #endif
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -116,6 +118,51 @@ TTT_API int ttt_mlp_fwd(const void *Q, const void *K, const void *V, int qkv_dty
                 const float *W1_0, const float *W2_0, const float *ln_gamma, const float *ln_beta,
                 float ln_eps, int B, int H, int T, int d, int hidden, int b, float *Z,
                 float *W1_out, float *W2_out, void *stream);
+
+/*
+ * The three forwards above with Q, K, V, eta, the per-head inputs and the outputs
+ * in HOST memory (§03.7 dual form, §03.9 variants: the same operation and results
+ * as ttt_linear_fwd / ttt_linear_ln_fwd / ttt_mlp_fwd, which it calls).
+ *
+ * variant: TTT_VARIANT_LINEAR (W0 = the state; W2_0, gamma, beta, ln_eps and
+ * hidden ignored), TTT_VARIANT_LINEAR_LN (W0, gamma, beta, ln_eps), or
+ * TTT_VARIANT_MLP (W0 = W1_0 [H][d][hidden], W2_0, gamma, beta, ln_eps, hidden;
+ * W2_out receives the final W2).  Layouts and sizes as for the device entry
+ * points; every host pointer 16-byte aligned.
+ *
+ * workspace: DEVICE memory owned by the caller, at least
+ * ttt_fwd_host_workspace_bytes(variant, qkv_dtype, B, H, T, d, hidden) bytes,
+ * 256-byte aligned; it receives the device copies of every input and output.
+ * The batch is split into `chunks` (>= 1; at most B are used) contiguous slices:
+ * the copy of slice i + 1 to the device, the forward of slice i and the copy of
+ * slice i - 1 back run on three streams and overlap.  Host buffers should be
+ * page-locked (cudaHostAlloc, or torch's pin_memory) for the copies to be
+ * asynchronous; pageable memory works but serialises them.
+ *
+ * Ordering and ownership: the call returns once everything is enqueued.  All of
+ * its work starts after the work already on `stream`, and `stream` waits for its
+ * last copy back, so synchronising `stream` (or an event recorded on it after the
+ * call) makes Z, W_out and W2_out valid in host memory.  Until then the caller
+ * must neither change the host inputs nor read the host outputs nor reuse the
+ * workspace.  Calls ordered on one stream may share a workspace.
+ *
+ * Errors: the argument rules of the device entry points (on the host pointers),
+ * plus TTT_ERR_ARG for an unknown variant, chunks < 1 or a workspace that is null
+ * or too small, TTT_ERR_ALIGN for a workspace not 256-byte aligned; TTT_ERR_CUDA
+ * if a copy, stream or event call fails.  On an error after the first copy was
+ * enqueued the outputs are unspecified.
+ */
+typedef enum { TTT_VARIANT_LINEAR = 0, TTT_VARIANT_LINEAR_LN = 1, TTT_VARIANT_MLP = 2 } ttt_variant;
+
+/* Bytes of device workspace ttt_fwd_host needs (0 for invalid arguments). */
+TTT_API size_t ttt_fwd_host_workspace_bytes(int variant, int qkv_dtype, int B, int H, int T, int d,
+                                            int hidden);
+
+TTT_API int ttt_fwd_host(int variant, const void *Q, const void *K, const void *V, int qkv_dtype,
+                         const float *eta, const float *W0, const float *W2_0, const float *ln_gamma,
+                         const float *ln_beta, float ln_eps, int B, int H, int T, int d, int hidden,
+                         int b, float *Z, float *W_out, float *W2_out, void *workspace,
+                         size_t workspace_bytes, int chunks, void *stream);
 
 /*
  * Forward of TTT-Linear (and, _ln_, TTT-Linear with LN and residual) over whole

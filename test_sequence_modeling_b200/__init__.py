@@ -19,7 +19,7 @@ def __getattr__(name):
                 "ttt_linear_momentum_decode", "ttt_linear_ln_momentum_decode",
                 "ttt_mlp_momentum_decode", "ttt_linear_bwd", "ttt_linear_momentum_fwd",
                 "ttt_linear_ln_bwd_noalloc", "ttt_mlp_bwd",
-                "ttt_mlp_momentum_fwd"):
+                "ttt_mlp_momentum_fwd", "ttt_fwd_host", "fwd_host_workspace_bytes"):
         from . import ttt
         return getattr(ttt, name)
     raise AttributeError(name)

@@ -11,6 +11,7 @@ TTT_OK, TTT_ERR_ARG, TTT_ERR_ALIGN, TTT_ERR_UNSUPPORTED, TTT_ERR_CUDA, TTT_ERR_T
     0, -1, -2, -3, -4, -5)
 TTT_F32, TTT_BF16 = 0, 1
 TTT_PATH_AUTO, TTT_PATH_SIMT, TTT_PATH_TC = 0, 1, 2
+TTT_VARIANT_LINEAR, TTT_VARIANT_LINEAR_LN, TTT_VARIANT_MLP = 0, 1, 2
 # Capacity of ttt_linear_ln_bwd_noalloc's built-in state array (d x d fp32 states).
 TTT_NOALLOC_BWD_MAX_STATES = 4096
 
@@ -52,6 +53,9 @@ SIGNATURES = {
                                      _fp, _fp, _f, _i, _i, _i, _i, _i, _i, _fp, _vp]),
     "ttt_mlp_decode": (_i, [_vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i, _i,
                             _i, _i, _fp, _vp]),
+    "ttt_fwd_host_workspace_bytes": (ctypes.c_size_t, [_i, _i, _i, _i, _i, _i, _i]),
+    "ttt_fwd_host": (_i, [_i, _vp, _vp, _vp, _i, _fp, _fp, _fp, _fp, _fp, _f, _i, _i, _i, _i, _i, _i,
+                          _fp, _fp, _fp, _vp, ctypes.c_size_t, _i, _vp]),
 }
 
 _lib = None

@@ -6,7 +6,9 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <mutex>
+#include <vector>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -645,9 +647,206 @@ int run(const Call &c) {
   return run_simt(c);
 }
 
+// ---- the forward with inputs and outputs in host memory -----------------------------
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Byte offsets of the device copies in the caller's workspace (each 256-byte aligned).
+struct HostLayout {
+  size_t q, k, v, eta, z, w, w2, p0, p1, p2, p3, total;
+};
+
+HostLayout host_layout(Kind kind, int qkv_dtype, long long B, long long H, long long T, long long d,
+                       long long hidden) {
+  const size_t in_elt = qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t units = (size_t)(B * H), elems = units * (size_t)(T * d);
+  const size_t P1 = (size_t)(kind == MLP_LN ? d * hidden : d * d);
+  HostLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  L.q = take(elems * in_elt);
+  L.k = take(elems * in_elt);
+  L.v = take(elems * in_elt);
+  L.eta = take(units * (size_t)T * 4);
+  L.z = take(elems * 4);
+  L.w = take(units * P1 * 4);
+  L.w2 = take(kind == MLP_LN ? units * P1 * 4 : 0);
+  L.p0 = take((size_t)H * P1 * 4);
+  L.p1 = take(kind == MLP_LN ? (size_t)H * P1 * 4 : 0);
+  L.p2 = take(kind != LINEAR ? (size_t)(H * d) * 4 : 0);
+  L.p3 = take(kind != LINEAR ? (size_t)(H * d) * 4 : 0);
+  L.total = off;
+  return L;
+}
+
+// Streams and events of one host-memory call, released on every return path (a
+// stream or event with work still pending is released once that work is done).
+struct HostCallResources {
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  std::vector<cudaEvent_t> events;
+  ~HostCallResources() {
+    for (cudaEvent_t e : events) cudaEventDestroy(e);
+    if (s_in) cudaStreamDestroy(s_in);
+    if (s_out) cudaStreamDestroy(s_out);
+  }
+  cudaEvent_t event() {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    events.push_back(e);
+    return e;
+  }
+};
+
+// The batch is split into `chunks` contiguous slices; slice i is copied in on s_in,
+// computed on the caller's stream and copied out on s_out, so that the copy in of
+// slice i + 1, the forward of slice i and the copy out of slice i - 1 overlap.
+// Every step is ordered after the work already on the caller's stream, and the
+// caller's stream waits for the last copy out.
+int run_host(const Call &h, void *workspace, size_t workspace_bytes, int chunks) {
+  const int st = validate(h);
+  if (st != TTT_OK) return st;
+  if (chunks < 1) return TTT_ERR_ARG;
+  const long long units = (long long)h.B * h.H;
+  if (units == 0) return TTT_OK;
+  const HostLayout L = host_layout(h.kind, h.qkv_dtype, h.B, h.H, h.T, h.d, h.hidden);
+  if (!workspace || workspace_bytes < L.total) return TTT_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return TTT_ERR_ALIGN;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  cudaStream_t s_run = static_cast<cudaStream_t>(h.stream);
+
+  HostCallResources r;
+  if (cudaStreamCreateWithFlags(&r.s_in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&r.s_out, cudaStreamNonBlocking) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  cudaEvent_t fork = r.event();
+  if (!fork || cudaEventRecord(fork, s_run) != cudaSuccess || cudaStreamWaitEvent(r.s_in, fork, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(r.s_out, fork, 0) != cudaSuccess)
+    return TTT_ERR_CUDA;
+
+  auto h2d = [&](size_t off, const void *src, size_t bytes) {
+    return bytes == 0 || cudaMemcpyAsync(ws + off, src, bytes, cudaMemcpyHostToDevice, r.s_in) == cudaSuccess;
+  };
+  auto d2h = [&](void *dst, size_t off, size_t bytes) {
+    return bytes == 0 || cudaMemcpyAsync(dst, ws + off, bytes, cudaMemcpyDeviceToHost, r.s_out) == cudaSuccess;
+  };
+
+  const size_t in_elt = h.qkv_dtype == TTT_BF16 ? 2 : 4;
+  const size_t P1 = (size_t)(h.kind == MLP_LN ? (size_t)h.d * h.hidden : (size_t)h.d * h.d);
+  const size_t tok_per_b = (size_t)h.H * h.T, elem_per_b = tok_per_b * h.d, state_per_b = (size_t)h.H * P1;
+  // Per-head inputs first.
+  if (!h2d(L.p0, h.W0, (size_t)h.H * P1 * 4)) return TTT_ERR_CUDA;
+  if (h.kind == MLP_LN && !h2d(L.p1, h.W2_0, (size_t)h.H * P1 * 4)) return TTT_ERR_CUDA;
+  if (h.kind != LINEAR && (!h2d(L.p2, h.gamma, (size_t)h.H * h.d * 4) || !h2d(L.p3, h.beta, (size_t)h.H * h.d * 4)))
+    return TTT_ERR_CUDA;
+
+  const int n = (int)std::min<long long>(chunks, h.B);
+  for (int i = 0; i < n; ++i) {
+    const size_t b0 = (size_t)((long long)h.B * i / n), b1 = (size_t)((long long)h.B * (i + 1) / n);
+    const size_t nb = b1 - b0;
+    if (nb == 0) continue;
+    const size_t qo = b0 * elem_per_b * in_elt, qn = nb * elem_per_b * in_elt;
+    const size_t eo = b0 * tok_per_b * 4, en = nb * tok_per_b * 4;
+    const size_t zo = b0 * elem_per_b * 4, zn = nb * elem_per_b * 4;
+    const size_t wo = b0 * state_per_b * 4, wn = nb * state_per_b * 4;
+    if (h.T > 0) {
+      const uint8_t *q = static_cast<const uint8_t *>(h.Q), *k = static_cast<const uint8_t *>(h.K),
+                    *v = static_cast<const uint8_t *>(h.V);
+      if (!h2d(L.q + qo, q + qo, qn) || !h2d(L.k + qo, k + qo, qn) || !h2d(L.v + qo, v + qo, qn) ||
+          !h2d(L.eta + eo, reinterpret_cast<const uint8_t *>(h.eta) + eo, en))
+        return TTT_ERR_CUDA;
+    }
+    cudaEvent_t loaded = r.event(), computed = r.event();
+    if (!loaded || !computed || cudaEventRecord(loaded, r.s_in) != cudaSuccess ||
+        cudaStreamWaitEvent(s_run, loaded, 0) != cudaSuccess)
+      return TTT_ERR_CUDA;
+    Call c = h;
+    c.B = (int)nb;
+    c.Q = ws + L.q + qo;
+    c.K = ws + L.k + qo;
+    c.V = ws + L.v + qo;
+    c.eta = reinterpret_cast<const float *>(ws + L.eta + eo);
+    c.Z = reinterpret_cast<float *>(ws + L.z + zo);
+    c.W_out = reinterpret_cast<float *>(ws + L.w + wo);
+    c.W2_out = h.kind == MLP_LN ? reinterpret_cast<float *>(ws + L.w2 + wo) : nullptr;
+    c.W0 = reinterpret_cast<const float *>(ws + L.p0);
+    c.W2_0 = h.kind == MLP_LN ? reinterpret_cast<const float *>(ws + L.p1) : nullptr;
+    c.gamma = h.kind != LINEAR ? reinterpret_cast<const float *>(ws + L.p2) : nullptr;
+    c.beta = h.kind != LINEAR ? reinterpret_cast<const float *>(ws + L.p3) : nullptr;
+    c.stream = s_run;
+    if (h.T == 0) c.Q = c.K = c.V = nullptr, c.eta = nullptr, c.Z = nullptr;
+    const int rs = run(c);
+    if (rs != TTT_OK) return rs;
+    if (cudaEventRecord(computed, s_run) != cudaSuccess || cudaStreamWaitEvent(r.s_out, computed, 0) != cudaSuccess)
+      return TTT_ERR_CUDA;
+    if ((h.T > 0 && !d2h(reinterpret_cast<uint8_t *>(h.Z) + zo, L.z + zo, zn)) ||
+        !d2h(reinterpret_cast<uint8_t *>(h.W_out) + wo, L.w + wo, wn) ||
+        (h.kind == MLP_LN && !d2h(reinterpret_cast<uint8_t *>(h.W2_out) + wo, L.w2 + wo, wn)))
+      return TTT_ERR_CUDA;
+  }
+  cudaEvent_t joined = r.event();
+  if (!joined || cudaEventRecord(joined, r.s_out) != cudaSuccess || cudaStreamWaitEvent(s_run, joined, 0) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  return TTT_OK;
+}
+
+Kind host_kind(int variant, bool *ok) {
+  *ok = true;
+  switch (variant) {
+    case TTT_VARIANT_LINEAR: return LINEAR;
+    case TTT_VARIANT_LINEAR_LN: return LINEAR_LN;
+    case TTT_VARIANT_MLP: return MLP_LN;
+    default: *ok = false; return LINEAR;
+  }
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t ttt_fwd_host_workspace_bytes(int variant, int qkv_dtype, int B, int H, int T, int d, int hidden) {
+  bool ok = false;
+  const Kind kind = host_kind(variant, &ok);
+  if (!ok || (qkv_dtype != TTT_F32 && qkv_dtype != TTT_BF16) || B < 0 || H < 0 || T < 0 || d <= 0 ||
+      (kind == MLP_LN && hidden <= 0))
+    return 0;
+  return host_layout(kind, qkv_dtype, B, H, T, d, hidden).total;
+}
+
+int ttt_fwd_host(int variant, const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
+                 const float *W0, const float *W2_0, const float *ln_gamma, const float *ln_beta, float ln_eps,
+                 int B, int H, int T, int d, int hidden, int b, float *Z, float *W_out, float *W2_out,
+                 void *workspace, size_t workspace_bytes, int chunks, void *stream) {
+  bool ok = false;
+  const Kind kind = host_kind(variant, &ok);
+  if (!ok) return TTT_ERR_ARG;
+  Call c{kind,
+         Q,
+         K,
+         V,
+         qkv_dtype,
+         eta,
+         W0,
+         kind == MLP_LN ? W2_0 : nullptr,
+         kind != LINEAR ? ln_gamma : nullptr,
+         kind != LINEAR ? ln_beta : nullptr,
+         kind != LINEAR ? ln_eps : 0.f,
+         B,
+         H,
+         T,
+         d,
+         kind == MLP_LN ? hidden : 0,
+         b,
+         Z,
+         W_out,
+         kind == MLP_LN ? W2_out : nullptr,
+         stream};
+  return run_host(c, workspace, workspace_bytes, chunks);
+}
+
 
 int ttt_linear_fwd(const void *Q, const void *K, const void *V, int qkv_dtype, const float *eta,
                    const float *W0, int B, int H, int T, int d, int b, float *Z, float *W_out,

@@ -85,6 +85,76 @@ def ttt_linear_fwd(Q, K, V, eta, W0, b, Z=None, W_out=None, stream=None):
     return Z, W_out
 
 
+VARIANTS = {"linear": _lib.TTT_VARIANT_LINEAR, "linear_ln": _lib.TTT_VARIANT_LINEAR_LN,
+            "mlp": _lib.TTT_VARIANT_MLP}
+
+
+def fwd_host_workspace_bytes(variant, shape, qkv_dtype, hidden=0) -> int:
+    """Device workspace bytes ttt_fwd_host needs for inputs of `shape` [B,H,T,d]."""
+    B, H, T, d = shape
+    dt = TTT_BF16 if qkv_dtype == torch.bfloat16 else TTT_F32
+    n = _lib.load().ttt_fwd_host_workspace_bytes(VARIANTS[variant], dt, B, H, T, d, int(hidden))
+    if n == 0:
+        raise TTTError(f"ttt_fwd_host_workspace_bytes: invalid arguments for {variant} {tuple(shape)}")
+    return int(n)
+
+
+def _host(t, name, dtype, shape):
+    """A contiguous host tensor of this dtype and shape (the C ABI reads plain pointers)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cpu" or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def ttt_fwd_host(variant, Q, K, V, eta, params, b, eps, Z, W_outs, workspace, chunks=4, stream=None):
+    """The forward with inputs and outputs in host memory (pinned for overlap).
+    params: (W0,) | (W0, gamma, beta) | (W1, W2, gamma, beta) per variant; Z and
+    W_outs ((W_out,) or (W1_out, W2_out)): host outputs written in place.  workspace:
+    a uint8 CUDA tensor of at least fwd_host_workspace_bytes.  Enqueues on `stream`
+    (default: the current stream of the workspace's device) and returns; the outputs
+    are valid once that stream has reached this point."""
+    if Q.dtype not in _QKV_DTYPES or Q.dim() != 4:
+        raise TypeError("Q must be a [B, H, T, d] float32 or bfloat16 tensor")
+    B, H, T, d = Q.shape
+    dt = _QKV_DTYPES[Q.dtype]
+    for n, t in (("Q", Q), ("K", K), ("V", V)):
+        _host(t, n, Q.dtype, (B, H, T, d))
+    _host(eta, "eta", torch.float32, (B, H, T))
+    _host(Z, "Z", torch.float32, (B, H, T, d))
+    if variant == "mlp":
+        hidden = params[0].shape[-1]
+        pshapes = [(H, d, hidden), (H, hidden, d), (H, d), (H, d)]
+        wshapes = [(B, H, d, hidden), (B, H, hidden, d)]
+    else:
+        hidden = 0
+        pshapes = [(H, d, d)] + ([(H, d), (H, d)] if variant == "linear_ln" else [])
+        wshapes = [(B, H, d, d)]
+    if len(params) != len(pshapes) or len(W_outs) != len(wshapes):
+        raise ValueError(f"ttt_fwd_host: {variant} takes {len(pshapes)} parameters and {len(wshapes)} states")
+    for i, (t, shp) in enumerate(zip(params, pshapes)):
+        _host(t, f"params[{i}]", torch.float32, shp)
+    for i, (t, shp) in enumerate(zip(W_outs, wshapes)):
+        _host(t, f"W_outs[{i}]", torch.float32, shp)
+    if not (isinstance(workspace, torch.Tensor) and workspace.is_cuda and workspace.dtype == torch.uint8):
+        raise TypeError("ttt_fwd_host: workspace must be a uint8 CUDA tensor")
+    W0 = params[0]
+    W2_0 = params[1] if variant == "mlp" else None
+    gamma, beta = (params[-2], params[-1]) if variant != "linear" else (None, None)
+    W2_out = W_outs[1] if variant == "mlp" else None
+    with torch.cuda.device(workspace.device):
+        st = _lib.load().ttt_fwd_host(VARIANTS[variant], _ptr(Q), _ptr(K), _ptr(V), dt, _ptr(eta), _ptr(W0),
+                                      _ptr(W2_0), _ptr(gamma), _ptr(beta), float(eps), B, H, T, d, int(hidden),
+                                      int(b), _ptr(Z), _ptr(W_outs[0]), _ptr(W2_out), _ptr(workspace),
+                                      workspace.numel(), int(chunks), _stream(stream, workspace.device))
+    check(st, "ttt_fwd_host")
+
+
 def ttt_linear_ln_fwd(Q, K, V, eta, W0, gamma, beta, b, eps=1e-6, Z=None, W_out=None, stream=None):
     """TTT-Linear with LN + residual.  gamma, beta [H,d] f32."""
     dt = _qkv(Q, K, V)

@@ -325,3 +325,46 @@ def test_noalloc_backward_checks_sizes_before_any_cuda_call(lib):
     assert call(2, 3, 48, d=32) == L.TTT_ERR_UNSUPPORTED
     assert call(2, 3, 64, b=32) == L.TTT_ERR_UNSUPPORTED
     assert call(0, 3, 48) == L.TTT_OK                       # no units: nothing to do
+
+
+def test_host_forward_workspace_size_and_argument_checks(lib):
+    """ttt_fwd_host: the workspace query on the host, and every argument error
+    (variant, chunks, workspace size and alignment, the forward's own rules)
+    rejected before any copy or launch (fake pointers are never touched)."""
+    ws_bytes = lib.ttt_fwd_host_workspace_bytes
+    B, H, T, d = 2, 3, 64, 64
+    n_ln = ws_bytes(L.TTT_VARIANT_LINEAR_LN, L.TTT_BF16, B, H, T, d, 0)
+    # Q, K, V bf16, eta, Z, W_out, W0, gamma, beta, each rounded up to 256 bytes.
+    up = lambda x: (x + 255) // 256 * 256
+    elems = B * H * T * d
+    expect = 3 * up(elems * 2) + up(B * H * T * 4) + up(elems * 4) + up(B * H * d * d * 4) + \
+        up(H * d * d * 4) + 2 * up(H * d * 4)
+    assert n_ln == expect
+    assert ws_bytes(L.TTT_VARIANT_LINEAR, L.TTT_F32, B, H, T, d, 0) == \
+        3 * up(elems * 4) + up(B * H * T * 4) + up(elems * 4) + up(B * H * d * d * 4) + up(H * d * d * 4)
+    n_mlp = ws_bytes(L.TTT_VARIANT_MLP, L.TTT_BF16, B, H, T, d, 256)
+    assert n_mlp == 3 * up(elems * 2) + up(B * H * T * 4) + up(elems * 4) + 2 * up(B * H * d * 256 * 4) + \
+        2 * up(H * d * 256 * 4) + 2 * up(H * d * 4)
+    assert ws_bytes(7, L.TTT_BF16, B, H, T, d, 0) == 0
+    assert ws_bytes(L.TTT_VARIANT_LINEAR, 5, B, H, T, d, 0) == 0
+    assert ws_bytes(L.TTT_VARIANT_MLP, L.TTT_BF16, B, H, T, d, 0) == 0
+    assert ws_bytes(L.TTT_VARIANT_LINEAR, L.TTT_BF16, -1, H, T, d, 0) == 0
+
+    p = _ptrs(12)
+    ws = p[11] + (1 << 30)  # 256-byte aligned fake device address
+
+    def call(variant=L.TTT_VARIANT_LINEAR_LN, B=B, T=T, b=16, chunks=4, wsp=ws, wsn=n_ln, eps=1e-6, g=p[6]):
+        return lib.ttt_fwd_host(variant, p[0], p[1], p[2], L.TTT_BF16, p[3], p[4], None, g, p[7], eps,
+                                B, H, T, d, 0, b, p[8], p[9], None, wsp, wsn, chunks, None)
+
+    n0 = lib.ttt_launch_count()
+    assert call(variant=9) == L.TTT_ERR_ARG
+    assert call(chunks=0) == L.TTT_ERR_ARG
+    assert call(wsp=None) == L.TTT_ERR_ARG
+    assert call(wsn=n_ln - 1) == L.TTT_ERR_ARG
+    assert call(wsp=ws + 16) == L.TTT_ERR_ALIGN
+    assert call(T=40) == L.TTT_ERR_ARG                       # T % b != 0
+    assert call(eps=0.0) == L.TTT_ERR_ARG
+    assert call(g=None) == L.TTT_ERR_ARG                     # LN without gamma
+    assert call(B=0) == L.TTT_OK                             # no units: nothing to do
+    assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"

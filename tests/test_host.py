@@ -1,5 +1,6 @@
-"""GPU: the host-memory forward (copies of batch chunks overlapped with the
-forwards on three streams) gives exactly the device-resident forward's outputs."""
+"""GPU: the host-memory forward (ttt_fwd_host through the C ABI: copies of batch
+chunks overlapped with the forwards on three streams) gives exactly the
+device-resident forward's outputs."""
 import numpy as np
 import pytest
 import torch
@@ -62,3 +63,35 @@ def test_back_to_back_calls_do_not_overlap():
     for (Z, W), (_, ref) in zip(outs, runs):
         assert np.array_equal(Z.numpy(), ref["Z"])
         assert np.array_equal(W.numpy(), ref["W"])
+
+
+def test_host_forward_edges():
+    """T = 0 (states pass through), more chunks than batch rows, pageable host
+    memory, and a workspace one byte short (rejected before anything runs)."""
+    from test_sequence_modeling_b200 import ttt
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=2, H=3, T=64)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    ref = run_gpu(cfg, dev)
+    host = {k: v.cpu() for k, v in dev.items()}          # pageable
+    params = [host["W0"], host["gamma"], host["beta"]]
+    n = ttt.fwd_host_workspace_bytes("linear_ln", tuple(host["Q"].shape), host["Q"].dtype)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    Z = torch.empty(cfg.B, cfg.H, cfg.T, cfg.d)
+    W = torch.empty(cfg.B, cfg.H, cfg.d, cfg.d)
+    ttt.ttt_fwd_host("linear_ln", host["Q"], host["K"], host["V"], host["eta"], params, cfg.b, cfg.ln_eps,
+                     Z, [W], ws, chunks=7)
+    torch.cuda.synchronize()
+    assert np.array_equal(Z.numpy(), ref["Z"]) and np.array_equal(W.numpy(), ref["W"])
+    with pytest.raises(ttt.TTTError):
+        ttt.ttt_fwd_host("linear_ln", host["Q"], host["K"], host["V"], host["eta"], params, cfg.b,
+                         cfg.ln_eps, Z, [W], ws[: n - 1], chunks=2)
+    # T = 0: no tokens; the final state is the initial one for every unit.
+    e = {k: torch.empty(cfg.B, cfg.H, 0, cfg.d, dtype=host[k].dtype) for k in ("Q", "K", "V")}
+    eta0 = torch.empty(cfg.B, cfg.H, 0)
+    Z0 = torch.empty(cfg.B, cfg.H, 0, cfg.d)
+    W0 = torch.zeros(cfg.B, cfg.H, cfg.d, cfg.d)
+    ws0 = torch.empty(ttt.fwd_host_workspace_bytes("linear_ln", (cfg.B, cfg.H, 0, cfg.d), host["Q"].dtype),
+                      dtype=torch.uint8, device="cuda")
+    ttt.ttt_fwd_host("linear_ln", e["Q"], e["K"], e["V"], eta0, params, cfg.b, cfg.ln_eps, Z0, [W0], ws0)
+    torch.cuda.synchronize()
+    assert np.array_equal(W0.numpy(), np.broadcast_to(host["W0"].numpy(), W0.shape))
