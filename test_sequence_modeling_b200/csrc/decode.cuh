@@ -232,20 +232,33 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_decode_kernel(const MlpParams
   float *S2 = MOMENTUM ? p.S2 + unit * HID * D : nullptr;
   // W1 -= eta k^T G2 (column i; or the momentum and decay update) and Z1 = q W1
   // with the updated W1.
+  // Rows in blocks of RB: every load of a block is issued before its stores, which
+  // the compiler could not otherwise move past (W1, W1b and S1 are distinct
+  // buffers, but nothing tells it so), keeping 2 RB loads per thread in flight.
+  constexpr int RB = 16;
   float z1 = 0.f;
-#pragma unroll 8
-  for (int pp = 0; pp < D; ++pp) {
-    float w;
-    if (MOMENTUM) {
-      const float sm = fmaf(al, S1[pp * HID + i], -ks[pp] * g2);
-      S1[pp * HID + i] = sm;
-      w = fmaf(keep, W1[pp * HID + i], sm);
-    } else {
-      w = fmaf(-ks[pp], g2, W1[pp * HID + i]);
+  for (int p0 = 0; p0 < D; p0 += RB) {
+    float wv[RB], sv[MOMENTUM ? RB : 1];
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      wv[u] = W1[(p0 + u) * HID + i];
+      if (MOMENTUM) sv[u] = S1[(p0 + u) * HID + i];
     }
-    W1[pp * HID + i] = w;
-    if (last) W1b[pp * HID + i] = w;
-    z1 = fmaf(qs[pp], w, z1);
+#pragma unroll
+    for (int u = 0; u < RB; ++u) {
+      const int pp = p0 + u;
+      float w;
+      if (MOMENTUM) {
+        const float sm = fmaf(al, sv[u], -ks[pp] * g2);
+        S1[pp * HID + i] = sm;
+        w = fmaf(keep, wv[u], sm);
+      } else {
+        w = fmaf(-ks[pp], g2, wv[u]);
+      }
+      W1[pp * HID + i] = w;
+      if (last) W1b[pp * HID + i] = w;
+      z1 = fmaf(qs[pp], w, z1);
+    }
   }
   z2s[i] = simt::gelu(z1);
   __syncthreads();
@@ -253,29 +266,43 @@ __global__ void __launch_bounds__(MLP_THREADS) mlp_decode_kernel(const MlpParams
   {
     const float eg0 = e * g3[lane], eg1 = e * g3[lane + 32];
     float a0 = 0.f, a1 = 0.f;
-#pragma unroll 8
-    for (int r = 0; r < 32; ++r) {
-      const int ii = 32 * warp + r;
-      float w0, w1;
-      if (MOMENTUM) {
-        const float s0 = fmaf(al, S2[ii * D + lane], -x2s[ii] * eg0);
-        const float s1 = fmaf(al, S2[ii * D + lane + 32], -x2s[ii] * eg1);
-        S2[ii * D + lane] = s0;
-        S2[ii * D + lane + 32] = s1;
-        w0 = fmaf(keep, W2[ii * D + lane], s0);
-        w1 = fmaf(keep, W2[ii * D + lane + 32], s1);
-      } else {
-        w0 = fmaf(-x2s[ii], eg0, W2[ii * D + lane]);
-        w1 = fmaf(-x2s[ii], eg1, W2[ii * D + lane + 32]);
+    constexpr int R2 = 8;  // rows per block, loads first (as for W1 above)
+    for (int r0 = 0; r0 < 32; r0 += R2) {
+      float wv0[R2], wv1[R2], sv0[MOMENTUM ? R2 : 1], sv1[MOMENTUM ? R2 : 1];
+#pragma unroll
+      for (int u = 0; u < R2; ++u) {
+        const int ii = 32 * warp + r0 + u;
+        wv0[u] = W2[ii * D + lane];
+        wv1[u] = W2[ii * D + lane + 32];
+        if (MOMENTUM) {
+          sv0[u] = S2[ii * D + lane];
+          sv1[u] = S2[ii * D + lane + 32];
+        }
       }
-      W2[ii * D + lane] = w0;
-      W2[ii * D + lane + 32] = w1;
-      if (last) {
-        W2b[ii * D + lane] = w0;
-        W2b[ii * D + lane + 32] = w1;
+#pragma unroll
+      for (int u = 0; u < R2; ++u) {
+        const int ii = 32 * warp + r0 + u;
+        float w0, w1;
+        if (MOMENTUM) {
+          const float s0 = fmaf(al, sv0[u], -x2s[ii] * eg0);
+          const float s1 = fmaf(al, sv1[u], -x2s[ii] * eg1);
+          S2[ii * D + lane] = s0;
+          S2[ii * D + lane + 32] = s1;
+          w0 = fmaf(keep, wv0[u], s0);
+          w1 = fmaf(keep, wv1[u], s1);
+        } else {
+          w0 = fmaf(-x2s[ii], eg0, wv0[u]);
+          w1 = fmaf(-x2s[ii], eg1, wv1[u]);
+        }
+        W2[ii * D + lane] = w0;
+        W2[ii * D + lane + 32] = w1;
+        if (last) {
+          W2b[ii * D + lane] = w0;
+          W2b[ii * D + lane + 32] = w1;
+        }
+        a0 = fmaf(z2s[ii], w0, a0);
+        a1 = fmaf(z2s[ii], w1, a1);
       }
-      a0 = fmaf(z2s[ii], w0, a0);
-      a1 = fmaf(z2s[ii], w1, a1);
     }
     __syncthreads();  // every warp has read part[] of the X3 pass long before; reuse it
     part[warp][lane] = a0;
