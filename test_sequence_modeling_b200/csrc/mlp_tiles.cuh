@@ -43,7 +43,7 @@ __device__ void mm_W(float *out, int ldo, const float *A, int lda, const float *
   float a[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) a[r] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
   for (int k = 0; k < Kd; ++k) {
     const float w = W[(size_t)k * N + j];
 #pragma unroll
@@ -66,7 +66,7 @@ __device__ void mm_WT(float *out, int ldo, const float *A, int lda, const float 
 #pragma unroll
   for (int r = 0; r < RPT; ++r) a[r] = 0.f;
   const float4 *wr = reinterpret_cast<const float4 *>(W + (size_t)j * Kd);
-#pragma unroll 2
+#pragma unroll 4
   for (int k = 0; k < Kd; k += 4) {
     const float4 w = wr[k >> 2];
 #pragma unroll
@@ -100,23 +100,35 @@ __device__ void small_corr(float *out, int ldo, const float *S, bool trans, cons
   }
 }
 
+// Rows per block of the element-wise state passes: every load of a block is
+// issued before its stores, which the compiler cannot otherwise move a load past
+// (the destination may be the source, or another buffer it cannot tell apart).
+constexpr int ROW_BLOCK = 8;
+
 // dst[r][c] = src[r][c] + sign sum_{t<b} L[t][r] Rt[t][c]   (dst, src global [R][C];
 // dst may be src: each thread reads and writes only its own entries).
 template <int R, int C>
 __device__ void outer(float *dst, const float *src, const float *L, int ldl, const float *Rt, int ldr,
                       int b, float sign, int tid) {
   constexpr int GROUPS = THREADS / C, RPG = R / GROUPS;
+  static_assert(RPG % ROW_BLOCK == 0, "rows per thread group must fill whole blocks");
   const int c = tid % C, g = tid / C;
   float rt[MAXB];
 #pragma unroll
   for (int t = 0; t < MAXB; ++t) rt[t] = t < b ? Rt[t * ldr + c] : 0.f;
-  for (int i = 0; i < RPG; ++i) {
-    const int r = g * RPG + i;
-    float a = 0.f;
+  for (int i0 = 0; i0 < RPG; i0 += ROW_BLOCK) {
+    float sv[ROW_BLOCK];
 #pragma unroll
-    for (int t = 0; t < MAXB; ++t)
-      if (t < b) a = fmaf(L[t * ldl + r], rt[t], a);
-    dst[(size_t)r * C + c] = src[(size_t)r * C + c] + sign * a;
+    for (int u = 0; u < ROW_BLOCK; ++u) sv[u] = src[(size_t)(g * RPG + i0 + u) * C + c];
+#pragma unroll
+    for (int u = 0; u < ROW_BLOCK; ++u) {
+      const int r = g * RPG + i0 + u;
+      float a = 0.f;
+#pragma unroll
+      for (int t = 0; t < MAXB; ++t)
+        if (t < b) a = fmaf(L[t * ldl + r], rt[t], a);
+      dst[(size_t)r * C + c] = sv[u] + sign * a;
+    }
   }
 }
 

@@ -74,7 +74,7 @@ __device__ void mm_two(float *out, int ldo, const float *A, int lda, const float
   float a[RPT], c[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) a[r] = c[r] = 0.f;
-#pragma unroll 4
+#pragma unroll 8
   for (int k = 0; k < Kd; ++k) {
     const float w = W[(size_t)k * N + j], sv = S[(size_t)k * N + j];
 #pragma unroll
@@ -107,20 +107,30 @@ __device__ void update_state(float *W, float *S, const float *L, int ldl, const 
     rw[t] = v * wW[t];
     rs[t] = v * wS[t];
   }
-  for (int i = 0; i < RPG; ++i) {
-    const int r = g * RPG + i;
-    float gw = 0.f, gs = 0.f;
+  static_assert(RPG % ROW_BLOCK == 0, "rows per thread group must fill whole blocks");
+  for (int i0 = 0; i0 < RPG; i0 += ROW_BLOCK) {
+    float wv[ROW_BLOCK], sv[ROW_BLOCK];
 #pragma unroll
-    for (int t = 0; t < MAXB; ++t)
-      if (t < b) {
-        const float l = L[t * ldl + r];
-        gw = fmaf(l, rw[t], gw);
-        gs = fmaf(l, rs[t], gs);
-      }
-    const size_t e = (size_t)r * C + c;
-    const float w = W[e], sv = S[e];
-    W[e] = lam * w + cc * sv - gw;
-    S[e] = aa * sv - gs;
+    for (int u = 0; u < ROW_BLOCK; ++u) {
+      const size_t e = (size_t)(g * RPG + i0 + u) * C + c;
+      wv[u] = W[e];
+      sv[u] = S[e];
+    }
+#pragma unroll
+    for (int u = 0; u < ROW_BLOCK; ++u) {
+      const int r = g * RPG + i0 + u;
+      float gw = 0.f, gs = 0.f;
+#pragma unroll
+      for (int t = 0; t < MAXB; ++t)
+        if (t < b) {
+          const float l = L[t * ldl + r];
+          gw = fmaf(l, rw[t], gw);
+          gs = fmaf(l, rs[t], gs);
+        }
+      const size_t e = (size_t)r * C + c;
+      W[e] = lam * wv[u] + cc * sv[u] - gw;
+      S[e] = aa * sv[u] - gs;
+    }
   }
 }
 
