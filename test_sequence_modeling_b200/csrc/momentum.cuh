@@ -58,8 +58,10 @@ struct Smem {
   float part[MAXB][4][D];    // per-quarter partial column sums: k_t W_base, then q_t W_t
 };
 
-template <bool LN, typename InT, bool MOMENTUM = true>
-__global__ void __launch_bounds__(THREADS) momentum_fwd_kernel(const Params p) {
+// MINB: CTAs per SM the registers are capped for (4: 64 registers and a few
+// spills, so that 4 x 148 units run in one wave; 1: no cap, 2-3 CTAs per SM).
+template <bool LN, typename InT, bool MOMENTUM = true, int MINB = 1>
+__global__ void __launch_bounds__(THREADS, MINB) momentum_fwd_kernel(const Params p) {
   __shared__ Smem s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int j = tid & (D - 1), rq = tid >> 6;

@@ -129,6 +129,30 @@ int validate(const Call &c) {
   return TTT_OK;
 }
 
+// Launches the register-state kernel (b <= 16) in whichever register budget runs
+// `grid` CTAs in fewer waves on this device: capped for 4 CTAs per SM (a few
+// spills) or uncapped (2-3 CTAs per SM); a tie keeps the uncapped one.
+template <bool LN, typename InT, bool MOMENTUM>
+int launch_register_state(unsigned grid, cudaStream_t s, const mom::Params &p) {
+  auto k1 = mom::momentum_fwd_kernel<LN, InT, MOMENTUM, 1>;
+  auto k4 = mom::momentum_fwd_kernel<LN, InT, MOMENTUM, 4>;
+  int dev = 0, sms = 0, occ1 = 0, occ4 = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, k1, mom::THREADS, 0) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ4, k4, mom::THREADS, 0) != cudaSuccess)
+    return TTT_ERR_CUDA;
+  auto waves = [&](int occ) {
+    const long long slots = (long long)sms * occ;
+    return slots > 0 ? ((long long)grid + slots - 1) / slots : (1LL << 62);
+  };
+  if (waves(occ4) < waves(occ1)) k4<<<grid, mom::THREADS, 0, s>>>(p);
+  else k1<<<grid, mom::THREADS, 0, s>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return TTT_OK;
+}
+
 template <typename KernelT>
 int launch(KernelT kernel, int grid, size_t smem, cudaStream_t stream,
            const simt::Params &p, int threads = simt::THREADS) {
@@ -173,16 +197,11 @@ int run_simt(const Call &c) {
     // instantiation of the momentum kernel).
     mom::Params q{c.Q, c.K, c.V, c.eta, nullptr, nullptr, c.W0, c.gamma, c.beta, c.eps,
                   c.H, c.T, c.b, c.Z, c.W_out, nullptr};
-    if (c.kind == LINEAR_LN) {
-      if (bf16) mom::momentum_fwd_kernel<true, __nv_bfloat16, false><<<grid, mom::THREADS, 0, s>>>(q);
-      else mom::momentum_fwd_kernel<true, float, false><<<grid, mom::THREADS, 0, s>>>(q);
-    } else {
-      if (bf16) mom::momentum_fwd_kernel<false, __nv_bfloat16, false><<<grid, mom::THREADS, 0, s>>>(q);
-      else mom::momentum_fwd_kernel<false, float, false><<<grid, mom::THREADS, 0, s>>>(q);
-    }
-    if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
-    g_launches.fetch_add(1, std::memory_order_relaxed);
-    return TTT_OK;
+    if (c.kind == LINEAR_LN)
+      return bf16 ? launch_register_state<true, __nv_bfloat16, false>(grid, s, q)
+                  : launch_register_state<true, float, false>(grid, s, q);
+    return bf16 ? launch_register_state<false, __nv_bfloat16, false>(grid, s, q)
+                : launch_register_state<false, float, false>(grid, s, q);
   }
   const size_t smem = simt::linear_smem_bytes(c.b);
   if (c.kind == LINEAR_LN)
@@ -569,16 +588,11 @@ int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int q
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)units;
   const bool bf16 = qkv_dtype == TTT_BF16;
-  if (ln) {
-    if (bf16) mom::momentum_fwd_kernel<true, __nv_bfloat16><<<grid, mom::THREADS, 0, s>>>(p);
-    else mom::momentum_fwd_kernel<true, float><<<grid, mom::THREADS, 0, s>>>(p);
-  } else {
-    if (bf16) mom::momentum_fwd_kernel<false, __nv_bfloat16><<<grid, mom::THREADS, 0, s>>>(p);
-    else mom::momentum_fwd_kernel<false, float><<<grid, mom::THREADS, 0, s>>>(p);
-  }
-  if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
-  g_launches.fetch_add(1, std::memory_order_relaxed);
-  return TTT_OK;
+  if (ln)
+    return bf16 ? launch_register_state<true, __nv_bfloat16, true>(grid, s, p)
+                : launch_register_state<true, float, true>(grid, s, p);
+  return bf16 ? launch_register_state<false, __nv_bfloat16, true>(grid, s, p)
+              : launch_register_state<false, float, true>(grid, s, p);
 }
 
 int run_mlp_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
