@@ -274,15 +274,15 @@ TF32_PER_BF16 = 1.1 / 2.25
 
 def tensor_peak_scale(cfg, path):
     """Peak of the path's contractions relative to the measured bf16 peak.  The
-    TTT-MLP tensor-core path runs, per head-token, 10 d h + 4 b d + 2 b h FLOPs as
-    tf32 ([K;Q] W1, G3 W2^T, both state updates, the masked Q K^T products) and
-    4 d h + 2 b h as fp16 (X2 W2, Zq2 W2 and the Gram Zq2 X2^T); each kind at its
-    own peak gives the time at the roofline."""
+    TTT-MLP tensor-core path runs, per head-token, 8 d h + 4 b d + 2 b h FLOPs as
+    tf32 ([K;Q] W1, both state updates, the masked Q K^T products) and 6 d h + 2 b h
+    as fp16 (X2 W2, Zq2 W2, G3 W2^T and the Gram Zq2 X2^T); each kind at its own
+    peak gives the time at the roofline."""
     if cfg.variant != "mlp" or not tc_path(cfg, path):
         return 1.0
     d, b, h = cfg.d, cfg.b, cfg.hidden
-    tf32 = 10.0 * d * h + 4.0 * b * d + 2.0 * b * h
-    f16 = 4.0 * d * h + 2.0 * b * h
+    tf32 = 8.0 * d * h + 4.0 * b * d + 2.0 * b * h
+    f16 = 6.0 * d * h + 2.0 * b * h
     return (tf32 + f16) / (tf32 / TF32_PER_BF16 + f16)
 
 

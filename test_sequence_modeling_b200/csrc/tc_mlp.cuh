@@ -92,7 +92,7 @@ constexpr uint32_t OFF_KQ = 32768;      // [K;Q] of the chunk [d-block 2][row 12
 constexpr uint32_t OFF_X2 = 65536;      // X2  [hidden-block 4][token 16][64 fp16], K-major
 constexpr uint32_t OFF_Z2 = 73728;      // Zq2 same layout
 constexpr uint32_t OFF_KM = 81920;      // K of the mini-batch [d-block 2][token 16][128B] fp32, MN-major
-constexpr uint32_t OFF_G3 = 86016;      // G3  [d-block 2][token 16][128B] fp32, K-major
+constexpr uint32_t OFF_G3 = 86016;      // G3  [token 16][64 d fp16], K-major
 constexpr uint32_t OFF_E3 = 90112;      // E3  same shape, MN-major
 constexpr uint32_t OFF_S1 = 94208;      // masked Q K^T in P1's column order [row 32][128B]
 constexpr uint32_t OFF_S2U = 98304;     // striu(S2) [query token 16][128B]
@@ -112,6 +112,8 @@ enum {
   BAR_LOAD0 = 0, BAR_LOAD1 = 1, BAR_S1C = 2, BAR_P1 = 3, BAR_X3 = 4, BAR_GW = 5, BAR_UPD = 6,
   BAR_S2 = 7, BAR_ZQ3 = 8, BAR_DRAIN = 9, BAR_NEVER = 10, NUM_BARS = 11
 };
+// The warp that issues Zq3 and its correction (and, with the next warp, P1).
+constexpr int ZQ3_WARP = 4;
 constexpr long long WAIT_LIMIT = 1ll << 32;
 constexpr long long INJECTED_WAIT_LIMIT = 1ll << 20;
 
@@ -202,7 +204,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t sbase = smem_u32(sm);
 
   if (tid == 0) {
-    for (int i = 0; i < NUM_BARS; ++i) mbar_init(&bars[i], 1);
+    // P1, X3 and GW arrive once per half (two issuing warps); the drain once per
+    // issuing warp.
+    for (int i = 0; i < NUM_BARS; ++i)
+      mbar_init(&bars[i], (i == BAR_P1 || i == BAR_X3 || i == BAR_GW) ? 2 : i == BAR_DRAIN ? 3 : 1);
     *abort = 0;
     fence_mbarrier_init();
     prefetch_tensormap(&tmQ);
@@ -289,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   // Instruction descriptors.
   constexpr uint32_t ID_P1 = idesc_tf32_f32(128, 32, false, false, false);   // W1^T(TMEM) x [K;Q]
   constexpr uint32_t ID_X3 = idesc_f16_f32(64, 16, true, false, false);      // W2^T x X2 (and Zq2)
-  constexpr uint32_t ID_GW = idesc_tf32_f32(128, 16, false, false, false);   // W2(TMEM) x G3
+  constexpr uint32_t ID_GW = idesc_f16_f32(128, 16, false, false, false);    // W2 copy x G3, fp16
   constexpr uint32_t ID_UPD = idesc_tf32_f32(128, 64, false, true, true);    // state -= A(TMEM) B
   constexpr uint32_t ID_ZQ1 = idesc_tf32_f32(128, 32, false, false, true);   // P1 -= E2^T(TMEM) S1^T
   constexpr uint32_t ID_S1 = idesc_tf32_f32(128, 64, false, false, false);   // [K;Q] x K
@@ -302,27 +307,28 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   // Phase counters of the MMA barriers (every thread waits on each in order).
   uint32_t n_s1c = 0, n_p1 = 0, n_x3 = 0, n_gw = 0, n_upd = 0, n_s2 = 0, n_zq3 = 0;
-  int issued_mma = 0;  // whether warp 0 has issued products (for the drain)
 
-  // Products are issued by warp 0 (one lane elected inside each instruction's asm
-  // block, the warp converged) after a CTA barrier.
-  auto issue_p1 = [&](int m) {
+  // Products are issued by whole converged warps (one lane elected inside each
+  // instruction's asm block) after a CTA barrier: warp 0 the chain's products and
+  // the Gram, warp ZQ3_WARP Zq3 and its correction, then, with warp ZQ3_WARP + 1,
+  // one half each of the next mini-batch's P1, so that P1 runs under the output LN.
+  // Half h of P1 = W1^T [K;Q]^T for mini-batch m, committed on BAR_P1.
+  auto issue_p1_half = [&](int m, int h) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint64_t b = smem_desc_sw128(aKQ + m * 4096 + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
-        umma_ts_tf32_w(tb + C_P1 + 32 * h, tb + C_W1 + 64 * h + 8 * i, b, ID_P1, i > 0);
-      }
+    for (int i = 0; i < 8; ++i) {
+      const uint64_t b = smem_desc_sw128(aKQ + m * 4096 + (i >> 2) * 16384 + (i & 3) * 32, 16, 1024);
+      umma_ts_tf32_w(tb + C_P1 + 32 * h, tb + C_W1 + 64 * h + 8 * i, b, ID_P1, i > 0);
+    }
     umma_commit_w(&bars[BAR_P1]);
   };
-  // W2^T (M = d, fp16) against a [16 token][hidden] fp16 operand (X2 or Zq2).
-  auto issue_w2t = [&](uint32_t d_tmem, uint32_t aB) {
+  // W2^T (M = d, fp16) against a [16 token][hidden] fp16 operand (X2 or Zq2), hidden
+  // steps i0 .. i1 - 1 of 16.
+  auto issue_w2t = [&](uint32_t d_tmem, uint32_t aB, int i0 = 0, int i1 = 16) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
+    for (int i = i0; i < i1; ++i) {
       const uint64_t a = smem_desc_sw128(aW2 + i * 2048, 8192, 1024);
       const uint64_t b = smem_desc_sw128(aB + (i >> 2) * 2048 + (i & 3) * 32, 16, 1024);
-      umma_ss_w(d_tmem, a, b, ID_X3, i > 0);
+      umma_ss_w(d_tmem, a, b, ID_X3, i > i0);
     }
   };
 
@@ -352,10 +358,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
+    if (warp == ZQ3_WARP || warp == ZQ3_WARP + 1) {
+      __syncwarp();
+      tc_fence_after_sync();
+      issue_p1_half(0, warp - ZQ3_WARP);
+      __syncwarp();
+    }
     if (warp == 0) {
       __syncwarp();
       tc_fence_after_sync();
-      issue_p1(0);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const uint32_t off = (i >> 2) * 16384 + (i & 3) * 32;
@@ -363,7 +374,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                        smem_desc_sw128(aKQ + off, 16, 2048), ID_S1, i > 0);
       }
       umma_commit_w(&bars[BAR_S1C]);
-      issued_mma = 1;
       __syncwarp();
     }
 
@@ -397,11 +407,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before_sync();
       __syncthreads();
       tc_fence_after_sync();
-      // ---- X3^T = W2^T X2^T ----------------------------------------------------
-      if (warp == 0) {
+      // ---- X3^T = W2^T X2^T: hidden units 0-127 by warp 0 into lanes 0-15, 128-255
+      // by warp ZQ3_WARP into lanes 16-31 of the same columns (summed when read) ----
+      if (warp == 0 || warp == ZQ3_WARP) {
         __syncwarp();
         tc_fence_after_sync();
-        issue_w2t(tb + C_X3, aX2);
+        if (warp == 0) issue_w2t(tb + C_X3, aX2, 0, 8);
+        else issue_w2t(tmem_addr(tb, 16, C_X3), aX2, 8, 16);
         umma_commit_w(&bars[BAR_X3]);
         __syncwarp();
       }
@@ -419,11 +431,12 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (warp < 4) {
         uint32_t r[16];
-        tmem_ld_32x32b_x16(tq + C_X3, r);  // lanes 0-15: d = 16 qd + lane, 16 tokens
+        tmem_ld_32x32b_x16(tq + C_X3, r);  // lanes 0-15 / 16-31: the two hidden halves, d = 16 qd + lane % 16
         tmem_wait_ld();
-        if (lane < 16) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) red[j * RS + 16 * qd + lane] = __uint_as_float(r[j]);
+        for (int j = 0; j < 16; ++j) {
+          const float v = __uint_as_float(r[j]) + __shfl_xor_sync(0xffffffffu, __uint_as_float(r[j]), 16);
+          if (lane < 16) red[j * RS + 16 * qd + lane] = v;
         }
       }
       tc_fence_before_sync();
@@ -449,8 +462,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const float g0 = r * (a0 - ma - h0 * mb), g1 = r * (a1 - ma - h1 * mb);
         const float e = eta_s[tc];
         const uint32_t blk = (dc >> 5) * 2048u;
-        *reinterpret_cast<float2 *>(sm + OFF_G3 + blk + swz32(t, dc & 31)) =
-            make_float2(round_tf32(g0), round_tf32(g1));
+        *reinterpret_cast<__half2 *>(sm + OFF_G3 + swz16(t, dc)) = __floats2half2_rn(g0, g1);
         *reinterpret_cast<float2 *>(sm + OFF_E3 + blk + swzb32(t, dc & 31)) =
             make_float2(round_tf32(e * g0), round_tf32(e * g1));
       }
@@ -458,17 +470,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before_sync();
       __syncthreads();
       tc_fence_after_sync();
-      // ---- GW^T = W2 G3^T (A = the W2 state in TMEM) --------------------------------
-      if (warp == 0) {
+      // ---- GW^T = W2 G3^T: fp16, A = the W2 copy ([hidden][d], K-major), hidden
+      // half h by warp 0 (h = 0) and warp ZQ3_WARP (h = 1) ---------------------------
+      if (warp == 0 || warp == ZQ3_WARP) {
         __syncwarp();
         tc_fence_after_sync();
+        const int h = warp == 0 ? 0 : 1;
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const uint64_t b = smem_desc_sw128(aG3 + (i >> 2) * 2048 + (i & 3) * 32, 16, 1024);
-            umma_ts_tf32_w(tb + C_GW + 16 * h, tb + C_W2 + 64 * h + 8 * i, b, ID_GW, i > 0);
-          }
+        for (int k = 0; k < 4; ++k)
+          umma_ss_w(tb + C_GW + 16 * h, smem_desc_sw128(aW2 + h * 16384 + 32 * k, 16, 1024),
+                    smem_desc_sw128(aG3 + 32 * k, 16, 1024), ID_GW, k > 0);
         umma_commit_w(&bars[BAR_GW]);
         __syncwarp();
       }
@@ -558,17 +569,20 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before_sync();
       __syncthreads();
       tc_fence_after_sync();
-      // ---- next P1 first (it starts the next mini-batch's chain), then the Gram of
-      // Zq2 X2^T and Zq3^T = W2'^T Zq2^T ------------------------------------------------
+      // ---- the Gram of Zq2 X2^T (warp 0) and Zq3^T = W2'^T Zq2^T (warp ZQ3_WARP) ------
       if (warp == 0) {
         __syncwarp();
         tc_fence_after_sync();
-        if (m + 1 < nmb) issue_p1(m + 1);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           umma_ss_w(tb + C_S2, smem_desc_sw128(aZ2 + i * 32, 16, 1024),
                     smem_desc_sw128(aX2 + i * 32, 16, 1024), ID_G2, i > 0);
         umma_commit_w(&bars[BAR_S2]);
+        __syncwarp();
+      }
+      if (warp == ZQ3_WARP) {
+        __syncwarp();
+        tc_fence_after_sync();
         issue_w2t(tmem_addr(tb, 16, C_X3), aZ2);
         __syncwarp();
       }
@@ -597,8 +611,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before_sync();
       __syncthreads();
       tc_fence_after_sync();
-      // ---- Zq3^T += E3^T striu(S2)^T ------------------------------------------------
-      if (warp == 0) {
+      // ---- Zq3^T += E3^T striu(S2)^T (after Zq3, by the same warp); then the next
+      // mini-batch's P1, which runs under the output LN ------------------------------
+      if (warp == ZQ3_WARP) {
         __syncwarp();
         tc_fence_after_sync();
 #pragma unroll
@@ -608,6 +623,12 @@ __global__ void __launch_bounds__(THREADS, 1)
           umma_ss_tf32_w(tmem_addr(tb, 16, C_X3), a, b, ID_ZC, true);
         }
         umma_commit_w(&bars[BAR_ZQ3]);
+        __syncwarp();
+      }
+      if ((warp == ZQ3_WARP || warp == ZQ3_WARP + 1) && m + 1 < nmb) {
+        __syncwarp();
+        tc_fence_after_sync();
+        issue_p1_half(m + 1, warp - ZQ3_WARP);
         __syncwarp();
       }
       mma_wait(&bars[BAR_ZQ3], n_zq3++ & 1u, abort);
@@ -651,12 +672,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int k = 0; k < loads_issued; ++k)
         mbar_wait(&bars[BAR_LOAD0 + (k & 1)], (uint32_t)(k >> 1) & 1u, WAIT_LIMIT);
     }
-    if (warp == 0 && issued_mma) {
+    // Every warp that issues products commits once (a commit with nothing in flight
+    // arrives at once), and those warps wait for all of them.
+    const bool issuer = warp == 0 || warp == ZQ3_WARP || warp == ZQ3_WARP + 1;
+    if (issuer) {
       __syncwarp();
       umma_commit_w(&bars[BAR_DRAIN]);
       __syncwarp();
+      mbar_wait(&bars[BAR_DRAIN], 0, WAIT_LIMIT);
     }
-    if (issued_mma) mbar_wait(&bars[BAR_DRAIN], 0, WAIT_LIMIT);
     tc_fence_after_sync();
   }
   __syncthreads();
