@@ -306,6 +306,8 @@ def main():
     ap.add_argument("--workload", default="linear_ln_B16H32T8192", choices=I.CONFIG_ORDER)
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-chunks", type=int, default=16,
+                    help="batch chunks whose copies overlap the kernels in the end-to-end line")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B (smaller profiling cases)")
     ap.add_argument("--seq", type=int, default=None, help="override T (smaller profiling cases)")
@@ -834,7 +836,8 @@ def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, 
         params = [pin["W0"]] + ([pin["gamma"], pin["beta"]] if cfg.variant == "linear_ln" else [])
         w_shapes = [(cfg.H, cfg.d, cfg.d)]
         w_keys = ["W_out"]
-    fwd = HostForward(cfg.variant, pin["Q"], w_shapes, [p.shape for p in params], chunks=4, device=dev)
+    fwd = HostForward(cfg.variant, pin["Q"], w_shapes, [p.shape for p in params], chunks=args.e2e_chunks,
+                      device=dev)
 
     def e2e_step(after=None):
         return fwd.run(pin["Q"], pin["K"], pin["V"], pin["eta"], params, cfg.b, cfg.ln_eps, h_out["Z"],
@@ -857,8 +860,8 @@ def measure_e2e(args, cfg, host, outs, d_in, step, stream, barrier, world, dev, 
     e2e_value = world * cfg.head_tokens * args.e2e_steps / (te / 1e3)
     return {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": args.e2e_steps,
-            "api": "ttt_fwd_host (C ABI, host buffers; 4 batch chunks, copies overlapped) through "
-                   "test_sequence_modeling_b200.host.HostForward"}
+            "api": f"ttt_fwd_host (C ABI, host buffers; {args.e2e_chunks} batch chunks, copies overlapped) "
+                   "through test_sequence_modeling_b200.host.HostForward"}
 
 
 def finish(args, cfg, world, rank, value, ms_per_step, kernel_avg_ms, clock_info, launches, e2e,
