@@ -30,8 +30,10 @@
 // caller's W_ckpt (so the reverse pass needs no recomputation chain), then the
 // reverse pass recomputes G, E (and the output LN) from W_n and applies the
 // step above.  One CTA of 256 threads per unit; every [row][D] tile, W and dW
-// live in shared memory with a padded row stride (D + 1), so row and column
-// walks are both free of bank conflicts.
+// live in shared memory with rows of D + 4 floats: 16-byte aligned, so that the
+// products read four consecutive elements per load, and a row stride of 17
+// 16-byte units, so that 16-byte walks down a column (one row per lane) are free
+// of bank conflicts.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -44,7 +46,7 @@ namespace bwd {
 
 constexpr int D = simt::D;
 constexpr int MAXB = 16;     // largest mini-batch of this kernel
-constexpr int LD = D + 1;    // padded row stride of every tile
+constexpr int LD = D + 4;    // row stride of every tile (16-byte rows, 17 x 16 bytes)
 constexpr int BLD = MAXB + 1;
 constexpr int THREADS = 256;
 
@@ -78,19 +80,26 @@ struct Smem {
 
 inline size_t smem_bytes() { return sizeof(Smem); }
 
+// Four consecutive floats of a tile (16-byte aligned: rows are LD = D + 4 floats).
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+
 // The [row][D] products are register-blocked over the four rows rq + 4k of a
-// thread: one column operand load serves four FMAs (the row operands are
-// warp-wide broadcasts).  Rows at or beyond b hold stale values; their sums are
-// computed and dropped.
+// thread and four steps of the inner index: the row operands are warp-wide
+// broadcasts read four elements at a time, so one column-operand load serves
+// four FMAs and one row-operand load four more.  Rows at or beyond b hold stale
+// values; their sums are computed and dropped.
 //
 // acc[k] += sum_i in[rq + 4k][i] W[i][c]
 __device__ __forceinline__ void rows_W(const float *in, const float *W, int rq, int c,
                                        float (&acc)[4]) {
-#pragma unroll 8
-  for (int i = 0; i < D; ++i) {
-    const float w = W[i * LD + c];
+#pragma unroll 2
+  for (int i = 0; i < D; i += 4) {
+    const float4 w = make_float4(W[i * LD + c], W[(i + 1) * LD + c], W[(i + 2) * LD + c], W[(i + 3) * LD + c]);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = fmaf(in[(rq + 4 * k) * LD + i], w, acc[k]);
+    for (int k = 0; k < 4; ++k) acc[k] = dot4(ld4(in + (rq + 4 * k) * LD + i), w, acc[k]);
   }
 }
 
@@ -197,7 +206,7 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
     __syncthreads();
     grad_rows<LN>(s, b, warp, lane, g0, g1, be0, be1, p.eps);
     __syncthreads();
-    // W -= K^T E; this thread's rows i = rq + 4k of column col.
+    // W -= K^T E; this thread's rows i = 16 rq + k of column col.
     {
       float acc[16];
 #pragma unroll
@@ -205,10 +214,16 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
       for (int r = 0; r < b; ++r) {
         const float e = s.E[r * LD + col];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc[k] = fmaf(s.K[r * LD + rq + 4 * k], e, acc[k]);
+        for (int q = 0; q < 4; ++q) {
+          const float4 kv = ld4(s.K + r * LD + 16 * rq + 4 * q);
+          acc[4 * q] = fmaf(kv.x, e, acc[4 * q]);
+          acc[4 * q + 1] = fmaf(kv.y, e, acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(kv.z, e, acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(kv.w, e, acc[4 * q + 3]);
+        }
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k) s.W[(rq + 4 * k) * LD + col] -= acc[k];
+      for (int k = 0; k < 16; ++k) s.W[(16 * rq + k) * LD + col] -= acc[k];
     }
     __syncthreads();
   }
@@ -235,8 +250,8 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
       if (t < b && u < b) {
         float a = 0.f;
         if (u <= t) {
-#pragma unroll 16
-          for (int i = 0; i < D; ++i) a = fmaf(s.Q[t * LD + i], s.K[u * LD + i], a);
+#pragma unroll 4
+          for (int i = 0; i < D; i += 4) a = dot4(ld4(s.Q + t * LD + i), ld4(s.K + u * LD + i), a);
         }
         s.A[t * BLD + u] = a;
       }
@@ -290,8 +305,8 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
       if (t < b && u < b) {
         float m = 0.f;
         if (u <= t) {
-#pragma unroll 16
-          for (int j = 0; j < D; ++j) m = fmaf(P[t * LD + j], s.E[u * LD + j], m);
+#pragma unroll 4
+          for (int j = 0; j < D; j += 4) m = dot4(ld4(P + t * LD + j), ld4(s.E + u * LD + j), m);
         }
         s.M[t * BLD + u] = m;
       }
@@ -301,13 +316,15 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
     // dQ (to global) and dE.  Here col is the output column (i for dQ, j for dE).
     {
       float q[4] = {0.f, 0.f, 0.f, 0.f}, e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-      for (int j = 0; j < D; ++j) {
-        const float w = s.W[col * LD + j], dw = s.dW[j * LD + col];
+#pragma unroll 2
+      for (int j = 0; j < D; j += 4) {
+        const float4 w = ld4(s.W + col * LD + j);
+        const float4 dw = make_float4(-s.dW[j * LD + col], -s.dW[(j + 1) * LD + col], -s.dW[(j + 2) * LD + col],
+                                      -s.dW[(j + 3) * LD + col]);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          q[k] = fmaf(P[(rq + 4 * k) * LD + j], w, q[k]);
-          e[k] = fmaf(-s.K[(rq + 4 * k) * LD + j], dw, e[k]);
+          q[k] = dot4(ld4(P + (rq + 4 * k) * LD + j), w, q[k]);
+          e[k] = dot4(ld4(s.K + (rq + 4 * k) * LD + j), dw, e[k]);
         }
       }
 #pragma unroll
@@ -376,13 +393,14 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
     // dK (to global); col is the output column i.
     {
       float kk[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-      for (int j = 0; j < D; ++j) {
-        const float dw = s.dW[col * LD + j], w = s.W[col * LD + j];
+#pragma unroll 2
+      for (int j = 0; j < D; j += 4) {
+        const float4 dw = ld4(s.dW + col * LD + j), w = ld4(s.W + col * LD + j);
+        const float4 ndw = make_float4(-dw.x, -dw.y, -dw.z, -dw.w);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          kk[k] = fmaf(-s.E[(rq + 4 * k) * LD + j], dw, kk[k]);
-          kk[k] = fmaf(s.dY[(rq + 4 * k) * LD + j], w, kk[k]);
+          kk[k] = dot4(ld4(s.E + (rq + 4 * k) * LD + j), ndw, kk[k]);
+          kk[k] = dot4(ld4(s.dY + (rq + 4 * k) * LD + j), w, kk[k]);
         }
       }
 #pragma unroll
@@ -397,7 +415,7 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
     }
     __syncthreads();
 
-    // dW_n = dW_{n+1} + Q^T P + K^T dY; this thread's rows i = rq + 4k of column col.
+    // dW_n = dW_{n+1} + Q^T P + K^T dY; this thread's rows i = 16 rq + k of column col.
     {
       float acc[16];
 #pragma unroll
@@ -405,13 +423,16 @@ __global__ void __launch_bounds__(THREADS) linear_bwd_kernel(const Params p) {
       for (int r = 0; r < b; ++r) {
         const float pr = P[r * LD + col], dyr = s.dY[r * LD + col];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          acc[k] = fmaf(s.Q[r * LD + rq + 4 * k], pr, acc[k]);
-          acc[k] = fmaf(s.K[r * LD + rq + 4 * k], dyr, acc[k]);
+        for (int q = 0; q < 4; ++q) {
+          const float4 qv = ld4(s.Q + r * LD + 16 * rq + 4 * q), kv = ld4(s.K + r * LD + 16 * rq + 4 * q);
+          acc[4 * q] = fmaf(kv.x, dyr, fmaf(qv.x, pr, acc[4 * q]));
+          acc[4 * q + 1] = fmaf(kv.y, dyr, fmaf(qv.y, pr, acc[4 * q + 1]));
+          acc[4 * q + 2] = fmaf(kv.z, dyr, fmaf(qv.z, pr, acc[4 * q + 2]));
+          acc[4 * q + 3] = fmaf(kv.w, dyr, fmaf(qv.w, pr, acc[4 * q + 3]));
         }
       }
 #pragma unroll
-      for (int k = 0; k < 16; ++k) s.dW[(rq + 4 * k) * LD + col] += acc[k];
+      for (int k = 0; k < 16; ++k) s.dW[(16 * rq + k) * LD + col] += acc[k];
     }
     __syncthreads();
   }
