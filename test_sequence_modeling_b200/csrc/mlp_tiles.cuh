@@ -23,6 +23,10 @@ constexpr int LDB = MAXB + 1;
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// Four consecutive floats of a tile: every tile row (LDD, LDH floats) and every
+// tile base is 16-byte aligned, and the callers index in steps of 4.
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+
 __device__ __forceinline__ float wsum(float x) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
@@ -43,11 +47,15 @@ __device__ void mm_W(float *out, int ldo, const float *A, int lda, const float *
   float a[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) a[r] = 0.f;
-#pragma unroll 8
-  for (int k = 0; k < Kd; ++k) {
-    const float w = W[(size_t)k * N + j];
+#pragma unroll 2
+  for (int k = 0; k < Kd; k += 4) {
+    const float w0 = W[(size_t)k * N + j], w1 = W[(size_t)(k + 1) * N + j];
+    const float w2 = W[(size_t)(k + 2) * N + j], w3 = W[(size_t)(k + 3) * N + j];
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) a[r] = fmaf(A[(g * RPT + r) * lda + k], w, a[r]);
+    for (int r = 0; r < RPT; ++r) {
+      const float4 x = ld4(A + (g * RPT + r) * lda + k);
+      a[r] = fmaf(x.w, w3, fmaf(x.z, w2, fmaf(x.y, w1, fmaf(x.x, w0, a[r]))));
+    }
   }
 #pragma unroll
   for (int r = 0; r < RPT; ++r) {
@@ -111,24 +119,36 @@ template <int R, int C>
 __device__ void outer(float *dst, const float *src, const float *L, int ldl, const float *Rt, int ldr,
                       int b, float sign, int tid) {
   constexpr int GROUPS = THREADS / C, RPG = R / GROUPS;
-  static_assert(RPG % ROW_BLOCK == 0, "rows per thread group must fill whole blocks");
+  static_assert(RPG % ROW_BLOCK == 0 && ROW_BLOCK == 8, "rows per thread group must fill whole 8-row blocks");
   const int c = tid % C, g = tid / C;
   float rt[MAXB];
 #pragma unroll
   for (int t = 0; t < MAXB; ++t) rt[t] = t < b ? Rt[t * ldr + c] : 0.f;
   for (int i0 = 0; i0 < RPG; i0 += ROW_BLOCK) {
-    float sv[ROW_BLOCK];
-#pragma unroll
-    for (int u = 0; u < ROW_BLOCK; ++u) sv[u] = src[(size_t)(g * RPG + i0 + u) * C + c];
+    const int r0 = g * RPG + i0;
+    float sv[ROW_BLOCK], a[ROW_BLOCK];
 #pragma unroll
     for (int u = 0; u < ROW_BLOCK; ++u) {
-      const int r = g * RPG + i0 + u;
-      float a = 0.f;
-#pragma unroll
-      for (int t = 0; t < MAXB; ++t)
-        if (t < b) a = fmaf(L[t * ldl + r], rt[t], a);
-      dst[(size_t)r * C + c] = sv[u] + sign * a;
+      sv[u] = src[(size_t)(r0 + u) * C + c];
+      a[u] = 0.f;
     }
+    // L[t][r0 .. r0 + 7]: two 16-byte loads per token (warp-wide broadcasts).
+#pragma unroll
+    for (int t = 0; t < MAXB; ++t)
+      if (t < b) {
+        const float4 l0 = ld4(L + t * ldl + r0), l1 = ld4(L + t * ldl + r0 + 4);
+        const float x = rt[t];
+        a[0] = fmaf(l0.x, x, a[0]);
+        a[1] = fmaf(l0.y, x, a[1]);
+        a[2] = fmaf(l0.z, x, a[2]);
+        a[3] = fmaf(l0.w, x, a[3]);
+        a[4] = fmaf(l1.x, x, a[4]);
+        a[5] = fmaf(l1.y, x, a[5]);
+        a[6] = fmaf(l1.z, x, a[6]);
+        a[7] = fmaf(l1.w, x, a[7]);
+      }
+#pragma unroll
+    for (int u = 0; u < ROW_BLOCK; ++u) dst[(size_t)(r0 + u) * C + c] = sv[u] + sign * a[u];
   }
 }
 

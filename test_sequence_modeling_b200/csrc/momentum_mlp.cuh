@@ -74,14 +74,19 @@ __device__ void mm_two(float *out, int ldo, const float *A, int lda, const float
   float a[RPT], c[RPT];
 #pragma unroll
   for (int r = 0; r < RPT; ++r) a[r] = c[r] = 0.f;
-#pragma unroll 8
-  for (int k = 0; k < Kd; ++k) {
-    const float w = W[(size_t)k * N + j], sv = S[(size_t)k * N + j];
+#pragma unroll 2
+  for (int k = 0; k < Kd; k += 4) {
+    float w[4], sv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      w[u] = W[(size_t)(k + u) * N + j];
+      sv[u] = S[(size_t)(k + u) * N + j];
+    }
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
-      const float x = A[(g * RPT + r) * lda + k];
-      a[r] = fmaf(x, w, a[r]);
-      c[r] = fmaf(x, sv, c[r]);
+      const float4 x = ld4(A + (g * RPT + r) * lda + k);
+      a[r] = fmaf(x.w, w[3], fmaf(x.z, w[2], fmaf(x.y, w[1], fmaf(x.x, w[0], a[r]))));
+      c[r] = fmaf(x.w, sv[3], fmaf(x.z, sv[2], fmaf(x.y, sv[1], fmaf(x.x, sv[0], c[r]))));
     }
   }
 #pragma unroll
@@ -116,20 +121,26 @@ __device__ void update_state(float *W, float *S, const float *L, int ldl, const 
       wv[u] = W[e];
       sv[u] = S[e];
     }
+    const int r0 = g * RPG + i0;
+    float gw[ROW_BLOCK], gs[ROW_BLOCK];
+#pragma unroll
+    for (int u = 0; u < ROW_BLOCK; ++u) gw[u] = gs[u] = 0.f;
+#pragma unroll
+    for (int t = 0; t < MAXB; ++t)
+      if (t < b) {
+        const float4 l0 = ld4(L + t * ldl + r0), l1 = ld4(L + t * ldl + r0 + 4);
+        const float l[ROW_BLOCK] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+#pragma unroll
+        for (int u = 0; u < ROW_BLOCK; ++u) {
+          gw[u] = fmaf(l[u], rw[t], gw[u]);
+          gs[u] = fmaf(l[u], rs[t], gs[u]);
+        }
+      }
 #pragma unroll
     for (int u = 0; u < ROW_BLOCK; ++u) {
-      const int r = g * RPG + i0 + u;
-      float gw = 0.f, gs = 0.f;
-#pragma unroll
-      for (int t = 0; t < MAXB; ++t)
-        if (t < b) {
-          const float l = L[t * ldl + r];
-          gw = fmaf(l, rw[t], gw);
-          gs = fmaf(l, rs[t], gs);
-        }
-      const size_t e = (size_t)r * C + c;
-      W[e] = lam * wv[u] + cc * sv[u] - gw;
-      S[e] = aa * sv[u] - gs;
+      const size_t e = (size_t)(r0 + u) * C + c;
+      W[e] = lam * wv[u] + cc * sv[u] - gw[u];
+      S[e] = aa * sv[u] - gs[u];
     }
   }
 }
