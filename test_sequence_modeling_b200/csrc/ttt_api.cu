@@ -23,6 +23,7 @@
 #include "momentum_mlp.cuh"
 #include "simt.cuh"
 #include "tc_linear.cuh"
+#include "tc_momentum.cuh"
 #include "tc_mlp.cuh"
 
 namespace simt = ttt::simt;
@@ -33,6 +34,7 @@ namespace bwd = ttt::bwd;
 namespace bwdmlp = ttt::bwdmlp;
 namespace mom = ttt::mom;
 namespace mommlp = ttt::mommlp;
+namespace tcmom = ttt::tcmom;
 
 namespace {
 
@@ -584,10 +586,28 @@ int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int q
     for (int o2 = o + 1; o2 < 3; ++o2)
       if (overlap(outs[o], outs[o2])) return TTT_ERR_ARG;
   }
-  mom::Params p{Q, K, V, eta, alpha, lambda, W0, gamma, beta, eps, H, T, b, Z, W_out, S_out};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)units;
   const bool bf16 = qkv_dtype == TTT_BF16;
+  // TTT-Linear + LN with bf16 inputs and b = 16: the tensor-core dual form (unless
+  // the CUDA-core path is selected).
+  if (ln && bf16 && b == tcmom::MB && T > 0 && g_path.load() != TTT_PATH_SIMT) {
+    CUtensorMap mq, mk, mv;
+    if (!make_qkv_map(&mq, Q, T, units, 8) || !make_qkv_map(&mk, K, T, units, 8) ||
+        !make_qkv_map(&mv, V, T, units, tcmom::CHUNK))
+      return TTT_ERR_CUDA;
+    tcmom::Params tp{eta, alpha, lambda, W0, gamma, beta, eps, H, T, Z, W_out, S_out, g_inject_timeout.load()};
+    if (cudaFuncSetAttribute(tcmom::momentum_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tcmom::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(tcmom::momentum_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return TTT_ERR_CUDA;
+    tcmom::momentum_tc_kernel<<<grid, tcmom::THREADS, tcmom::SMEM_BYTES, s>>>(mq, mk, mv, tp);
+    if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return TTT_OK;
+  }
+  mom::Params p{Q, K, V, eta, alpha, lambda, W0, gamma, beta, eps, H, T, b, Z, W_out, S_out};
   if (ln)
     return bf16 ? launch_register_state<true, __nv_bfloat16, true>(grid, s, p)
                 : launch_register_state<true, float, true>(grid, s, p);
