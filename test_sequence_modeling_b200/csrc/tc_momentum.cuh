@@ -32,9 +32,16 @@
 // forward.
 //
 // Layout: the linear kernel's (one CTA of 4 warps per unit, [K;Q] rows in 8-row
-// groups, each mini-batch's chain step shared by two warps), with TMEM holding
-// X, Y, the corrections and S = [K;Q] K^T (256 columns: 2 CTAs per SM), W and S
-// in registers (fp32) and as bf16 hi + lo operands.  Precision: X, Y exact bf16
+// groups, each mini-batch's chain step shared by two warps), W and S in registers
+// (fp32) and as bf16 hi + lo operands.  The chunk head computes X, Y and the
+// Gram S = [K;Q] K^T on the tensor cores while one warp builds the coefficient
+// table c_{tau,sigma} (a walk down each column sigma, tau ascending:
+// c_{tau,sigma} = (1 - lambda_tau) c_{tau-1,sigma} + a_{tau,sigma}) and another
+// the prefix scans; every thread then scales its row of S by its coefficient row
+// (fp16, packed in place) and folds its rows of X and Y into one accumulator
+// P = rho X + kappa Y, which the chain's corrections decrement.  The state update
+// MMAs follow the last chain step directly, overlapping the last outputs.  TMEM:
+// P, Y (then dS), dW, S: 256 columns, 2 CTAs per SM.  Precision: X, Y exact bf16
 // K, Q against hi + lo pairs; the coefficient-weighted Gram, eta G and the
 // weighted K of the state update as fp16; fp32 accumulation.
 #pragma once
@@ -70,7 +77,7 @@ constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t OFF_A = 0;          // [K;Q] rows in 8-row groups (tc::kq_group); K rows later c-weighted fp16
 constexpr uint32_t OFF_WHI = 16384;    // W hi [d_in][d_out] bf16
 constexpr uint32_t OFF_WLO = 24576;    // W lo
-constexpr uint32_t OFF_SHI = 32768;    // S hi
+constexpr uint32_t OFF_SHI = 32768;    // S hi (W hi + 16 KB: the second atom of one B operand)
 constexpr uint32_t OFF_SLO = 40960;    // S lo
 constexpr uint32_t OFF_G = 49152;      // eta*G [token][d_out] fp16
 constexpr uint32_t OFF_V = 57344;      // V tile; then a-weighted K [token][d_in] fp16 (natural order)
@@ -88,7 +95,9 @@ constexpr uint32_t OFF_W2 = 68368;     // 2 gamma^2, 64 floats
 constexpr uint32_t OFF_BAR = 68624;    // mbarriers (14 x 8 bytes)
 constexpr uint32_t OFF_TSLOT = 68736;
 constexpr uint32_t OFF_ABORT = 68740;
-constexpr uint32_t SMEM_USED = 68744;
+constexpr uint32_t OFF_COEF = 68752;   // c_{tau,sigma} [tau][sigma], fp32, row stride COEF_LD
+constexpr int COEF_LD = 68;            // 17 x 16 bytes: 8 consecutive rows hit 8 distinct bank groups
+constexpr uint32_t SMEM_USED = OFF_COEF + CHUNK * COEF_LD * 4;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 
 enum {
@@ -151,10 +160,10 @@ __global__ void __launch_bounds__(THREADS, 2)
   float *CW = reinterpret_cast<float *>(sm + OFF_CW);
   float *AW = reinterpret_cast<float *>(sm + OFF_AW);
   float *FIN = reinterpret_cast<float *>(sm + OFF_FIN);
+  float *COEF = reinterpret_cast<float *>(sm + OFF_COEF);
   const uint32_t sbase = smem_u32(sm);
   const uint32_t aA = sbase + OFF_A;
-  const uint32_t aWhi = sbase + OFF_WHI, aWlo = sbase + OFF_WLO;
-  const uint32_t aShi = sbase + OFF_SHI, aSlo = sbase + OFF_SLO;
+  const uint32_t aWhi = sbase + OFF_WHI, aWlo = sbase + OFF_WLO;  // S hi, lo: 16 KB further
   const uint32_t aG = sbase + OFF_G, aV = sbase + OFF_V;
   const int q4 = lane & 3;
   const int fr = lane >> 2;
@@ -254,13 +263,14 @@ __global__ void __launch_bounds__(THREADS, 2)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tb = *tslot;
+  // P (first X), Y (then dS), dW, S.
   const uint32_t tX = tb, tY = tb + 64, tC = tb + 128, tS = tb + 192;
   if (tid == 0 && nchunks > 0) issue_loads_kv(0);
   if (lane == 0 && nchunks > 0) issue_load_q(0);
 
-  constexpr uint32_t ID_P = idesc_bf16_f32(128, 64, false, true, false);    // [K;Q] x W (or S)
   constexpr uint32_t ID_S = idesc_bf16_f32(128, 64, false, false, false);   // [K;Q] x K^T
-  constexpr uint32_t ID_CORR = idesc_f16_f32(128, 64, false, true, false);  // Corr += A' x (eta G)
+  constexpr uint32_t ID_P2 = idesc_bf16_f32(128, 128, false, true, false);  // [K;Q] x [W | S]
+  constexpr uint32_t ID_CORR = idesc_f16_f32(128, 64, false, true, true);   // P -= A' x (eta G)
   constexpr uint32_t ID_DW = idesc_f16_f32(128, 64, true, true, false);     // [K'^T;K'^T] x (eta G)
 
   uint32_t kr[8], vr[8];
@@ -285,25 +295,19 @@ __global__ void __launch_bounds__(THREADS, 2)
     }
     um = quad_sum(um) * (1.f / D);
   };
-  // rho X + kappa Y - Corr of this thread's K (which = 0) or Q (which = 1) row of
-  // the 16-lane block i; the correction is absent before the first update.
-  auto combine_rows = [&](int i, int which, float rho, float kap, bool corr, float2 (&y)[8]) {
-    float2 x[8], yy[8];
-    tmem_rows_16x256b(tmem_addr(tX, 32 * warp + 16 * i, 0), which, x);
-    tmem_rows_16x256b(tmem_addr(tY, 32 * warp + 16 * i, 0), which, yy);
-    const float2 r2 = make_float2(rho, rho), k2 = make_float2(kap, kap);
-#pragma unroll
-    for (int j = 0; j < 8; ++j) y[j] = __ffma2_rn(k2, yy[j], __fmul2_rn(r2, x[j]));
-    if (corr) {
-      float2 cr[8];
-      tmem_rows_16x256b(tmem_addr(tC, 32 * warp + 16 * i, 0), which, cr);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) y[j] = fsub2(y[j], cr[j]);
-    }
+  // P = rho X + kappa Y - corrections of this thread's K (which = 0) or Q (which = 1)
+  // row of the 16-lane block i.
+  auto read_p = [&](int i, int which, float2 (&y)[8]) {
+    tmem_rows_16x256b(tmem_addr(tX, 32 * warp + 16 * i, 0), which, y);
   };
 
-  // Chunk head: wait for the tiles, issue S, X, Y; the coefficient arrays (warp 2);
-  // the coefficient-weighted Gram into the fp16 A operand (every thread its row).
+  // The Q residuals of this thread's two output rows (read at the chunk head, so
+  // that the next chunk's Q tile can load under the chain).
+  uint32_t qres[2][8];
+
+  // Chunk head: wait for the tiles; issue S, X, Y; the prefix scans (warp 2) and the
+  // coefficient table (warp 3); every thread's row of the coefficient-weighted Gram
+  // (the fp16 A operand) and of P = rho X + kappa Y; the Q residuals.
   auto chunk_head = [&](int c) {
     const int ntok = chunk_tokens(c);
     const uint32_t par = (uint32_t)c & 1u;
@@ -318,13 +322,13 @@ __global__ void __launch_bounds__(THREADS, 2)
         umma_ss_w(tS, smem_desc_sw128(aA + 32 * k, 16, 1024), smem_desc_sw128(aA + 32 * k, 16, 2048), ID_S,
                   k > 0);
       umma_commit_w(&bars[BAR_S]);
+      // X | Y = [K;Q] [W | S] as N = 128 products into adjacent accumulators: the
+      // W and S operands are the two 64-column atoms of B, 16 KB apart (lbo).
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const uint64_t ak = smem_desc_sw128(aA + 32 * k, 16, 1024);
-        umma_ss_w(tX, ak, smem_desc_sw128(aWhi + 2048 * k, 8192, 1024), ID_P, k > 0);
-        umma_ss_w(tX, ak, smem_desc_sw128(aWlo + 2048 * k, 8192, 1024), ID_P, true);
-        umma_ss_w(tY, ak, smem_desc_sw128(aShi + 2048 * k, 8192, 1024), ID_P, k > 0);
-        umma_ss_w(tY, ak, smem_desc_sw128(aSlo + 2048 * k, 8192, 1024), ID_P, true);
+        umma_ss_w(tX, ak, smem_desc_sw128(aWhi + 2048 * k, OFF_SHI - OFF_WHI, 1024), ID_P2, k > 0);
+        umma_ss_w(tX, ak, smem_desc_sw128(aWlo + 2048 * k, OFF_SLO - OFF_WLO, 1024), ID_P2, true);
       }
       umma_commit_w(&bars[BAR_P]);
       __syncwarp();
@@ -335,77 +339,29 @@ __global__ void __launch_bounds__(THREADS, 2)
         *reinterpret_cast<uint32_t *>(sm + OFF_G + sw128_offset(row, col)) = 0u;
       }
     }
+    const int L = ntok - 1;  // the chunk's last token
     if (warp == 2) {
-      // Lam, A, C (forward scans) and c_{L,.}, a_{L,.} (backward scans from the
-      // last token L); absent tokens act as identities.
-      const int L = ntok - 1;
-      float dl[2], el[2], da[2], ea[2];
+      // Lam_t = prod (1 - lambda), A_t = prod alpha and C_t = (1 - lambda_t) C_{t-1} + A_t;
+      // absent tokens of a ragged chunk act as identities.
+      float dl[2], da[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int t = lane + 32 * h;
         const bool in = t < ntok;
         dl[h] = in ? 1.f - lam_s[t] : 1.f;
-        el[h] = 0.f;
         da[h] = in ? alpha_s[t] : 1.f;
-        ea[h] = 0.f;
       }
-      // Products: x_t = d_t x_{t-1} with x_{-1} = 1 is the scan's d.
+      // A product x_t = d_t x_{t-1} (x_{-1} = 1) is the scan's composed d.
       float pl[2] = {dl[0], dl[1]}, pa[2] = {da[0], da[1]};
-      {
-        float d1[2] = {dl[0], dl[1]}, e1[2] = {0.f, 0.f};
-        affine_scan64(d1, e1, lane);
-        pl[0] = d1[0];
-        pl[1] = d1[1];
-        float d2[2] = {da[0], da[1]}, e2[2] = {0.f, 0.f};
-        affine_scan64(d2, e2, lane);
-        pa[0] = d2[0];
-        pa[1] = d2[1];
-      }
-      // C_t = (1 - lambda_t) C_{t-1} + A_t.
+      float e0[2] = {0.f, 0.f}, e1[2] = {0.f, 0.f};
+      affine_scan64(pl, e0, lane);
+      affine_scan64(pa, e1, lane);
       float dc[2] = {dl[0], dl[1]}, ec[2] = {pa[0], pa[1]};
       affine_scan64(dc, ec, lane);
-      // Backward from L over tokens s = L - r (r = lane + 32 h): a_{L,s} = prod_{s < r' <= L} alpha,
-      // c_{L,s} = D_{L,s} + alpha_{s+1} c_{L,s+1}, D_{L,s} = prod_{s < v <= L} (1 - lambda_v):
-      // the step from s + 1 to s multiplies by alpha_{s+1} (a, c) and (1 - lambda_{s+1}) (D).
-      float db[2], eb[2], dd[2], ed[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int s = L - (lane + 32 * h);
-        const bool step = s >= 0 && s < L;  // s = L starts the walk (identity)
-        db[h] = step ? alpha_s[s + 1] : 1.f;
-        eb[h] = 0.f;
-        dd[h] = step ? 1.f - lam_s[s + 1] : 1.f;
-        ed[h] = 0.f;
-      }
-      float aw[2], dw[2];
-      {
-        float d1[2] = {db[0], db[1]}, e1[2] = {0.f, 0.f};
-        affine_scan64(d1, e1, lane);
-        aw[0] = d1[0];
-        aw[1] = d1[1];
-        float d2[2] = {dd[0], dd[1]}, e2[2] = {0.f, 0.f};
-        affine_scan64(d2, e2, lane);
-        dw[0] = d2[0];
-        dw[1] = d2[1];
-      }
-      // c_{L,s} = alpha_{s+1} c_{L,s+1} + D_{L,s}, c_{L,L} = 1 (= D_{L,L}).
-      float dcw[2], ecw[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        dcw[h] = db[h];
-        ecw[h] = dw[h];
-      }
-      affine_scan64(dcw, ecw, lane);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int t = lane + 32 * h;
-        PL[t] = pl[h];
-        CC[t] = ec[h];
-        const int s = L - t;
-        if (s >= 0) {
-          AW[s] = aw[h];
-          CW[s] = ecw[h];
-        }
+        PL[lane + 32 * h] = pl[h];
+        CC[lane + 32 * h] = ec[h];
       }
       if (lane == (L & 31)) {  // the lane that holds token L in half L / 32
         const int h = L >> 5;
@@ -413,58 +369,121 @@ __global__ void __launch_bounds__(THREADS, 2)
         FIN[1] = ec[h];
         FIN[2] = pa[h];
       }
+    } else if (warp == 3) {
+      // The coefficient table, column sigma walked up from tau = sigma:
+      // a_{tau,sigma} = alpha_tau a_{tau-1,sigma}, c_{tau,sigma} = (1 - lambda_tau)
+      // c_{tau-1,sigma} + a_{tau,sigma}, both 1 at tau = sigma and 0 above the
+      // diagonal.  Lane l walks columns l and 63 - l (65 steps each lane); the row
+      // tau = L is c_{L,.} and a_{L,.} of the state update.  Both start at 0 and the
+      // step a = alpha a + [tau = sigma] gives the 1 on the diagonal.  alpha and
+      // lambda are read four tokens at a time, a group ahead (ntok is a multiple of
+      // 16), so that no read waits behind the table's stores.
+      const int s0 = lane, s1 = CHUNK - 1 - lane;
+      float a0 = 0.f, c0 = 0.f, a1 = 0.f, c1 = 0.f;
+      auto step = [&](int t, float al, float la) {
+        const float om = 1.f - la;
+        a0 = fmaf(al, a0, t == s0 ? 1.f : 0.f);
+        c0 = fmaf(om, c0, a0);
+        a1 = fmaf(al, a1, t == s1 ? 1.f : 0.f);
+        c1 = fmaf(om, c1, a1);
+        COEF[t * COEF_LD + s0] = c0;
+        COEF[t * COEF_LD + s1] = c1;
+      };
+      float4 al4 = *reinterpret_cast<const float4 *>(alpha_s);
+      float4 la4 = *reinterpret_cast<const float4 *>(lam_s);
+      for (int t = 0; t < ntok; t += 4) {
+        const float4 al = al4, la = la4;
+        if (t + 4 < ntok) {
+          al4 = *reinterpret_cast<const float4 *>(alpha_s + t + 4);
+          la4 = *reinterpret_cast<const float4 *>(lam_s + t + 4);
+        }
+        step(t, al.x, la.x);
+        step(t + 1, al.y, la.y);
+        step(t + 2, al.z, la.z);
+        step(t + 3, al.w, la.w);
+      }
+      CW[s0] = c0;
+      AW[s0] = a0;
+      CW[s1] = c1;
+      AW[s1] = a1;
     }
-    wait_or_abort(&bars[BAR_S], par, abort);
-    tc_fence_after_sync();
-    __syncwarp();
+    __syncthreads();  // coefficients, Lam, C visible
     {
       // This thread's row of [K;Q]: group 4 warp + lane / 8.  Its coefficient row
       // tau*: 16 m - 1 for a K row of mini-batch m (none for m = 0), its token for
-      // a Q row; column sigma gets c_{tau*,sigma} S for sigma <= tau*, else 0.
+      // a Q row (none for an absent token of a ragged chunk); column sigma gets
+      // c_{tau*,sigma} S (0 above the diagonal).
       const bool qrow = (lane >> 3) & 1;
       const int mrow = mb0 + (lane >> 4);
       const int t = MB * mrow + 8 * hh + (lane & 7);
-      // (Rows of absent tokens in a ragged last chunk get none: their alpha and
-      // lambda were not loaded.)
       const int tstar = t >= ntok ? -1 : (qrow ? t : MB * mrow - 1);
-      float cco = 0.f, dco = 1.f;  // c_{tau*,sigma} and D_{tau*,sigma} of the walk
-      // Blocks from the last to the first (the walk goes down sigma); each block is
-      // read from S columns 8j.. and 32+8j.. and written back as fp16 over the first.
+      const float *crow = COEF + (tstar < 0 ? 0 : tstar) * COEF_LD;
+      wait_or_abort(&bars[BAR_S], par, abort);
+      tc_fence_after_sync();
+      __syncwarp();
+      // Block j: tokens 16 j .. 16 j + 15 in S columns 8 j .. (the first eight) and
+      // 32 + 8 j .. (the second), written back as fp16 pairs over the first.
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int j = 3 - jj;
+      for (int j = 0; j < 4; ++j) {
         uint32_t pk[8];
         if (j <= mb0 + 1) {
           uint32_t v0[8], v1[8];
           tmem_ld_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), v0);
           tmem_ld_32x32b_x8(tmem_addr(tS, 32 * warp, 32 + 8 * j), v1);
-          tmem_wait_ld();
-          float a[16];
+          float cf[16];
 #pragma unroll
-          for (int ee = 0; ee < 16; ++ee) {
-            const int e = 15 - ee;
-            const int s = MB * j + e;
-            const uint32_t bits = e < 8 ? v0[e] : v1[e - 8];
-            if (s == tstar) {
-              cco = 1.f;
-              dco = 1.f;
-            } else if (s < tstar) {
-              dco *= 1.f - lam_s[s + 1];
-              cco = fmaf(alpha_s[s + 1], cco, dco);
-            }
-            a[e] = s <= tstar ? cco * __uint_as_float(bits) : 0.f;
+          for (int q = 0; q < 4; ++q) {
+            const float4 c4 = *reinterpret_cast<const float4 *>(crow + MB * j + 4 * q);
+            cf[4 * q] = c4.x;
+            cf[4 * q + 1] = c4.y;
+            cf[4 * q + 2] = c4.z;
+            cf[4 * q + 3] = c4.w;
           }
+          tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) pk[e] = pack_f16x2(a[2 * e], a[2 * e + 1]);
+          for (int e = 0; e < 8; ++e) {
+            const float x0 = tstar < 0 ? 0.f : cf[2 * e] * __uint_as_float(2 * e < 8 ? v0[2 * e] : v1[2 * e - 8]);
+            const float x1 =
+                tstar < 0 ? 0.f : cf[2 * e + 1] * __uint_as_float(2 * e + 1 < 8 ? v0[2 * e + 1] : v1[2 * e - 7]);
+            pk[e] = pack_f16x2(x0, x1);
+          }
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) pk[e] = 0u;
         }
         tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), pk);
       }
+      // P = rho X + kappa Y over this thread's row: (Lam, C) at the row's base,
+      // token 16 m - 1 for a K row of mini-batch m (Lam = 1, C = 0 for m = 0), the
+      // row's own token for a Q row.
+      const int tb_row = qrow ? t : MB * mrow - 1;
+      const float rho = tb_row < 0 ? 1.f : PL[tb_row], kap = tb_row < 0 ? 0.f : CC[tb_row];
+      wait_or_abort(&bars[BAR_P], par, abort);
+      tc_fence_after_sync();
+      __syncwarp();
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t xr[16], yr[16];
+        tmem_ld_32x32b_x16(tmem_addr(tX, 32 * warp, 16 * q), xr);
+        tmem_ld_32x32b_x16(tmem_addr(tY, 32 * warp, 16 * q), yr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          xr[e] = __float_as_uint(fmaf(kap, __uint_as_float(yr[e]), rho * __uint_as_float(xr[e])));
+        tmem_st_32x32b_x16(tmem_addr(tX, 32 * warp, 16 * q), xr);
+      }
       tmem_wait_st();
     }
+    // Every MMA that reads this chunk's Q tile is complete (BAR_S, BAR_P): this
+    // warp takes its residuals and loads its part of the next chunk's Q.
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        qres[i][j] = lds_u32(sbase + kq_offset(MB * (mb0 + i) + 8 * hh + fr, 1, 8 * j + 2 * q4));
     fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -479,21 +498,37 @@ __global__ void __launch_bounds__(THREADS, 2)
     const uint32_t par = (uint32_t)c & 1u;
 
     // ---- the chain: mini-batch m on warps m/2 and 2 + m/2 ------------------------
+    // (u of the warp's second mini-batch first: it would otherwise sit between the
+    // two updates.)
+    float2 u1[8];
+    float um1 = 0.f;
+    if (mb0 + 1 < nmb) {
+      load_kv(MB * (mb0 + 1) + 8 * hh + fr);
+      make_u();
+#pragma unroll
+      for (int j = 0; j < 8; ++j) u1[j] = u[j];
+      um1 = um;
+    }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int m = mb0 + i;
       if (m >= nmb) break;
       const int tk = MB * m + 8 * hh + fr;
       const float e0 = eta_s[tk];
-      const float rho = m == 0 ? 1.f : PL[MB * m - 1], kap = m == 0 ? 0.f : CC[MB * m - 1];
       const float cwk = CW[tk], awk = AW[tk];
       load_kv(tk);
-      make_u();
+      if (i == 0) {
+        make_u();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) u[j] = u1[j];
+        um = um1;
+      }
       wait_or_abort(&bars[m == 0 ? BAR_P : BAR_C0 + m - 1], par, abort);
       tc_fence_after_sync();
       __syncwarp();
       float2 y[8];
-      combine_rows(i, 0, rho, kap, m > 0, y);
+      read_p(i, 0, y);
       // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y (as in the
       // linear kernel: one reduction round for the mean, one for four sums).
       const float mean = quad_sum(sum8(y)) * (1.f / D);
@@ -539,23 +574,33 @@ __global__ void __launch_bounds__(THREADS, 2)
       if (hh == 0) {
         __syncwarp();
         tc_fence_after_sync();
-        umma_ts_w(tC, tS + 8 * m, smem_desc_sw128(aG + 2048 * m, 8192, 1024), ID_CORR, m > 0);
+        umma_ts_w(tX, tS + 8 * m, smem_desc_sw128(aG + 2048 * m, 8192, 1024), ID_CORR, true);
         umma_commit_w(&bars[m == nmb - 1 ? BAR_LAST : BAR_C0 + m]);
+        if (m == nmb - 1) {
+          // Every eta G row and weighted K row of the chunk is written (each step's
+          // writers fenced them before the barrier that its issue followed): the
+          // state update's MMAs go now, under the last outputs.  dW = (c-weighted
+          // K)^T (eta G): the K rows of groups 4k, 4k + 2 read twice (lbo 0) against
+          // the eta G rows of the same tokens (two 8-row groups 2 KB apart); dS =
+          // (a-weighted K, natural order in the V buffer)^T (eta G).
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t gk = 4096u * (k & 1) + 1024u * (k >> 1);
+            umma_ss_w(tC, smem_desc_sw128(aA + 4096 * k, 0, 2048), smem_desc_sw128(aG + gk, 8192, 2048), ID_DW,
+                      k > 0);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_ss_w(tY, smem_desc_sw128(aV + 2048 * k, 0, 1024), smem_desc_sw128(aG + 2048 * k, 8192, 1024),
+                      ID_DW, k > 0);
+          umma_commit_w(&bars[BAR_DW]);
+        }
         __syncwarp();
       }
     }
 
     // ---- outputs of this warp's Q rows (final once their mini-batch's update is in)
     float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
-    uint32_t qres[2][8];
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        qres[i][j] = lds_u32(sbase + kq_offset(MB * (mb0 + i) + 8 * hh + fr, 1, 8 * j + 2 * q4));
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int m = mb0 + i;
@@ -565,7 +610,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       tc_fence_after_sync();
       __syncwarp();
       float2 z[8];
-      combine_rows(i, 1, PL[tq], CC[tq], true, z);
+      read_p(i, 1, z);
       const float mean = quad_sum(sum8(z)) * (1.f / D);
       const float2 nm = make_float2(-mean, -mean);
       float2 qa = make_float2(0.f, 0.f), qb = qa;
@@ -589,29 +634,7 @@ __global__ void __launch_bounds__(THREADS, 2)
       }
     }
 
-    // ---- the end-of-chunk state: X, Y are free once every output is read ----------
-    tc_fence_before_sync();
-    __syncthreads();
-    tc_fence_after_sync();
-    if (warp == 0) {
-      __syncwarp();
-      // dW = (c-weighted K)^T (eta G) into X: the K rows of groups 4k, 4k + 2 read
-      // twice (lbo 0) against the eta*G rows of the same tokens (two 8-row groups
-      // 2 KB apart); dS = (a-weighted K, natural order in the V buffer)^T (eta G)
-      // into Y.
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t gk = 4096u * (k & 1) + 1024u * (k >> 1);
-        umma_ss_w(tX, smem_desc_sw128(aA + 4096 * k, 0, 2048), smem_desc_sw128(aG + gk, 8192, 2048), ID_DW,
-                  k > 0);
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        umma_ss_w(tY, smem_desc_sw128(aV + 2048 * k, 0, 1024), smem_desc_sw128(aG + 2048 * k, 8192, 1024), ID_DW,
-                  k > 0);
-      umma_commit_w(&bars[BAR_DW]);
-      __syncwarp();
-    }
+    // ---- the end-of-chunk state --------------------------------------------------
     wait_or_abort(&bars[BAR_DW], par, abort);
     tc_fence_after_sync();
     __syncwarp();
@@ -621,7 +644,7 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t dw[16], ds[16];
-        tmem_ld_32x32b_x16(tmem_addr(tX, 32 * warp, wc0 + 16 * h), dw);
+        tmem_ld_32x32b_x16(tmem_addr(tC, 32 * warp, wc0 + 16 * h), dw);
         tmem_ld_32x32b_x16(tmem_addr(tY, 32 * warp, wc0 + 16 * h), ds);
         tmem_wait_ld();
 #pragma unroll
