@@ -577,7 +577,9 @@ def run_backward_mlp(args):
 def run_momentum(args):
     """The momentum and decay forward's own line: one step = one launch of
     ttt_linear_ln_momentum_fwd over the linear + LN workload (B=16 H=32 T=8192, b=16),
-    or (``--workload mlp_B8H32T8192``) of ttt_mlp_momentum_fwd over the TTT-MLP one."""
+    or (``--workload mlp_B8H32T8192``) of ttt_mlp_momentum_fwd over the TTT-MLP one.
+    TTT-Linear + LN runs the tensor-core dual form by default (bf16 operands, fp32
+    accumulation) and the exact-fp32 register-state kernel with ``--path simt``."""
     if args.workload.startswith("mlp"):
         return run_momentum_mlp(args)
     import torch
@@ -597,6 +599,7 @@ def run_momentum(args):
     W_out, S_out = torch.empty(B, H, d, d, device=dev), torch.empty(B, H, d, d, device=dev)
     stream = torch.cuda.current_stream(dev)
     lib = _lib.load()
+    ttt.set_path({"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT, "tc": ttt.TTT_PATH_TC}[args.path])
 
     def step():
         ttt.ttt_linear_momentum_fwd(qkv["Q"], qkv["K"], qkv["V"], eta, alpha, lam, W0, b, gamma=gamma,
@@ -625,15 +628,17 @@ def run_momentum(args):
     nbytes = units * (T * (3 * d * 2 + 3 * 4 + d * 4) + 3 * d * d * 4)
     peaks, peak_kind = load_peaks()
     achieved = nbytes / (ms / 1e3) / 1e9
+    full = args.path != "simt" and (B, T) == (16, 8192)
+    traffic = committed_traffic("momentum_" + cfg.name) if full else None
     line = {
         "metric": "TTT-Linear+LN momentum/decay forward tokens/s (B x H x T / s)",
         "value": units * T / (ms / 1e3), "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f32" if args.path == "simt" else "bf16", "data": "synthetic",
         "config": {"workload": "momentum_" + cfg.name, "B": B, "H": H, "T": T, "d": d, "b": b,
-                   "qkv_dtype": "bf16", "l2": "inputs larger than L2 (no flush needed)"},
+                   "qkv_dtype": "bf16", "path": args.path, "l2": "inputs larger than L2 (no flush needed)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json)", "algorithmic_bytes_per_launch": nbytes},
         "clocks": clock_info, "gpu_launches": int(launches),
     }

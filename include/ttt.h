@@ -175,8 +175,13 @@ TTT_API int ttt_fwd_host(int variant, const void *Q, const void *K, const void *
  * Inputs as for the forward, plus alpha, lambda [B][H][T] fp32 (per token, like
  * eta).  Outputs: Z [B][H][T][d], W_out and S_out [B][H][d][d] (the final state
  * and momentum), fp32.  1 <= b <= 16 and d = 64 (else TTT_ERR_UNSUPPORTED),
- * T % b == 0.  alpha = lambda = 0 is the plain TTT forward.  Errors as for the
- * forward entry points.
+ * T % b == 0.  alpha = lambda = 0 is the plain TTT forward.  Arithmetic: with
+ * LN, bf16 Q, K, V and b = 16, the dual form over 64-token chunks on the tensor
+ * cores (the recursion unrolled into per-token decay coefficients; W and S as
+ * bf16 hi + lo operands, the coefficient-weighted Gram, eta G and K as fp16, fp32
+ * accumulation: about 3e-4 relative to an fp64 evaluation), unless
+ * ttt_set_path(TTT_PATH_SIMT); every other case, fp32 on the CUDA cores.  Errors
+ * as for the forward entry points.
  */
 TTT_API int ttt_linear_momentum_fwd(const void *Q, const void *K, const void *V, int qkv_dtype,
                                     const float *eta, const float *alpha, const float *lambda,
@@ -397,8 +402,11 @@ TTT_API int ttt_last_device_status(void *stream);
  * Kernel path selection for the next calls from any thread: TTT_PATH_AUTO
  * (default: tensor cores where supported), TTT_PATH_SIMT (exact-fp32 CUDA-core
  * kernels for every case) or TTT_PATH_TC (tensor cores; calls outside the
- * tensor-core sizes return TTT_ERR_UNSUPPORTED).  Returns the previous path, or
- * TTT_ERR_ARG for an unknown value.
+ * tensor-core sizes return TTT_ERR_UNSUPPORTED).  It applies to the entry points
+ * that have a tensor-core kernel: ttt_linear_fwd, ttt_linear_ln_fwd, ttt_mlp_fwd
+ * (and ttt_fwd_host) and ttt_linear_momentum_fwd / ttt_linear_ln_momentum_fwd;
+ * the others run their CUDA-core kernels under every path.  Returns the previous
+ * path, or TTT_ERR_ARG for an unknown value.
  */
 typedef enum { TTT_PATH_AUTO = 0, TTT_PATH_SIMT = 1, TTT_PATH_TC = 2 } ttt_path;
 TTT_API int ttt_set_path(int path);

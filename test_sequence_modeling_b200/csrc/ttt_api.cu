@@ -591,7 +591,10 @@ int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int q
   const bool bf16 = qkv_dtype == TTT_BF16;
   // TTT-Linear + LN with bf16 inputs and b = 16: the tensor-core dual form (unless
   // the CUDA-core path is selected).
-  if (ln && bf16 && b == tcmom::MB && T > 0 && g_path.load() != TTT_PATH_SIMT) {
+  const int path = g_path.load();
+  const bool tc_ok = ln && bf16 && b == tcmom::MB;
+  if (path == TTT_PATH_TC && !tc_ok) return TTT_ERR_UNSUPPORTED;
+  if (tc_ok && T > 0 && path != TTT_PATH_SIMT) {
     CUtensorMap mq, mk, mv;
     if (!make_qkv_map(&mq, Q, T, units, 8) || !make_qkv_map(&mk, K, T, units, 8) ||
         !make_qkv_map(&mv, V, T, units, tcmom::CHUNK))

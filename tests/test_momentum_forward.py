@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import test_sequence_modeling_b200 as ttt
-from test_sequence_modeling_b200 import inputs as I
+from test_sequence_modeling_b200 import _lib, inputs as I
 from gpu_helpers import rel_fro, to_device
 
 pytestmark = pytest.mark.gpu
@@ -206,3 +206,19 @@ def test_tc_momentum_bounded_wait_expiry_is_reported_and_recoverable():
     out = run_gpu(cfg, dev, a, l_, ttt.TTT_PATH_TC)
     worst = worst_error(cfg, out, alpha, lam, [(0, 0), (1, 2)])
     assert max(worst.values()) <= TC_REGRESSION, worst
+
+
+def test_tc_path_rejects_cases_without_a_tensor_core_kernel():
+    """Under TTT_PATH_TC a case the dual form does not take (fp32 inputs) is refused,
+    as for the plain forwards; AUTO runs it on the CUDA cores."""
+    cfg = I.CONFIGS["linear_f32_B1H1T256"].replace(B=1, H=2, T=32, b=16)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    alpha, lam = (torch.from_numpy(x).cuda() for x in I.momentum_rates(cfg))
+    prev = ttt.set_path(ttt.TTT_PATH_TC)
+    try:
+        with pytest.raises(ttt.TTTError) as e:
+            ttt.ttt_linear_momentum_fwd(dev["Q"], dev["K"], dev["V"], dev["eta"], alpha, lam, dev["W0"], cfg.b)
+        assert e.value.status == _lib.TTT_ERR_UNSUPPORTED
+    finally:
+        ttt.set_path(prev)
+    run_gpu(cfg, dev, alpha, lam, ttt.TTT_PATH_AUTO)
