@@ -104,11 +104,12 @@ def test_momentum_forward_agrees_with_the_decode_steps():
     torch.testing.assert_close(S, Sd, rtol=1e-6, atol=1e-7)
 
 
-def test_momentum_forward_empty_sequence():
+@pytest.mark.parametrize("path", [ttt.TTT_PATH_SIMT, ttt.TTT_PATH_AUTO])
+def test_momentum_forward_empty_sequence(path):
     cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=2, H=2, T=0)
     dev = to_device(cfg, I.make_inputs(cfg))
     e = torch.empty(2, 2, 0, device="cuda")
-    Z, W, S = run_gpu(cfg, dev, e, e)
+    Z, W, S = run_gpu(cfg, dev, e, e, path)
     assert Z.numel() == 0
     assert torch.equal(W, dev["W0"].unsqueeze(0).expand(2, 2, 64, 64))
     assert torch.all(S == 0)
@@ -222,3 +223,32 @@ def test_tc_path_rejects_cases_without_a_tensor_core_kernel():
     finally:
         ttt.set_path(prev)
     run_gpu(cfg, dev, alpha, lam, ttt.TTT_PATH_AUTO)
+
+
+def test_tc_momentum_forward_is_deterministic_and_stays_in_bounds():
+    """Two runs agree bit for bit, and outputs carved from one larger buffer leave the
+    guard bytes around them untouched (ragged last chunk: T = 208)."""
+    cfg, dev, alpha, lam = tc_case(208)
+    a, l_ = torch.from_numpy(alpha).cuda(), torch.from_numpy(lam).cuda()
+    nz = cfg.B * cfg.H * cfg.T * cfg.d
+    nw = cfg.B * cfg.H * cfg.d * cfg.d
+    outs = []
+    for _ in range(2):
+        buf = torch.full((nz + 2 * nw + 4 * 1024,), 7.0, device="cuda")
+        Z = buf[1024:1024 + nz].view(cfg.B, cfg.H, cfg.T, cfg.d)
+        W = buf[2048 + nz:2048 + nz + nw].view(cfg.B, cfg.H, cfg.d, cfg.d)
+        S = buf[3072 + nz + nw:3072 + nz + 2 * nw].view(cfg.B, cfg.H, cfg.d, cfg.d)
+        prev = ttt.set_path(ttt.TTT_PATH_TC)
+        try:
+            ttt.ttt_linear_momentum_fwd(dev["Q"], dev["K"], dev["V"], dev["eta"], a, l_, dev["W0"], cfg.b,
+                                        gamma=dev["gamma"], beta=dev["beta"], eps=cfg.ln_eps, Z=Z, W_out=W,
+                                        S_out=S)
+            torch.cuda.synchronize()
+        finally:
+            ttt.set_path(prev)
+        assert ttt.last_device_status() == 0
+        h = buf.cpu().numpy()
+        assert np.all(h[:1024] == 7.0) and np.all(h[1024 + nz:2048 + nz] == 7.0)
+        assert np.all(h[2048 + nz + nw:3072 + nz + nw] == 7.0) and np.all(h[3072 + nz + 2 * nw:] == 7.0)
+        outs.append(h)
+    assert np.array_equal(outs[0], outs[1])
