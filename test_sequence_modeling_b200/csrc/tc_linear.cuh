@@ -160,8 +160,11 @@ __device__ __forceinline__ void wait_or_abort(uint64_t *bar, uint32_t parity, vo
   }
 }
 
-template <bool LN>
-__global__ void __launch_bounds__(THREADS, 4)
+// MINB = 4: <= 128 registers, so that 4 CTAs share an SM (a grid of up to 592
+// units in one wave); MINB = 2: the register budget of 2 CTAs per SM, for grids
+// that leave SMs to spare (the launch picks by wave count).
+template <bool LN, int MINB = 4>
+__global__ void __launch_bounds__(THREADS, MINB)
     linear_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const Params p) {
