@@ -68,6 +68,9 @@ constexpr int D = 64;
 constexpr int CHUNK = 64;  // tokens per chunk (4 mini-batches of 16)
 constexpr int MB = 16;     // mini-batch size of this kernel
 constexpr int THREADS = 128;
+// Hardware named barriers (0 is __syncthreads): 1 and 2 pair the two warps of a
+// chain step; NB_STATE_BACK gathers every warp's state back from TMEM before dW.
+constexpr uint32_t NB_STATE_BACK = 3;
 constexpr uint32_t TMEM_COLS = 128;
 
 // Shared-memory map (bytes from a 1024-byte aligned base).
@@ -392,6 +395,18 @@ __global__ void __launch_bounds__(THREADS, MINB)
         }
         tmem_st_32x32b_x8(tmem_addr(tS, 32 * warp, 8 * j), pk);
       }
+      // The fp32 state waits out the chain in this thread's TMEM lane, S columns
+      // 32-63 (free from here until dW), so that its 32 registers serve the chain.
+      {
+        uint32_t w0r[16], w1r[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          w0r[e] = __float_as_uint(wm[e]);
+          w1r[e] = __float_as_uint(wm[16 + e]);
+        }
+        tmem_st_32x32b_x16(tmem_addr(tS, 32 * warp, 32), w0r);
+        tmem_st_32x32b_x16(tmem_addr(tS, 32 * warp, 48), w1r);
+      }
       tmem_wait_st();
     }
     fence_proxy_async_smem();
@@ -487,6 +502,21 @@ __global__ void __launch_bounds__(THREADS, MINB)
       }
     }
 
+    // The state back from TMEM; warps 1-3 count themselves toward the named
+    // barrier NB_STATE_BACK, which warp 0 waits on before dW overwrites those columns.
+    {
+      uint32_t r0[16], r1[16];
+      tmem_ld_32x32b_x16(tmem_addr(tS, 32 * warp, 32), r0);
+      tmem_ld_32x32b_x16(tmem_addr(tS, 32 * warp, 48), r1);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        wm[e] = __uint_as_float(r0[e]);
+        wm[16 + e] = __uint_as_float(r1[e]);
+      }
+      tc_fence_before_sync();
+      if (warp != 0) named_barrier_arrive(NB_STATE_BACK, THREADS);
+    }
     // Outputs of this warp's Q rows: after their mini-batch's update they are
     // final (later updates add exactly zero to them, A being zero there).
     float *Zc = p.Z + (tok_base + (size_t)c * CHUNK) * D;
@@ -545,6 +575,8 @@ __global__ void __launch_bounds__(THREADS, MINB)
     wait_or_abort(&bars[BAR_LAST], par, abort);
     tc_fence_after_sync();
     if (warp == 0) {
+      named_barrier_sync(NB_STATE_BACK, THREADS);  // every warp has its state back
+      tc_fence_after_sync();
       __syncwarp();
       // dW = K^T (eta G) into the S columns (their operand is consumed).  Step k
       // takes the K rows of groups 4k and 4k + 2 (tokens of mini-batches
