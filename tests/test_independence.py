@@ -40,18 +40,17 @@ def test_cuda_sources_and_oracle_share_no_includes():
         assert not inc.startswith(("cuda", "ttt.h")) and not inc.endswith(".cuh"), inc
 
 
-def test_nothing_reads_the_reference_pages():
-    """No product file, bench.py or the entry points names the location of the
-    reference pages (taken from the workload description beside the repository)."""
-    import json
-    desc = os.path.join(ROOT, "BASELINE.json")
-    ref = json.load(open(desc)).get("reference_path") if os.path.exists(desc) else None
-    if not ref:
-        pytest.skip("no reference location recorded")
+def test_nothing_reads_files_outside_the_repository():
+    """No product file, bench.py or the entry points names an absolute filesystem
+    path (a quoted string starting with '/'): everything they read lives in the
+    repository, so nothing reads the reference pages or any other outside file."""
     files = _product_modules() + [os.path.join(ROOT, "bench.py"), os.path.join(ROOT, "__graft_entry__.py")]
     files += [os.path.join(CSRC, f) for f in os.listdir(CSRC)]
+    files += [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))]
+    pattern = re.compile(r"""["'](/[A-Za-z_][^"'\n]*)["']""")
     for path in files:
-        assert ref not in open(path).read(), path
+        found = pattern.findall(open(path).read())
+        assert not found, (path, found)
 
 
 def test_missing_library_raises():
