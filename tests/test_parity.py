@@ -149,6 +149,24 @@ def test_tensor_core_ragged_chunks(variant, T):
     assert max(worst.values()) <= TOL[cfg.dtype], (variant, T, worst)
 
 
+def test_bounded_wait_expiry_on_the_four_cta_kernel():
+    """A grid that the launch runs on the 4-CTA-per-SM register budget (more units
+    than 2 per SM hold): expiry reported, context usable, next call exact."""
+    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=10, H=32, T=128)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    ttt.set_path(ttt.TTT_PATH_TC)
+    ttt.debug_inject_timeout(True)
+    try:
+        run_gpu(cfg, dev)
+        assert ttt.last_device_status() == ttt.TTT_ERR_TIMEOUT
+    finally:
+        ttt.debug_inject_timeout(False)
+    out = run_gpu(cfg, dev)
+    assert ttt.last_device_status() == 0
+    worst = compare(cfg, out, sample_units(cfg, 6))
+    assert max(worst.values()) <= REGRESSION[cfg.name], worst
+
+
 # Agreement of the tensor-core path with the exact-fp32 CUDA-core path: fp16
 # chain and update operands (11-bit significand) for TTT-Linear, tf32 and fp16
 # operands for TTT-MLP, both far below the oracle tolerance.
