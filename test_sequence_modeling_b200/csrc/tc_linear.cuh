@@ -6,7 +6,8 @@
 // (§03.5).
 //
 // Work decomposition.  One CTA of 4 warps owns one (batch, head) sequence for
-// its whole length and keeps the fp32 state W in registers.  Tokens are taken
+// its whole length and keeps the fp32 state W in registers (in TMEM while the
+// chain of a chunk runs, step 3 to 5).  Tokens are taken
 // in chunks of 64 (four mini-batches), so that every tensor-core product has
 // M = 128 rows: the 64 K rows and the 64 Q rows of the chunk.  With W_c the
 // state at the start of the chunk and G_m the gradient of the loss w.r.t. the
@@ -31,7 +32,9 @@
 //   2. tcgen05: S = [K;Q] K^T (TMEM cols 64..127) and P = [K;Q] W_c (cols 0..63).
 //   3. Every thread masks its own row of S in TMEM, in place, into the fp16 A
 //      operand of step 4: K rows keep the columns of earlier mini-batches, Q
-//      rows keep s <= t (the causal mask of the dual form, diagonal included).
+//      rows keep s <= t (the causal mask of the dual form, diagonal included);
+//      it then parks its 32 state elements in its lane's S columns 96..127,
+//      free until dW, and takes them back after its chain steps.
 //   4. For m = 0..3, the two warps that hold mini-batch m read its K rows of P
 //      (already corrected for mini-batches < m), compute G_m (LN backward in
 //      registers, 16 elements per thread), write eta*G_m as fp16, turn their K
@@ -49,7 +52,7 @@
 // Precision: W enters P = [K;Q] W as a bf16 pair hi + lo (~2^-16 relative) against
 // the exact bf16 K and Q; the masked Q K^T, eta*G and K enter the chain's
 // corrections and dW as fp16 (2^-11 relative); accumulation is fp32 and the
-// state stays fp32 in registers.
+// state stays fp32.
 #pragma once
 
 #include <cuda.h>
