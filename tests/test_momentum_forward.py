@@ -252,3 +252,14 @@ def test_tc_momentum_forward_is_deterministic_and_stays_in_bounds():
         assert np.all(h[2048 + nz + nw:3072 + nz + nw] == 7.0) and np.all(h[3072 + nz + 2 * nw:] == 7.0)
         outs.append(h)
     assert np.array_equal(outs[0], outs[1])
+
+
+def test_tc_momentum_forward_long_sequence():
+    """512 chunks (T = 32768): no drift of the dual form's error along the sequence."""
+    cfg = I.CONFIGS["linear_ln_B1H32T32768"].replace(H=2)
+    dev = to_device(cfg, I.make_inputs(cfg))
+    alpha, lam = I.momentum_rates(cfg)
+    out = run_gpu(cfg, dev, torch.from_numpy(alpha).cuda(), torch.from_numpy(lam).cuda(), ttt.TTT_PATH_TC)
+    worst = worst_error(cfg, out, alpha, lam, [(0, 0), (0, 1)])
+    print(f"tensor-core momentum T=32768: {worst}")
+    assert max(worst.values()) <= TC_REGRESSION, worst
