@@ -577,9 +577,11 @@ def run_backward_mlp(args):
 def run_momentum(args):
     """The momentum and decay forward's own line: one step = one launch of
     ttt_linear_ln_momentum_fwd over the linear + LN workload (B=16 H=32 T=8192, b=16),
-    or (``--workload mlp_B8H32T8192``) of ttt_mlp_momentum_fwd over the TTT-MLP one.
-    TTT-Linear + LN runs the tensor-core dual form by default (bf16 operands, fp32
-    accumulation) and the exact-fp32 register-state kernel with ``--path simt``."""
+    of ttt_linear_momentum_fwd over another bf16 TTT-Linear (+ LN) workload named by
+    ``--workload``, or (``--workload mlp_B8H32T8192``) of ttt_mlp_momentum_fwd over the
+    TTT-MLP one.  TTT-Linear (+ LN) runs the tensor-core dual form by default (bf16
+    operands, fp32 accumulation) and the exact-fp32 register-state kernel with
+    ``--path simt``."""
     if args.workload.startswith("mlp"):
         return run_momentum_mlp(args)
     import torch
@@ -587,13 +589,18 @@ def run_momentum(args):
     from test_sequence_modeling_b200 import _lib
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
-    cfg = I.CONFIGS["linear_ln_B16H32T8192"]
-    cfg = cfg.replace(B=args.batch or cfg.B, T=args.seq or cfg.T)  # smaller profiling cases
+    base = I.CONFIGS[args.workload]
+    if base.dtype != "bf16" or base.variant not in ("linear", "linear_ln"):
+        raise SystemExit(f"--momentum takes a bf16 TTT-Linear (+ LN) or the TTT-MLP workload, not {args.workload}")
+    cfg = base.replace(B=args.batch or base.B, T=args.seq or base.T)  # smaller profiling cases
+    ln = cfg.variant == "linear_ln"
     data = I.make_inputs(cfg)
     B, H, T, d, b = cfg.B, cfg.H, cfg.T, cfg.d, cfg.b
     qkv = {k: torch.from_numpy(data[k].view(np.int16)).to(dev).view(torch.bfloat16) for k in "QKV"}
     eta = torch.from_numpy(np.ascontiguousarray(data["eta"])).to(dev)
-    W0, gamma, beta = (torch.from_numpy(data[k]).to(dev) for k in ("W0", "gamma", "beta"))
+    W0 = torch.from_numpy(data["W0"]).to(dev)
+    ln_kw = dict(gamma=torch.from_numpy(data["gamma"]).to(dev), beta=torch.from_numpy(data["beta"]).to(dev),
+                 eps=cfg.ln_eps) if ln else {}
     alpha, lam = (torch.from_numpy(x).to(dev) for x in I.momentum_rates(cfg))
     Z = torch.empty(B, H, T, d, device=dev)
     W_out, S_out = torch.empty(B, H, d, d, device=dev), torch.empty(B, H, d, d, device=dev)
@@ -602,8 +609,8 @@ def run_momentum(args):
     ttt.set_path({"auto": ttt.TTT_PATH_AUTO, "simt": ttt.TTT_PATH_SIMT, "tc": ttt.TTT_PATH_TC}[args.path])
 
     def step():
-        ttt.ttt_linear_momentum_fwd(qkv["Q"], qkv["K"], qkv["V"], eta, alpha, lam, W0, b, gamma=gamma,
-                                    beta=beta, eps=cfg.ln_eps, Z=Z, W_out=W_out, S_out=S_out, stream=stream)
+        ttt.ttt_linear_momentum_fwd(qkv["Q"], qkv["K"], qkv["V"], eta, alpha, lam, W0, b, Z=Z, W_out=W_out,
+                                    S_out=S_out, stream=stream, **ln_kw)
 
     for _ in range(max(args.warmup, 0)):
         step()
@@ -628,10 +635,10 @@ def run_momentum(args):
     nbytes = units * (T * (3 * d * 2 + 3 * 4 + d * 4) + 3 * d * d * 4)
     peaks, peak_kind = load_peaks()
     achieved = nbytes / (ms / 1e3) / 1e9
-    full = args.path != "simt" and (B, T) == (16, 8192)
+    full = args.path != "simt" and (B, T) == (base.B, base.T)
     traffic = committed_traffic("momentum_" + cfg.name) if full else None
     line = {
-        "metric": "TTT-Linear+LN momentum/decay forward tokens/s (B x H x T / s)",
+        "metric": ("TTT-Linear+LN" if ln else "TTT-Linear") + " momentum/decay forward tokens/s (B x H x T / s)",
         "value": units * T / (ms / 1e3), "unit": "head-tokens/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32" if args.path == "simt" else "bf16", "data": "synthetic",

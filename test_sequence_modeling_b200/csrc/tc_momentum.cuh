@@ -1,5 +1,5 @@
-// tc_momentum.cuh - tensor-core (tcgen05) forward of TTT-Linear + LN with the
-// momentum and decay update of the Titans article (§二.1(2): momentum on past
+// tc_momentum.cuh - tensor-core (tcgen05) forward of TTT-Linear and TTT-Linear +
+// LN with the momentum and decay update of the Titans article (§二.1(2): momentum on past
 // surprise, a forget gate that decays the memory), kept to the TTT mini-batch
 // rule (§03.6: every gradient of a mini-batch taken at its base state), for bf16
 // Q, K, V, d = 64, b = 16.
@@ -140,6 +140,7 @@ __device__ __forceinline__ void affine_scan64(float (&d)[2], float (&e)[2], int 
   d[1] = td * d[1];
 }
 
+template <bool LN>
 __global__ void __launch_bounds__(THREADS, 2)
     momentum_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -183,8 +184,8 @@ __global__ void __launch_bounds__(THREADS, 2)
     tmem_relinquish();
   }
   if (tid < D) {
-    const float g = p.gamma[head * D + tid];
-    const float b = p.beta[head * D + tid];
+    const float g = LN ? p.gamma[head * D + tid] : 1.f;
+    const float b = LN ? p.beta[head * D + tid] : 0.f;
     float *gb = reinterpret_cast<float *>(sm + OFF_GB + 16 * (tid >> 1)) + (tid & 1);
     float *uc = reinterpret_cast<float *>(sm + OFF_UC + 16 * (tid >> 1)) + (tid & 1);
     gb[0] = g;
@@ -289,11 +290,15 @@ __global__ void __launch_bounds__(THREADS, 2)
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const float2 v = unpack_bf16x2(vr[j]);
-      const float4 c = *reinterpret_cast<const float4 *>(sm + OFF_UC + 16 * (4 * j + q4));
-      u[j] = __ffma2_rn(make_float2(c.x, c.y), fsub2(unpack_bf16x2(kr[j]), v), make_float2(c.z, c.w));
-      um += u[j].x + u[j].y;
+      if (LN) {
+        const float4 c = *reinterpret_cast<const float4 *>(sm + OFF_UC + 16 * (4 * j + q4));
+        u[j] = __ffma2_rn(make_float2(c.x, c.y), fsub2(unpack_bf16x2(kr[j]), v), make_float2(c.z, c.w));
+        um += u[j].x + u[j].y;
+      } else {
+        u[j] = v;  // the plain model's target
+      }
     }
-    um = quad_sum(um) * (1.f / D);
+    if (LN) um = quad_sum(um) * (1.f / D);
   };
   // P = rho X + kappa Y - corrections of this thread's K (which = 0) or Q (which = 1)
   // row of the 16-lane block i.
@@ -475,12 +480,14 @@ __global__ void __launch_bounds__(THREADS, 2)
       tmem_wait_st();
     }
     // Every MMA that reads this chunk's Q tile is complete (BAR_S, BAR_P): this
-    // warp takes its residuals and loads its part of the next chunk's Q.
+    // warp takes its residuals (with LN) and loads its part of the next chunk's Q.
+    if (LN) {
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+      for (int i = 0; i < 2; ++i)
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        qres[i][j] = lds_u32(sbase + kq_offset(MB * (mb0 + i) + 8 * hh + fr, 1, 8 * j + 2 * q4));
+        for (int j = 0; j < 8; ++j)
+          qres[i][j] = lds_u32(sbase + kq_offset(MB * (mb0 + i) + 8 * hh + fr, 1, 8 * j + 2 * q4));
+    }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0 && c + 1 < nchunks && !*abort) issue_load_q(c + 1);
@@ -529,34 +536,44 @@ __global__ void __launch_bounds__(THREADS, 2)
       __syncwarp();
       float2 y[8];
       read_p(i, 0, y);
-      // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y (as in the
-      // linear kernel: one reduction round for the mean, one for four sums).
-      const float mean = quad_sum(sum8(y)) * (1.f / D);
-      const float2 nm = make_float2(-mean, -mean);
-      float2 w2[8];
-      float2 sdd = make_float2(0.f, 0.f), swd = sdd, swdd = sdd, sud = sdd;
+      if (!LN) {
+        // dl/dy = 2 (y - v)
+        const float2 f = make_float2(2.f * e0, 2.f * e0);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        w2[j] = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
-        y[j] = __fadd2_rn(y[j], nm);
-        const float2 t = __fmul2_rn(w2[j], y[j]);
-        swd = __fadd2_rn(swd, t);
-        swdd = __ffma2_rn(t, y[j], swdd);
-        sdd = __ffma2_rn(y[j], y[j], sdd);
-        sud = __ffma2_rn(u[j], y[j], sud);
-      }
-      const float vdd = quad_sum(sdd.x + sdd.y), vwd = quad_sum(swd.x + swd.y);
-      const float vwdd = quad_sum(swdd.x + swdd.y), vud = quad_sum(sud.x + sud.y);
-      const float r = rsqrtf(vdd * (1.f / D) + p.eps);
-      const float A = um + r * vwd * (1.f / D);
-      const float B = (r * vud + r * r * vwdd) * (1.f / D);
-      const float2 f = make_float2(e0 * r, e0 * r), rr = make_float2(r, r);
-      const float2 nA = make_float2(-A, -A), nB = make_float2(-B, -B);
+        for (int j = 0; j < 8; ++j) {
+          const float2 g = __fmul2_rn(f, fsub2(y[j], u[j]));
+          *reinterpret_cast<uint32_t *>(sm + OFF_G + sw128_offset(tk, 8 * j + 2 * q4)) = pack_f16x2(g.x, g.y);
+        }
+      } else {
+        // LN backward of ||k + gamma xhat + beta - v||^2 w.r.t. y (as in the
+        // linear kernel: one reduction round for the mean, one for four sums).
+        const float mean = quad_sum(sum8(y)) * (1.f / D);
+        const float2 nm = make_float2(-mean, -mean);
+        float2 w2[8];
+        float2 sdd = make_float2(0.f, 0.f), swd = sdd, swdd = sdd, sud = sdd;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float2 xh = __fmul2_rn(y[j], rr);
-        const float2 g = __fmul2_rn(f, __fadd2_rn(__ffma2_rn(xh, __fadd2_rn(w2[j], nB), u[j]), nA));
-        *reinterpret_cast<uint32_t *>(sm + OFF_G + sw128_offset(tk, 8 * j + 2 * q4)) = pack_f16x2(g.x, g.y);
+        for (int j = 0; j < 8; ++j) {
+          w2[j] = *reinterpret_cast<const float2 *>(sm + OFF_W2 + 4 * (8 * j + 2 * q4));
+          y[j] = __fadd2_rn(y[j], nm);
+          const float2 t = __fmul2_rn(w2[j], y[j]);
+          swd = __fadd2_rn(swd, t);
+          swdd = __ffma2_rn(t, y[j], swdd);
+          sdd = __ffma2_rn(y[j], y[j], sdd);
+          sud = __ffma2_rn(u[j], y[j], sud);
+        }
+        const float vdd = quad_sum(sdd.x + sdd.y), vwd = quad_sum(swd.x + swd.y);
+        const float vwdd = quad_sum(swdd.x + swdd.y), vud = quad_sum(sud.x + sud.y);
+        const float r = rsqrtf(vdd * (1.f / D) + p.eps);
+        const float A = um + r * vwd * (1.f / D);
+        const float B = (r * vud + r * r * vwdd) * (1.f / D);
+        const float2 f = make_float2(e0 * r, e0 * r), rr = make_float2(r, r);
+        const float2 nA = make_float2(-A, -A), nB = make_float2(-B, -B);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 xh = __fmul2_rn(y[j], rr);
+          const float2 g = __fmul2_rn(f, __fadd2_rn(__ffma2_rn(xh, __fadd2_rn(w2[j], nB), u[j]), nA));
+          *reinterpret_cast<uint32_t *>(sm + OFF_G + sw128_offset(tk, 8 * j + 2 * q4)) = pack_f16x2(g.x, g.y);
+        }
       }
       // The weighted K rows of the end-of-chunk update, fp16: c_{L,.} k in place
       // of K (X, Y and S, its bf16 readers, are complete), a_{L,.} k over the V
@@ -611,26 +628,31 @@ __global__ void __launch_bounds__(THREADS, 2)
       __syncwarp();
       float2 z[8];
       read_p(i, 1, z);
-      const float mean = quad_sum(sum8(z)) * (1.f / D);
-      const float2 nm = make_float2(-mean, -mean);
-      float2 qa = make_float2(0.f, 0.f), qb = qa;
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        z[j] = __fadd2_rn(z[j], nm);
-        z[j + 1] = __fadd2_rn(z[j + 1], nm);
-        qa = __ffma2_rn(z[j], z[j], qa);
-        qb = __ffma2_rn(z[j + 1], z[j + 1], qb);
-      }
-      const float rstd = rsqrtf(quad_sum((qa.x + qb.x) + (qa.y + qb.y)) * (1.f / D) + p.eps);
-      const float2 rs = make_float2(rstd, rstd);
       float *zrow = Zc + tq * D;
+      if (!LN) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = 8 * j + 2 * q4;
-        const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_GB + 16 * (4 * j + q4));
-        const float2 q = unpack_bf16x2(qres[i][j]);
-        *reinterpret_cast<float2 *>(zrow + col) =
-            __fadd2_rn(q, __ffma2_rn(make_float2(gb.x, gb.y), __fmul2_rn(z[j], rs), make_float2(gb.z, gb.w)));
+        for (int j = 0; j < 8; ++j) *reinterpret_cast<float2 *>(zrow + 8 * j + 2 * q4) = z[j];
+      } else {
+        const float mean = quad_sum(sum8(z)) * (1.f / D);
+        const float2 nm = make_float2(-mean, -mean);
+        float2 qa = make_float2(0.f, 0.f), qb = qa;
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+          z[j] = __fadd2_rn(z[j], nm);
+          z[j + 1] = __fadd2_rn(z[j + 1], nm);
+          qa = __ffma2_rn(z[j], z[j], qa);
+          qb = __ffma2_rn(z[j + 1], z[j + 1], qb);
+        }
+        const float rstd = rsqrtf(quad_sum((qa.x + qb.x) + (qa.y + qb.y)) * (1.f / D) + p.eps);
+        const float2 rs = make_float2(rstd, rstd);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int col = 8 * j + 2 * q4;
+          const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_GB + 16 * (4 * j + q4));
+          const float2 q = unpack_bf16x2(qres[i][j]);
+          *reinterpret_cast<float2 *>(zrow + col) =
+              __fadd2_rn(q, __ffma2_rn(make_float2(gb.x, gb.y), __fmul2_rn(z[j], rs), make_float2(gb.z, gb.w)));
+        }
       }
     }
 

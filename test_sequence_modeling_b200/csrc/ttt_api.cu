@@ -621,10 +621,10 @@ int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int q
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const unsigned grid = (unsigned)units;
   const bool bf16 = qkv_dtype == TTT_BF16;
-  // TTT-Linear + LN with bf16 inputs and b = 16: the tensor-core dual form (unless
-  // the CUDA-core path is selected).
+  // bf16 inputs and b = 16: the tensor-core dual form (unless the CUDA-core path
+  // is selected).
   const int path = g_path.load();
-  const bool tc_ok = ln && bf16 && b == tcmom::MB;
+  const bool tc_ok = bf16 && b == tcmom::MB;
   if (path == TTT_PATH_TC && !tc_ok) return TTT_ERR_UNSUPPORTED;
   if (tc_ok && T > 0 && path != TTT_PATH_SIMT) {
     CUtensorMap mq, mk, mv;
@@ -632,12 +632,13 @@ int run_momentum_fwd(bool ln, const void *Q, const void *K, const void *V, int q
         !make_qkv_map(&mv, V, T, units, tcmom::CHUNK))
       return TTT_ERR_CUDA;
     tcmom::Params tp{eta, alpha, lambda, W0, gamma, beta, eps, H, T, Z, W_out, S_out, g_inject_timeout.load()};
-    if (cudaFuncSetAttribute(tcmom::momentum_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)tcmom::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(tcmom::momentum_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+    auto kernel = ln ? tcmom::momentum_tc_kernel<true> : tcmom::momentum_tc_kernel<false>;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tcmom::SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return TTT_ERR_CUDA;
-    tcmom::momentum_tc_kernel<<<grid, tcmom::THREADS, tcmom::SMEM_BYTES, s>>>(mq, mk, mv, tp);
+    kernel<<<grid, tcmom::THREADS, tcmom::SMEM_BYTES, s>>>(mq, mk, mv, tp);
     if (cudaGetLastError() != cudaSuccess) return TTT_ERR_CUDA;
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return TTT_OK;

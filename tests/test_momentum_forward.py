@@ -137,26 +137,32 @@ def test_momentum_forward_full_size_sampled_units():
 
 # ---- the tensor-core dual form ------------------------------------------------------
 
-def tc_case(T, B=2, H=3):
-    cfg = I.CONFIGS["linear_ln_B16H32T8192"].replace(B=B, H=H, T=T, b=16)
+TC_NAMES = ["linear_ln_B16H32T8192", "linear_bf16_B16H12T2048"]
+
+
+def tc_case(T, B=2, H=3, name="linear_ln_B16H32T8192"):
+    cfg = I.CONFIGS[name].replace(B=B, H=H, T=T, b=16)
     dev = to_device(cfg, I.make_inputs(cfg))
     alpha, lam = I.momentum_rates(cfg)
     return cfg, dev, alpha, lam
 
 
 @pytest.mark.parametrize("T", [16, 48, 64, 128, 208])
-def test_tc_momentum_forward_matches_oracle(T):
-    """Every unit, one to four chunks, ragged last chunks (T % 64 != 0)."""
-    cfg, dev, alpha, lam = tc_case(T)
+@pytest.mark.parametrize("name", TC_NAMES)
+def test_tc_momentum_forward_matches_oracle(name, T):
+    """Every unit, one to four chunks, ragged last chunks (T % 64 != 0); TTT-Linear
+    with and without LN."""
+    cfg, dev, alpha, lam = tc_case(T, name=name)
     out = run_gpu(cfg, dev, torch.from_numpy(alpha).cuda(), torch.from_numpy(lam).cuda(), ttt.TTT_PATH_TC)
     worst = worst_error(cfg, out, alpha, lam, [(b, h) for b in range(cfg.B) for h in range(cfg.H)])
-    print(f"tensor-core momentum T={T}: {worst}")
+    print(f"tensor-core momentum {cfg.variant} T={T}: {worst}")
     assert max(worst.values()) <= TC_REGRESSION, worst
 
 
-def test_tc_momentum_forward_agrees_with_cuda_core_path():
+@pytest.mark.parametrize("name", TC_NAMES)
+def test_tc_momentum_forward_agrees_with_cuda_core_path(name):
     """The two CUDA paths on the same inputs, far below the oracle tolerance."""
-    cfg, dev, alpha, lam = tc_case(512, B=2, H=4)
+    cfg, dev, alpha, lam = tc_case(512, B=2, H=4, name=name)
     a, l_ = torch.from_numpy(alpha).cuda(), torch.from_numpy(lam).cuda()
     tc = [x.cpu().numpy() for x in run_gpu(cfg, dev, a, l_, ttt.TTT_PATH_TC)]
     cc = [x.cpu().numpy() for x in run_gpu(cfg, dev, a, l_, ttt.TTT_PATH_SIMT)]
@@ -164,29 +170,35 @@ def test_tc_momentum_forward_agrees_with_cuda_core_path():
         assert rel_fro(x, y) < TC_REGRESSION
 
 
-def test_tc_momentum_without_momentum_or_decay_is_ttt():
+@pytest.mark.parametrize("name", TC_NAMES)
+def test_tc_momentum_without_momentum_or_decay_is_ttt(name):
     """alpha = lambda = 0 makes the dual form's coefficients the causal mask: the
-    TTT-Linear + LN tensor-core forward's outputs, and S_T = -eta_T g_T."""
-    cfg, dev, _, _ = tc_case(256)
+    TTT-Linear (+ LN) tensor-core forward's outputs, and S_T = -eta_T g_T."""
+    cfg, dev, _, _ = tc_case(256, name=name)
     z = torch.zeros(cfg.B, cfg.H, cfg.T, device="cuda")
     Z, W, S = run_gpu(cfg, dev, z, z, ttt.TTT_PATH_TC)
-    Zt, Wt = ttt.ttt_linear_ln_fwd(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], dev["gamma"],
-                                   dev["beta"], cfg.b, cfg.ln_eps)
+    if cfg.variant == "linear_ln":
+        Zt, Wt = ttt.ttt_linear_ln_fwd(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], dev["gamma"],
+                                       dev["beta"], cfg.b, cfg.ln_eps)
+    else:
+        Zt, Wt = ttt.ttt_linear_fwd(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], cfg.b)
     torch.cuda.synchronize()
     assert rel_fro(Z.cpu().numpy(), Zt.cpu().numpy()) < 1e-4
     assert rel_fro(W.cpu().numpy(), Wt.cpu().numpy()) < 1e-4
     assert torch.isfinite(S).all() and S.abs().max() > 0
 
 
-def test_tc_momentum_forward_full_size_sampled_units():
-    """The full linear + LN workload (B16 H32 T8192), first and last units."""
-    cfg = I.CONFIGS["linear_ln_B16H32T8192"]
+@pytest.mark.parametrize("name", TC_NAMES)
+def test_tc_momentum_forward_full_size_sampled_units(name):
+    """The full workload (linear + LN B16 H32 T8192, linear B16 H12 T2048), first and
+    last units."""
+    cfg = I.CONFIGS[name]
     dev = to_device(cfg, I.make_inputs(cfg))
     alpha, lam = I.momentum_rates(cfg)
     out = run_gpu(cfg, dev, torch.from_numpy(alpha).cuda(), torch.from_numpy(lam).cuda(), ttt.TTT_PATH_AUTO)
     assert all(bool(torch.isfinite(x).all()) for x in out)
     worst = worst_error(cfg, out, alpha, lam, [(0, 0), (cfg.B - 1, cfg.H - 1)])
-    print(f"tensor-core momentum full size: {worst}")
+    print(f"tensor-core momentum full size {name}: {worst}")
     assert max(worst.values()) <= TC_REGRESSION, worst
 
 
