@@ -176,7 +176,7 @@ TTT_API int ttt_fwd_host(int variant, const void *Q, const void *K, const void *
  * eta).  Outputs: Z [B][H][T][d], W_out and S_out [B][H][d][d] (the final state
  * and momentum), fp32.  1 <= b <= 16 and d = 64 (else TTT_ERR_UNSUPPORTED),
  * T % b == 0.  alpha = lambda = 0 is the plain TTT forward.  Arithmetic: with
- * LN, bf16 Q, K, V and b = 16, the dual form over 64-token chunks on the tensor
+ * bf16 Q, K, V and b = 16, the dual form over 64-token chunks on the tensor
  * cores (the recursion unrolled into per-token decay coefficients; W and S as
  * bf16 hi + lo operands, the coefficient-weighted Gram, eta G and K as fp16, fp32
  * accumulation: about 3e-4 relative to an fp64 evaluation), unless
