@@ -437,6 +437,18 @@ __global__ void __launch_bounds__(THREADS, MINB)
       // in flight.
       load_kv(tk);
       make_u();
+      // This thread's K row elements become fp16 in place (the dW operand); P and
+      // S, the bf16 readers, are complete.  Under the 4-CTA register cap this is
+      // done before the wait, so that the K elements are not held through the LN
+      // backward.
+      auto k_to_f16 = [&]() {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float2 k2 = unpack_bf16x2(kr[j]);
+          *reinterpret_cast<uint32_t *>(sm + kq_offset(tk, 0, 8 * j + 2 * q4)) = pack_f16x2(k2.x, k2.y);
+        }
+      };
+      if (MINB == 4) k_to_f16();
       wait_or_abort(&bars[m == 0 ? BAR_P : BAR_C0 + m - 1], par, abort);
       tc_fence_after_sync();
       __syncwarp();
@@ -485,13 +497,7 @@ __global__ void __launch_bounds__(THREADS, MINB)
           store_grad(8 * j + 2 * q4, __fmul2_rn(f, __fadd2_rn(__ffma2_rn(xh, __fadd2_rn(w2[j], nB), u[j]), nA)));
         }
       }
-      // This thread's K row elements become fp16 in place (the dW operand); P and
-      // S, the bf16 readers, are complete.
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float2 k2 = unpack_bf16x2(kr[j]);
-        *reinterpret_cast<uint32_t *>(sm + kq_offset(tk, 0, 8 * j + 2 * q4)) = pack_f16x2(k2.x, k2.y);
-      }
+      if (MINB != 4) k_to_f16();
       // Both halves of eta*G_m written: the pair's first warp issues the update.
       fence_proxy_async_smem();
       tc_fence_before_sync();
