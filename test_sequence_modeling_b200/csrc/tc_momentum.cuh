@@ -1,8 +1,8 @@
 // tc_momentum.cuh - tensor-core (tcgen05) forward of TTT-Linear and TTT-Linear +
-// LN with the momentum and decay update of the Titans article (§二.1(2): momentum on past
-// surprise, a forget gate that decays the memory), kept to the TTT mini-batch
-// rule (§03.6: every gradient of a mini-batch taken at its base state), for bf16
-// Q, K, V, d = 64, b = 16.
+// LN with the momentum and decay update of the Titans article (§二.1(2): momentum
+// on past surprise, a forget gate that decays the memory), kept to the TTT
+// mini-batch rule (§03.6: every gradient of a mini-batch taken at its base
+// state), for bf16 Q, K, V, d = 64, b = 16.
 //
 // Per token t, with g_t = k_t^T G_t the loss gradient at the base of t's
 // mini-batch:  S_t = alpha_t S_{t-1} - eta_t g_t,  W_t = (1 - lambda_t) W_{t-1} + S_t.
@@ -108,7 +108,7 @@ enum {
 struct Params {
   const float *eta, *alpha, *lambda;  // [units][T]
   const float *W0;                    // [H][D][D]
-  const float *gamma, *beta;          // [H][D]
+  const float *gamma, *beta;          // [H][D] (with LN only)
   float eps;
   int H, T;
   float *Z;                           // [units][T][D]
