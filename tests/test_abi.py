@@ -306,6 +306,21 @@ def test_momentum_forward_argument_errors(lib, ln):
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
 
 
+@pytest.mark.parametrize("ln", [False, True])
+def test_momentum_forward_tensor_core_path_refuses_other_cases(lib, ln):
+    """Under TTT_PATH_TC a well-formed call the dual form does not take (fp32 inputs,
+    b < 16) is refused on the host, before any CUDA call (fake pointers)."""
+    n0 = lib.ttt_launch_count()
+    prev = lib.ttt_set_path(L.TTT_PATH_TC)
+    try:
+        assert momentum_fwd(lib, ln, dt=L.TTT_F32) == L.TTT_ERR_UNSUPPORTED
+        assert momentum_fwd(lib, ln, b=8) == L.TTT_ERR_UNSUPPORTED
+        assert momentum_fwd(lib, ln, T=36, b=8) == L.TTT_ERR_ARG  # argument errors come first
+    finally:
+        lib.ttt_set_path(prev)
+    assert lib.ttt_launch_count() == n0, "a refused call launched a kernel"
+
+
 def test_noalloc_backward_checks_sizes_before_any_cuda_call(lib):
     """ttt_linear_ln_bwd_noalloc rejects a call whose states exceed its built-in
     array, and malformed sizes, on the host (fake pointers are never touched)."""
