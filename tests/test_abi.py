@@ -99,6 +99,21 @@ def test_argument_errors(lib, fn):
     assert lib.ttt_launch_count() == n0, "a rejected call launched a kernel"
 
 
+@pytest.mark.parametrize("fn", [linear, ln, mlp])
+def test_tensor_core_path_refuses_cases_it_has_no_kernel_for(lib, fn):
+    """Under TTT_PATH_TC a well-formed forward the tensor cores do not take (fp32
+    inputs; b != 16) is refused on the host, before any CUDA call."""
+    n0 = lib.ttt_launch_count()
+    prev = lib.ttt_set_path(L.TTT_PATH_TC)
+    try:
+        assert fn(lib, dt=L.TTT_F32) == L.TTT_ERR_UNSUPPORTED
+        assert fn(lib, b=8) == L.TTT_ERR_UNSUPPORTED
+        assert fn(lib, B=0) == L.TTT_OK  # empty: nothing to do on any path
+    finally:
+        lib.ttt_set_path(prev)
+    assert lib.ttt_launch_count() == n0, "a refused call launched a kernel"
+
+
 def test_ln_specific_errors(lib):
     assert ln(lib, eps=0.0) == L.TTT_ERR_ARG
     assert ln(lib, eps=float("nan")) == L.TTT_ERR_ARG
